@@ -1,0 +1,397 @@
+"""Benchmark of the CSA2 decode hot path on synthetic inputs shaped like the pages' workloads.
+
+Workload (one step): decode of B = 32 queries at 131,072 compressed entries
+(m = 1) through one CSA2 group, 1 Full layer + 3 Reuse layers: the Full layer
+appends the new token (NVFP4 latent + FP4 indexer K), quantises its indexer
+query, scores every entry and keeps the Top-512; all four layers run sparse
+attention (Top-512 FP4 rows + their own 128-token FP8 window) with their own
+16-head queries.  Inputs are resident in HBM when timing starts; L2 is flushed
+(256 MiB write) between timed steps, outside the per-step events.
+
+`python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]`
+prints one JSON line (rank 0).  Under torchrun every rank runs its own replica
+(weak scaling: the batch is independent per rank; no collective on the data
+path) and `value` is N * 32 / (max over ranks of the per-step time).
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "CSA2 decode queries/s @128K ctx; index+attn HBM GB/s and % of B200 roofline"
+B, N_CTX, T_SWA, TOPK, LAYERS = 32, 131072, 128, 512, ["full", "reuse", "reuse", "reuse"]
+WORKLOAD = "c1: decode, B=32, 131,072 entries, m=1, 1 Full + 3 Reuse, Top-512, SWA-128"
+
+# algorithmic bytes (each byte the method must move once)
+IDX_BYTES_PER_ENTRY = 36                         # 32 B FP4 indexer K + 4 B E4M3 scales
+ROW_BYTES = 288                                  # 256 B FP4 latent + 32 B scales
+SWA_BYTES = 516                                  # 512 B FP8 + 4 B fp32 scale
+Q_OUT_BYTES = 2 * 16 * 512 * 2                   # bf16 query in + bf16 output
+IDX_LIST_BYTES = TOPK * 4
+INDEX_LAUNCH_BYTES = B * N_CTX * IDX_BYTES_PER_ENTRY + B * (128 + 16 + 16) + B * TOPK * 4
+ATTN_LAYER_BYTES = B * (TOPK * ROW_BYTES + T_SWA * SWA_BYTES + Q_OUT_BYTES + IDX_LIST_BYTES)
+STEP_BYTES = B * N_CTX * IDX_BYTES_PER_ENTRY + len(LAYERS) * ATTN_LAYER_BYTES
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def _kernel_hash():
+    h = hashlib.sha256()
+    for f in ("index.cu", "topk.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "sparse_attention_fp4_quant_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _ncu_traffic():
+    """DRAM bytes per launch of the index kernel from the committed ncu summary, if it
+    was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "index_topk_decode_b32_131k.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        if d.get("kernel_hash") == _kernel_hash():
+            return float(d["dram_bytes_per_launch"])
+    except (OSError, ValueError, KeyError):
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of the SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index, self.rows, self.proc = index, [], None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 6:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[2 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# ------------------------------------------------------------------ our arm
+class DecodeGroup:
+    """Device state and per-step inputs of the config-1 workload on one GPU."""
+
+    def __init__(self, csa, seed, device):
+        self.csa = csa
+        self.device = device
+        self.kv = csa.KV(B, N_CTX, 1, device)
+        self.W = synth.proj_w(seed).to(device)
+        # context: N_CTX - 1 cached entries; the step appends the new token at N_CTX - 1
+        for b in range(B):
+            lat = synth.latent(synth.seed_of("bench-ctx", seed, b), N_CTX - 1, 0, device)
+            csa.csa2_quant_nvfp4(lat, self.kv.lat[b].view(-1, 256), self.kv.lat_sc[b].view(-1, 32))
+            csa.csa2_index_k_proj(lat, self.W, self.kv.ik[b].view(-1, 32), self.kv.ik_sc[b].view(-1, 4))
+            del lat
+        self.kv.n_entries.fill_(N_CTX)
+        self.new_lat = torch.stack([synth.latent(synth.seed_of("bench-new", seed, b), 1, N_CTX - 1, device)[0]
+                                    for b in range(B)])
+        self.new_rows = (torch.arange(B, device=device, dtype=torch.int64) * N_CTX + (N_CTX - 1))
+        self.iq_bf = synth.index_q(synth.seed_of("bench-iq", seed), B, 1, device)
+        self.w = synth.index_w(B, 1, device)
+        self.q_pos = torch.full((B, 1), N_CTX - 1, dtype=torch.int32, device=device)
+        self.q = [synth.attn_q(synth.seed_of("bench-q", seed, li), B, 1, device) for li in range(len(LAYERS))]
+        self.swa = []
+        for li in range(len(LAYERS)):
+            cs = [synth.swa_kv(synth.seed_of("bench-swa", seed, li, b), T_SWA, N_CTX - T_SWA, device) for b in range(B)]
+            self.swa.append((torch.stack([c[0] for c in cs]), torch.stack([c[1] for c in cs])))
+        self.swa_pos0 = torch.full((B,), N_CTX - T_SWA, dtype=torch.int32, device=device)
+        self.iq = torch.empty((B, 1, 128), dtype=torch.uint8, device=device)
+        self.iqs = torch.empty((B, 1, 16), dtype=torch.uint8, device=device)
+        self.idx = torch.empty((B, 1, TOPK), dtype=torch.int32, device=device)
+        self.out = [torch.empty((B, 1, 16, 512), dtype=torch.bfloat16, device=device) for _ in LAYERS]
+        nbytes = max(csa.csa2_workspace_bytes(csa.OP_INDEX_TOPK, B, 1, N_CTX, TOPK),
+                     csa.csa2_workspace_bytes(csa.OP_SPARSE_ATTN, B, 1, N_CTX, TOPK))
+        self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+    # the three segments of a step (each is captured into its own CUDA graph)
+    def front(self):
+        c = self.csa
+        c.csa2_quant_nvfp4(self.new_lat, self.kv.lat.view(-1, 256), self.kv.lat_sc.view(-1, 32), self.new_rows)
+        c.csa2_index_k_proj(self.new_lat, self.W, self.kv.ik.view(-1, 32), self.kv.ik_sc.view(-1, 4), self.new_rows)
+        c.csa2_quant_nvfp4(self.iq_bf.view(-1, 64), self.iq.view(-1, 32), self.iqs.view(-1, 4))
+
+    def index(self):
+        self.csa.csa2_index_topk(self.iq, self.iqs, self.w, self.kv, self.q_pos, TOPK, self.idx, ws=self.ws)
+
+    def attention(self):
+        for li in range(len(LAYERS)):
+            swa, swa_sc = self.swa[li]
+            self.csa.csa2_sparse_attn(self.q[li], self.kv, self.idx, swa, swa_sc, self.swa_pos0, self.q_pos,
+                                      out=self.out[li], ws=self.ws)
+
+    LAUNCHES_PER_STEP = 3 + 1 + len(LAYERS)
+
+
+def _graph(fn):
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # warm (first-call attributes) outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def _oracle_baseline(seconds_target=12.0, max_reps=64):
+    """The oracle (single-threaded C) on a bounded sample of the same workload:
+    one batch row at the full 131,072-entry context, the whole step repeated."""
+    import oracle
+    seed = 9
+    lat = synth.latent(synth.seed_of("bench-ctx", seed, 0), N_CTX, 0, "cpu")
+    lb = synth.bf16_bits(lat)
+    W = synth.proj_w(seed).numpy()
+    t0 = time.perf_counter()
+    olat, olsc = oracle.quant_nvfp4(lb)
+    oik, oiks = oracle.index_k_proj(lb, W)
+    setup_s = time.perf_counter() - t0
+    olat, olsc = olat.reshape(1, N_CTX, 256), olsc.reshape(1, N_CTX, 32)
+    oik, oiks = oik.reshape(1, N_CTX, 32), oiks.reshape(1, N_CTX, 4)
+    new_lb = lb[-1:].copy()
+    iq = synth.bf16_bits(synth.index_q(synth.seed_of("bench-iq", seed), 1, 1, "cpu")).reshape(-1, 64)
+    w = synth.index_w(1, 1).numpy()
+    q_pos = np.array([[N_CTX - 1]], np.int32)
+    qs = [synth.bf16_bits(synth.attn_q(synth.seed_of("bench-q", seed, li), 1, 1)) for li in range(len(LAYERS))]
+    swas = [synth.swa_kv(synth.seed_of("bench-swa", seed, li, 0), T_SWA, N_CTX - T_SWA) for li in range(len(LAYERS))]
+    swas = [(c.numpy()[None], s.numpy()[None]) for c, s in swas]
+    ne = np.array([N_CTX], np.int32)
+    pos0 = np.array([N_CTX - T_SWA], np.int32)
+
+    def step():
+        a, b_ = oracle.quant_nvfp4(new_lb)
+        olat[0, -1], olsc[0, -1] = a[0], b_[0]
+        c_, d_ = oracle.index_k_proj(new_lb, W)
+        oik[0, -1], oiks[0, -1] = c_[0], d_[0]
+        qc, qsc = oracle.quant_nvfp4(iq)
+        idx = oracle.index_topk(qc.reshape(1, 1, 128), qsc.reshape(1, 1, 16), w, oik, oiks, ne, 1, q_pos, TOPK)
+        for li in range(len(LAYERS)):
+            oracle.sparse_attn(qs[li], olat, olsc, ne, idx, swas[li][0], swas[li][1], pos0, T_SWA, None, q_pos)
+
+    step()
+    reps, t0 = 0, time.perf_counter()
+    while reps < max_reps and (time.perf_counter() - t0) < seconds_target:
+        step()
+        reps += 1
+    el = time.perf_counter() - t0
+    return {"value": reps / el, "unit": "queries/s", "cores": 1, "kind": "oracle",
+            "sample": f"1 of the 32 batch rows at the full 131,072-entry context; the whole step (append, "
+                      f"indexer-q quantisation, index + Top-512, 4 attention layers) repeated {reps} times in "
+                      f"{el:.1f} s (cache setup {setup_s:.1f} s untimed)"}
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the oracle as it stands, on the host cores, rank 0 only."""
+    if rank != 0:
+        return
+    cb = _oracle_baseline(seconds_target=max(3.0, min(20.0, 2.0 * args.steps)))
+    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "queries/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / cb["value"] * B,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e2m1+f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "l2": "n/a (CPU)"},
+            "cpu_baseline": cb, "e2e": {"value": cb["value"], "unit": "queries/s", "h2d_bytes_per_step": 0,
+                                        "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import sparse_attention_fp4_quant_b200 as csa
+    device = f"cuda:{local_rank}"
+    torch.cuda.set_device(local_rank)
+    csa.lib()
+    grp = DecodeGroup(csa, seed=9 + rank, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    g_front, g_index, g_attn = _graph(grp.front), _graph(grp.index), _graph(grp.attention)
+    st = torch.cuda.current_stream()
+
+    def step(evs):
+        evs[0].record(st)
+        g_front.replay()
+        evs[1].record(st)
+        g_index.replay()
+        evs[2].record(st)
+        g_attn.replay()
+        evs[3].record(st)
+
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(4)]  # noqa: E731
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(mk())
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    all_ev = []
+    t_wall = time.perf_counter()
+    for _ in range(args.steps):
+        flush.zero_()
+        evs = mk()
+        step(evs)
+        all_ev.append(evs)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    wall_s = time.perf_counter() - t_wall
+    clocks = sampler.stop()
+    step_ms = [e[0].elapsed_time(e[3]) for e in all_ev]
+    index_ms = [e[1].elapsed_time(e[2]) for e in all_ev]
+    attn_ms = [e[2].elapsed_time(e[3]) for e in all_ev]
+    ms = float(np.mean(step_ms))
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(t.item())
+
+    # end to end through the public API with host buffers: pinned inputs copied in,
+    # the step, the four outputs copied back, every step
+    h_new = grp.new_lat.cpu().pin_memory()
+    h_iq = grp.iq_bf.cpu().pin_memory()
+    h_q = [q.cpu().pin_memory() for q in grp.q]
+    h_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in grp.out]
+    h2d = h_new.numel() * 2 + h_iq.numel() * 2 + sum(q.numel() * 2 for q in h_q)
+    d2h = sum(o.numel() * 2 for o in h_out)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = []
+    for it in range(args.warmup + args.steps):
+        flush.zero_()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        e0.record(st)
+        grp.new_lat.copy_(h_new, non_blocking=True)
+        grp.iq_bf.copy_(h_iq, non_blocking=True)
+        for q, hq in zip(grp.q, h_q):
+            q.copy_(hq, non_blocking=True)
+        g_front.replay()
+        g_index.replay()
+        g_attn.replay()
+        for o, ho in zip(grp.out, h_out):
+            ho.copy_(o, non_blocking=True)
+        e1.record(st)
+        e1.synchronize()
+        if it >= args.warmup:
+            e2e_ms.append(max(e0.elapsed_time(e1), (time.perf_counter() - t0) * 1000.0))
+    e2e = float(np.mean(e2e_ms))
+    t = torch.tensor([e2e], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    e2e_max = float(t.item())
+
+    if rank != 0:
+        return
+    peak, peak_kind = _peaks()
+    idx_s = float(np.mean(index_ms)) / 1000.0
+    achieved = INDEX_LAUNCH_BYTES / idx_s / 1e9
+    traffic = _ncu_traffic()
+    cb = _oracle_baseline() if (world == 1 and not args.no_cpu_baseline) else None
+    value = world * B / (ms_max / 1000.0)
+    line = {
+        "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e2m1+bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B_per_gpu": B, "ctx_entries": N_CTX, "topk": TOPK, "swa": T_SWA,
+                   "l2": "flushed between timed steps (256 MiB write outside the step events)",
+                   "graphs": "3 CUDA graphs per step (front, index, attention)"},
+        "index_attn_gbs": STEP_BYTES / (ms_max / 1000.0) / 1e9,
+        "index_attn_frac_of_hbm": STEP_BYTES / (ms_max / 1000.0) / 1e9 / peak,
+        "step_algorithmic_bytes": STEP_BYTES,
+        "segments_ms": {"front": float(np.mean([e[0].elapsed_time(e[1]) for e in all_ev])),
+                        "index_topk": float(np.mean(index_ms)), "attention_x4": float(np.mean(attn_ms))},
+        "roofline": {"kernel": "csa2_index_topk (select_kernel<dense>)", "bound": "hbm", "achieved": achieved,
+                     "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                     "bytes_per_launch": INDEX_LAUNCH_BYTES},
+        "cpu_baseline": cb,
+        "e2e": {"value": world * B / (e2e_max / 1000.0), "unit": "queries/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_max},
+        "gpu_launches": DecodeGroup.LAUNCHES_PER_STEP * args.steps,
+        "clocks": clocks,
+        "wall_s_timed_region": wall_s,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

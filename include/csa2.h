@@ -1,0 +1,286 @@
+/*
+ * csa2.h -- C ABI of libcsa2.so, the B200 (sm_100a) hot path of CSA2
+ * (Compressed Sparse Attention 2) as the public write-ups of the
+ * DeepSeek-V4.1-Flash report describe it.
+ *
+ * Sources cited below:
+ *   [Blog]  "一个 token 只花 890 字节：DeepSeek-V4.1-Flash 把 KV 缓存压到了什么程度"
+ *           (shibing624.github.io ai-paper-analysis): sections
+ *           "CSA2：跨层复用，能借就不自己算" (Fig. 4), "分层稀疏索引器：让深层
+ *           indexer 别全文搜索" (Fig. 5), "FP4 与 SWA Bounded Replay：另外两刀".
+ *   [Jdon]  "557亿参数只唤醒80亿！…" (jdon.com), section "缓存压缩真的是越大越好吗".
+ *   [Lsln]  m.lsln.cn news 211874, section "4.3 消融实验".
+ *
+ * General rules for every call
+ *   - Pointers marked "device" must point to device memory of the current
+ *     CUDA device; "host" pointers to host memory.  The library keeps no
+ *     pointer after the call returns and never frees caller memory.
+ *   - All work is enqueued on `stream` (a cudaStream_t passed as void*, NULL =
+ *     the legacy default stream).  No call synchronises the stream.
+ *   - Arguments are validated on the host before anything is launched; an
+ *     invalid argument returns CSA2_ERR_INVALID_ARG and launches nothing.
+ *     Device-resident counts and positions (n_entries, q_pos, idx, pool) are
+ *     clamped or treated as padding on the device; they never cause an
+ *     out-of-bounds access.
+ *   - A failed launch returns CSA2_ERR_CUDA; csa2_last_cuda_error() then gives
+ *     the cudaError_t value.  No C++ exception crosses this interface.
+ *
+ * Data layout (row-major, all sizes in bytes unless stated):
+ *   main latent row  : 512 channels -> 256 B of E2M1 codes (channel 2j in the
+ *                      low nibble of byte j, 2j+1 in the high nibble) plus 32 B
+ *                      of E4M3 scales, one per 16 channels (NVFP4 without the
+ *                      second-level scale: [Blog] FP4 section, [Lsln] 4.3).
+ *   indexer K row    : 64 channels -> 32 B codes + 4 B scales.
+ *   indexer Q        : per query [4 heads][32 B] codes + [4][4] scales.
+ *   E2M1 code        : bit 3 sign, bits 2:1 exponent (bias 1), bit 0 mantissa.
+ *   E4M3 byte        : "FN" variant, bias 7, no infinities, 0x7F/0xFF NaN
+ *                      (NaN scale bytes are not valid input).
+ *   SWA KV           : per token 512 E4M3 bytes and one fp32 scale (value =
+ *                      e4m3 * scale): the sliding-window KV stays FP8 ([Jdon]).
+ *   bf16             : IEEE bfloat16 bit patterns (uint16).
+ */
+#ifndef CSA2_C_ABI_H
+#define CSA2_C_ABI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CSA2_API __attribute__((visibility("default")))
+#else
+#define CSA2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CSA2_D 512          /* latent channels = attention head dim (K = V = latent) */
+#define CSA2_H 16           /* attention heads per query */
+#define CSA2_IH 4           /* indexer heads */
+#define CSA2_ID 64          /* indexer head dim */
+#define CSA2_BLOCK 8        /* positions per pool block ([Blog] Fig. 5) */
+#define CSA2_MAX_K 2048     /* largest Top-K / pool size a call accepts */
+#define CSA2_MAX_WINDOW 128 /* largest sliding window ([Blog]: n_win = 128) */
+
+typedef enum {
+    CSA2_OK = 0,
+    CSA2_ERR_INVALID_ARG = 1,
+    CSA2_ERR_UNSUPPORTED = 2,
+    CSA2_ERR_WORKSPACE = 3,
+    CSA2_ERR_CUDA = 4
+} csa2_status;
+
+/* Human-readable name of a status (static storage, never NULL). */
+CSA2_API const char* csa2_status_str(csa2_status s);
+
+/* The cudaError_t (as int) recorded by the last call that returned CSA2_ERR_CUDA
+ * on this host thread, or 0. */
+CSA2_API int csa2_last_cuda_error(void);
+
+/*
+ * The shared global KV of one CSA2 layer group: the FP4 main latent and the FP4
+ * indexer K, both written by the group's Full layer and borrowed by its
+ * Reindex and Reuse layers ([Blog] "CSA2" section, Fig. 4).
+ *   lat       device [B][cap][256]  E2M1 codes of the main latent
+ *   lat_sc    device [B][cap][32]   E4M3 scales of the main latent
+ *   ik        device [B][cap][32]   E2M1 codes of the indexer K
+ *   ik_sc     device [B][cap][4]    E4M3 scales of the indexer K
+ *   n_entries device [B] int32      valid entries per batch row (clamped to [0, cap])
+ *   cap       entries allocated per batch row (>= 1)
+ *   m         tokens compressed into one entry: 1 (decoder) or 2 (encoder).
+ *             Entry e covers tokens [m e, m e + m - 1] and is visible to the
+ *             query at token p once complete: m e + m - 1 <= p.
+ * All four byte arrays must be 16-byte aligned.
+ */
+typedef struct csa2_kv {
+    uint8_t* lat;
+    uint8_t* lat_sc;
+    uint8_t* ik;
+    uint8_t* ik_sc;
+    const int32_t* n_entries;
+    int64_t cap;
+    int32_t m;
+} csa2_kv;
+
+/*
+ * Step 1 -- NVFP4 quantisation ([Blog] FP4 section: E2M1 values, one E4M3
+ * scale per 16 channels, applied after RoPE; [Lsln] 4.3: no global scale).
+ * For each group of 16 channels: scale = E4M3 round-to-nearest-even
+ * (saturating at 448) of the fp32 quotient amax / 6; each code is the E2M1
+ * value nearest to x / scale (ties to the even code, saturating at 6) with the
+ * sign of x; a group whose scale rounds to 0 is written as all-zero codes.
+ *   x        device bf16 [rows][ch], 16-byte aligned
+ *   rows     >= 0 (0 is a no-op)
+ *   ch       multiple of 16, 16..4096
+ *   codes    device u8 [out_rows][ch/2], 8-byte aligned; row r goes to row dst_rows[r] (or r)
+ *   scales   device u8 [out_rows][ch/16]; same row mapping
+ *   dst_rows device int64 [rows] or NULL: destination row of each input row
+ *            (used to append one new entry per batch row into a [B][cap] cache);
+ *            a destination outside [0, out_rows) is skipped
+ *   out_rows rows of codes/scales (>= rows when dst_rows is NULL)
+ */
+CSA2_API csa2_status csa2_quant_nvfp4(const void* x, int64_t rows, int32_t ch, uint8_t* codes, uint8_t* scales,
+                                      const int64_t* dst_rows, int64_t out_rows, void* stream);
+
+/*
+ * Indexer-K projection ([Blog] "CSA2" section: the indexer K is projected from
+ * the main KV).  k = x W computed per output as an fp32 fused multiply-add
+ * chain over the 512 input channels in ascending order (starting from +0),
+ * then NVFP4-quantised exactly as csa2_quant_nvfp4 does (64 channels -> 32 B
+ * codes + 4 B scales).
+ *   x        device bf16 [rows][512] (post-RoPE latent rows), 16-byte aligned
+ *   W        device fp32 [512][64]
+ *   k_codes  device u8 [out_rows][32] (8-byte aligned), k_scales device u8 [out_rows][4];
+ *            row mapping and out_rows as for csa2_quant_nvfp4
+ */
+CSA2_API csa2_status csa2_index_k_proj(const void* x, int64_t rows, const float* W, uint8_t* k_codes,
+                                       uint8_t* k_scales, const int64_t* dst_rows, int64_t out_rows, void* stream);
+
+/*
+ * Step 2 -- FP4 index scoring + Top-K ([Blog] "CSA2" section: a lightweight
+ * indexer scores the causally visible compressed entries and keeps the Top-K,
+ * K = 512; [Blog] FP4 section: FP4 indexer Q/K).
+ * score(t) = sum_h w_h ReLU(q_h . k_t), evaluated in a fixed order:
+ *   I[h][b] = integer dot product of the doubled E2M1 values of block b (16 ch)
+ *   T[h][b] = I[h][b] * sq[h][b] * sk[b] / 4            (exact in fp32)
+ *   d_h = ((T0 + T1) + T2) + T3 (fp32);  r_h = max(d_h, +0)
+ *   score = ((w0 r0 + w1 r1) + w2 r2) + w3 r3 (fp32, each product rounded)
+ * The Top-K is the first min(k, n_visible) entries in (score descending,
+ * position ascending) order; their positions are written in ascending order
+ * and the rest of the row is -1.
+ *   q, q_sc       device u8 [B][Q][4][32], [B][Q][4][4]  FP4 indexer queries
+ *   w             device fp32 [B][Q][4]                  head weights
+ *   kv            host pointer to the group's KV (ik, ik_sc, n_entries, cap, m used)
+ *   q_pos         device int32 [B][Q]  token position of each query (visibility)
+ *   B, Q          >= 1 with B * Q <= 65535; k in [1, CSA2_MAX_K]
+ *   idx_out       device int32 [B][Q][k]
+ *   blockmax_out  device fp32 [B][Q][ceil(cap/8)] or NULL: the maximum score of
+ *                 each block of 8 positions (visible positions only), -inf for
+ *                 blocks with no visible position ([Blog] Fig. 5)
+ *   ws, ws_bytes  device workspace of at least csa2_workspace_bytes(CSA2_OP_INDEX_TOPK, ...)
+ *                 bytes, zero-filled before its first use; every call leaves its
+ *                 counters at zero again.  Calls that share a workspace must not
+ *                 overlap on the GPU.
+ */
+CSA2_API csa2_status csa2_index_topk(const uint8_t* q, const uint8_t* q_sc, const float* w, const csa2_kv* kv,
+                            const int32_t* q_pos, int32_t B, int32_t Q, int32_t k, int32_t* idx_out,
+                            float* blockmax_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Step 3a -- hierarchical sparse indexer, pool build ([Blog] "分层稀疏索引器",
+ * Fig. 5: the first Full layer's scores build a shared candidate pool of at
+ * most 2,048 blocks of 8 positions, blocks being chosen by maximum indexer
+ * score).  Keeps the first min(max_blocks, visible blocks) blocks in (block
+ * max descending, block id ascending) order, written as ascending block ids
+ * padded with -1.
+ *   blockmax   device fp32 [B][Q][ceil(kv->cap/8)] from csa2_index_topk
+ *   kv         host pointer (n_entries, cap, m used)
+ *   max_blocks in [1, CSA2_MAX_K]
+ *   pool_out   device int32 [B][Q][max_blocks]
+ *   ws         as for csa2_index_topk (CSA2_OP_POOL_BUILD)
+ */
+CSA2_API csa2_status csa2_pool_build(const float* blockmax, const csa2_kv* kv, const int32_t* q_pos, int32_t B, int32_t Q,
+                            int32_t max_blocks, int32_t* pool_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Step 3b -- Reindex layer: Top-K inside the pool ([Blog] "分层稀疏索引器":
+ * later Reindex layers select their Top-512 only inside the pool; [Blog] Fig. 4:
+ * a Reindex layer re-scores the borrowed global KV with its own indexer Q).
+ * Candidates are the visible positions 8b .. 8b+7 of every pool block b >= 0;
+ * the score, order and output are those of csa2_index_topk.  Pool block ids
+ * must be distinct; out-of-range ids are ignored.
+ *   pool   device int32 [B][Q][P]
+ *   ws     as above (CSA2_OP_POOL_TOPK)
+ */
+CSA2_API csa2_status csa2_pool_topk(const uint8_t* q, const uint8_t* q_sc, const float* w, const csa2_kv* kv,
+                           const int32_t* pool, int32_t P, const int32_t* q_pos, int32_t B, int32_t Q, int32_t k,
+                           int32_t* idx_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Step 4 -- sparse attention over the selected FP4 entries and the layer's own
+ * FP8 sliding-window KV ([Blog] "CSA2" section: Top-K sparse attention plus the
+ * layer's own SWA KV; K = V = the dequantised latent) under the SWA Bounded
+ * Replay mask ([Blog] FP4/SWA section: replaying from start s, the query at
+ * token i sees SWA keys in [max(s, i - W + 1), i]).  One softmax runs jointly
+ * over the main and SWA keys of each head:
+ *   z_j = (q_h . k_j) * sm_scale, p = softmax(z), out_h = sum_j p_j v_j.
+ *   q            device bf16 [B][Q][16][512], 16-byte aligned
+ *   kv           host pointer (lat, lat_sc, n_entries, cap used)
+ *   idx, k       device int32 [B][Q][k] main entries; -1 or out-of-range = padding; k in [0, CSA2_MAX_K]
+ *   swa, swa_sc  device u8 [B][T][512] (16-byte aligned), fp32 [B][T]; row r holds token swa_pos0[b] + r
+ *   swa_pos0     device int32 [B];  T >= 0
+ *   window       W in [1, CSA2_MAX_WINDOW]
+ *   replay_start device int32 [B] (s) or NULL (no replay bound)
+ *   q_pos        device int32 [B][Q] token position i of each query
+ *   sm_scale     softmax scale (1/sqrt(512) in the synthetic workloads)
+ *   out          device bf16 [B][Q][16][512]; a query with no visible key gets zeros
+ *   lse          device fp32 [B][Q][16] (natural-log sum-exp of z) or NULL
+ *   ws           as above (CSA2_OP_SPARSE_ATTN)
+ */
+CSA2_API csa2_status csa2_sparse_attn(const void* q, const csa2_kv* kv, const int32_t* idx, int32_t k, const uint8_t* swa,
+                             const float* swa_sc, const int32_t* swa_pos0, int32_t T, int32_t window,
+                             const int32_t* replay_start, const int32_t* q_pos, int32_t B, int32_t Q,
+                             float sm_scale, void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace sizes.  `op` selects the call; the other arguments are those of the
+ * call (k = Top-K or max_blocks; P = pool size for CSA2_OP_POOL_TOPK, else 0). */
+typedef enum {
+    CSA2_OP_INDEX_TOPK = 0,
+    CSA2_OP_POOL_BUILD = 1,
+    CSA2_OP_POOL_TOPK = 2,
+    CSA2_OP_SPARSE_ATTN = 3,
+    CSA2_OP_LAYER = 4
+} csa2_op;
+CSA2_API size_t csa2_workspace_bytes(csa2_op op, int32_t B, int32_t Q, int64_t cap, int32_t k, int32_t P);
+
+/*
+ * Step 5 -- one CSA2 layer dispatched by its static mode ([Blog] "CSA2"
+ * section, Fig. 4): FULL computes the group's main KV and indexer K for the new
+ * entries and a fresh Top-K (and, if pool != NULL, builds the pool from this
+ * layer's block maxima); REINDEX re-scores the borrowed KV inside the pool with
+ * its own indexer Q; REUSE borrows the indices as well.  Every mode then runs
+ * sparse attention with the layer's own Q and SWA KV.
+ */
+typedef enum { CSA2_MODE_FULL = 0, CSA2_MODE_REINDEX = 1, CSA2_MODE_REUSE = 2 } csa2_mode;
+
+typedef struct csa2_layer_args {
+    csa2_mode mode;
+    const csa2_kv* kv;            /* host pointer to the group's shared KV */
+    int32_t B, Q;
+    const int32_t* q_pos;         /* device [B][Q] */
+    /* FULL only: append new entries (skipped when n_new == 0) */
+    const void* new_latent;       /* device bf16 [n_new][512] post-RoPE latent rows */
+    int64_t n_new;
+    const int64_t* new_rows;      /* device int64 [n_new]: destination row b*cap + e */
+    const float* k_proj;          /* device fp32 [512][64] indexer-K projection */
+    /* FULL and REINDEX: the layer's own indexer query */
+    const uint8_t* iq;            /* device [B][Q][4][32] */
+    const uint8_t* iq_sc;         /* device [B][Q][4][4] */
+    const float* w;               /* device [B][Q][4] */
+    /* shared selection state of the group */
+    int32_t* idx;                 /* device [B][Q][k]: written by FULL/REINDEX, read by all */
+    int32_t k;
+    int32_t* pool;                /* device [B][Q][pool_blocks]: written by FULL (if not NULL), read by REINDEX */
+    int32_t pool_blocks;
+    float* blockmax;              /* device [B][Q][ceil(cap/8)] scratch for the FULL layer's pool build */
+    /* the layer's own attention inputs */
+    const void* q;                /* device bf16 [B][Q][16][512] */
+    const uint8_t* swa;           /* device [B][T][512] */
+    const float* swa_sc;          /* device [B][T] */
+    const int32_t* swa_pos0;      /* device [B] */
+    int32_t T, window;
+    const int32_t* replay_start;  /* device [B] or NULL */
+    float sm_scale;
+    void* out;                    /* device bf16 [B][Q][16][512] */
+    float* lse;                   /* device [B][Q][16] or NULL */
+    void* ws;                     /* workspace of csa2_workspace_bytes(CSA2_OP_LAYER, B, Q, cap, k, pool_blocks) */
+    size_t ws_bytes;
+} csa2_layer_args;
+
+CSA2_API csa2_status csa2_layer_step(const csa2_layer_args* a, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA2_C_ABI_H */

@@ -1,0 +1,435 @@
+// attn.cu -- sparse attention over the Top-K FP4 main rows plus the layer's own
+// FP8 sliding-window KV, under the SWA Bounded Replay mask.
+//
+// Key slots of a query: [0, k) are the main rows idx[0..k), [k, k + W) are the
+// window tokens i - W + 1 .. i.  A slot is live if its row exists and (for the
+// window) the token lies in [max(s, i - W + 1), i] and in the stored SWA rows.
+// A CTA takes a split of the slot range in tiles of 64 keys: the tile is
+// gathered and dequantised to bf16 in swizzled shared memory (K = V), S = Q K^T
+// and O += P V run on warp-level tensor-core MMAs with the 16 heads as the M
+// dimension, and the softmax is online across tiles.  FP4 rows dequantise
+// exactly to bf16; an SWA row is stored as its E4M3 values (exact in bf16) and
+// its fp32 token scale multiplies the logit and the probability instead.  P
+// enters the P V product as two bf16 terms (rounded value + remainder), so the
+// product carries about 16 bits of P rather than 8.
+// Splits of one query are merged by the last CTA to finish (atomic ticket).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace csa2 {
+
+constexpr int kAT = 128;      // threads per CTA (4 warps)
+constexpr int kKT = 64;       // keys per tile
+constexpr int kRowB = kD * 2; // bytes per bf16 row of 512
+
+struct AttnSmem {
+    uint8_t K[kKT * kRowB];   // 64 KB, 16-byte chunks XOR-swizzled by row & 7
+    uint8_t Qs[kH * kRowB];   // 16 KB, same swizzle
+    uint8_t P[kH * kKT * 2];  // 2 KB, bf16 P (rounded), same swizzle over 8 chunks per row
+    uint8_t Pl[kH * kKT * 2]; // 2 KB, bf16 remainder P - rounded(P)
+    float kf[kKT];            // per-key factor (1 for FP4 rows, token scale for SWA)
+    int kvalid[kKT];
+    float red_max[4][kH];
+    float red_sum[4][kH];
+    float m_run[kH], l_run[kH], alpha[kH];
+    int last;
+};
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk) { return (uint32_t)(row * kRowB + ((chunk ^ (row & 7)) << 4)); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// 8 E2M1 codes (nibble n = dim n) times the block scale -> 8 bf16 (exact).
+__device__ __forceinline__ uint4 fp4x8_to_bf16(uint32_t w, float s) {
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) o[j] = pack_bf16(e2m1_to_f32(w >> (8 * j)) * s, e2m1_to_f32(w >> (8 * j + 4)) * s);
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// 4 E4M3 bytes -> 4 bf16 (exact).
+__device__ __forceinline__ uint2 fp8x4_to_bf16(uint32_t w) {
+    float f[4];
+    e4m3x4_to_f32(w, f);
+    return make_uint2(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16(float c[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, qd = lane & 3;
+    const int bq = blockIdx.y;
+    const int split = blockIdx.x, S = gridDim.x;
+    const int b = bq / p.Q;
+    const int64_t i_pos = p.q_pos[bq];
+    int64_t lo = i_pos - p.window + 1;
+    if (p.replay_start && lo < (int64_t)p.replay_start[b]) lo = p.replay_start[b];
+    const int64_t pos0 = p.swa_pos0[b];
+    int64_t nmain = p.n_entries[b];
+    if (nmain > p.cap) nmain = p.cap;
+    const float scale_log2 = p.sm_scale * 1.4426950408889634f;
+
+    const uint32_t sK = (uint32_t)__cvta_generic_to_shared(sm.K);
+    const uint32_t sQ = (uint32_t)__cvta_generic_to_shared(sm.Qs);
+    const uint32_t sP = (uint32_t)__cvta_generic_to_shared(sm.P);
+    const uint32_t sPl = (uint32_t)__cvta_generic_to_shared(sm.Pl);
+
+    // Q [16][512] bf16 -> swizzled smem
+    {
+        const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (int64_t)bq * kH * kD);
+#pragma unroll
+        for (int it = 0; it < (kH * kD / 8) / kAT; ++it) {
+            int c = it * kAT + tid;  // 16-byte chunk id
+            int row = c >> 6, ch = c & 63;
+            uint4 v = __ldg(qsrc + c);
+            *reinterpret_cast<uint4*>(sm.Qs + swz(row, ch)) = v;
+        }
+    }
+    if (tid < kH) {
+        sm.m_run[tid] = -INFINITY;
+        sm.l_run[tid] = 0.0f;
+    }
+
+    float o[16][4];
+#pragma unroll
+    for (int n = 0; n < 16; ++n)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o[n][j] = 0.0f;
+
+    const int ntiles = (p.slots_total + kKT - 1) / kKT;
+    const int t0 = split * p.tiles_per_split;
+    const int t1 = min(ntiles, t0 + p.tiles_per_split);
+
+    for (int tile = t0; tile < t1; ++tile) {
+        // ---- gather + dequantise 64 key rows (2 threads per row) ----
+        {
+            const int r = tid >> 1, half = tid & 1;
+            const int slot = tile * kKT + r;
+            bool live = false;
+            float fac = 1.0f;
+            if (slot < p.k) {
+                int32_t e = __ldg(p.idx + (int64_t)bq * p.k + slot);
+                if (e >= 0 && e < nmain) {
+                    live = true;
+                    const int64_t row = (int64_t)b * p.cap + e;
+                    const uint4* cs = reinterpret_cast<const uint4*>(p.lat + row * (kD / 2) + 128 * half);
+                    uint4 scw = __ldg(reinterpret_cast<const uint4*>(p.lat_sc + row * (kD / 16) + 16 * half));
+                    uint32_t scb[4] = {scw.x, scw.y, scw.z, scw.w};
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        uint4 cw = __ldg(cs + v);
+                        uint32_t ws[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            int word = 4 * v + j;                    // 8 dims per word, 32 words per half row
+                            int sbyte = word >> 1;                   // one scale per 16 dims
+                            float s = e4m3_to_f32((scb[sbyte >> 2] >> (8 * (sbyte & 3))) & 0xFFu);
+                            int chunk = 32 * half + word;
+                            *reinterpret_cast<uint4*>(sm.K + swz(r, chunk)) = fp4x8_to_bf16(ws[j], s);
+                        }
+                    }
+                }
+            } else if (slot < p.slots_total) {
+                int64_t tau = i_pos - p.window + 1 + (slot - p.k);
+                int64_t rr = tau - pos0;
+                if (tau >= lo && tau <= i_pos && rr >= 0 && rr < p.T) {
+                    live = true;
+                    const int64_t row = (int64_t)b * p.T + rr;
+                    fac = __ldg(p.swa_sc + row);
+                    const uint4* cs = reinterpret_cast<const uint4*>(p.swa + row * kD + 256 * half);
+#pragma unroll
+                    for (int v = 0; v < 16; ++v) {
+                        uint4 cw = __ldg(cs + v);
+                        uint2 a = fp8x4_to_bf16(cw.x), bb = fp8x4_to_bf16(cw.y);
+                        uint2 c = fp8x4_to_bf16(cw.z), d = fp8x4_to_bf16(cw.w);
+                        int chunk = 32 * half + 2 * v;
+                        *reinterpret_cast<uint4*>(sm.K + swz(r, chunk)) = make_uint4(a.x, a.y, bb.x, bb.y);
+                        *reinterpret_cast<uint4*>(sm.K + swz(r, chunk + 1)) = make_uint4(c.x, c.y, d.x, d.y);
+                    }
+                }
+            }
+            if (!live) {
+#pragma unroll
+                for (int c = 0; c < 32; ++c) *reinterpret_cast<uint4*>(sm.K + swz(r, 32 * half + c)) = make_uint4(0, 0, 0, 0);
+            }
+            if (half == 0) {
+                sm.kvalid[r] = live;
+                sm.kf[r] = fac;
+            }
+        }
+        __syncthreads();
+
+        // ---- S = Q K^T for keys 16*warp .. +15 ----
+        float s[2][4];
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) s[n][j] = 0.0f;
+#pragma unroll 4
+        for (int ks = 0; ks < kD / 16; ++ks) {
+            uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+            ldsm_x4(sQ + swz(lane & 15, 2 * ks + (lane >> 4)), a0, a1, a2, a3);
+            const int mi = lane >> 3;
+            const int key = 16 * warp + (mi >> 1) * 8 + (lane & 7);
+            ldsm_x4(sK + swz(key, 2 * ks + (mi & 1)), b0, b1, b2, b3);
+            mma_bf16(s[0], a0, a1, a2, a3, b0, b1);
+            mma_bf16(s[1], a0, a1, a2, a3, b2, b3);
+        }
+        // logits (log2 units), masked keys -> -inf
+        float z[2][4];
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                int key = 16 * warp + 8 * n + 2 * qd + (j & 1);
+                float v = sm.kvalid[key] ? s[n][j] * sm.kf[key] * scale_log2 : -INFINITY;
+                z[n][j] = v;
+                if (j < 2) mx0 = fmaxf(mx0, v); else mx1 = fmaxf(mx1, v);
+            }
+#pragma unroll
+        for (int o2 = 1; o2 < 4; o2 <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, o2));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xFFFFFFFFu, mx1, o2));
+        }
+        if (qd == 0) {
+            sm.red_max[warp][g] = mx0;
+            sm.red_max[warp][g + 8] = mx1;
+        }
+        __syncthreads();
+        float mt0 = fmaxf(fmaxf(sm.red_max[0][g], sm.red_max[1][g]), fmaxf(sm.red_max[2][g], sm.red_max[3][g]));
+        float mt1 = fmaxf(fmaxf(sm.red_max[0][g + 8], sm.red_max[1][g + 8]),
+                          fmaxf(sm.red_max[2][g + 8], sm.red_max[3][g + 8]));
+        float mn0 = fmaxf(sm.m_run[g], mt0), mn1 = fmaxf(sm.m_run[g + 8], mt1);
+        float mu0 = (mn0 == -INFINITY) ? 0.0f : mn0, mu1 = (mn1 == -INFINITY) ? 0.0f : mn1;
+        float sum0 = 0.0f, sum1 = 0.0f;
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+            int key0 = 16 * warp + 8 * n + 2 * qd;
+            float p00 = exp2f(z[n][0] - mu0), p01 = exp2f(z[n][1] - mu0);
+            float p10 = exp2f(z[n][2] - mu1), p11 = exp2f(z[n][3] - mu1);
+            sum0 += p00 + p01;
+            sum1 += p10 + p11;
+            float f0 = sm.kf[key0], f1 = sm.kf[key0 + 1];
+            // P row = head, column = key; 2 keys per 32-bit word
+            int chunk = key0 >> 3, within = (key0 & 7) * 2;
+            const uint32_t o0 = g * 128 + ((chunk ^ (g & 7)) << 4) + within;
+            const uint32_t o1 = (g + 8) * 128 + ((chunk ^ ((g + 8) & 7)) << 4) + within;
+            float v00 = p00 * f0, v01 = p01 * f1, v10 = p10 * f0, v11 = p11 * f1;
+            __nv_bfloat162 h0 = __floats2bfloat162_rn(v00, v01), h1 = __floats2bfloat162_rn(v10, v11);
+            *reinterpret_cast<__nv_bfloat162*>(sm.P + o0) = h0;
+            *reinterpret_cast<__nv_bfloat162*>(sm.P + o1) = h1;
+            *reinterpret_cast<uint32_t*>(sm.Pl + o0) =
+                pack_bf16(v00 - __low2float(h0), v01 - __high2float(h0));
+            *reinterpret_cast<uint32_t*>(sm.Pl + o1) =
+                pack_bf16(v10 - __low2float(h1), v11 - __high2float(h1));
+        }
+#pragma unroll
+        for (int o2 = 1; o2 < 4; o2 <<= 1) {
+            sum0 += __shfl_xor_sync(0xFFFFFFFFu, sum0, o2);
+            sum1 += __shfl_xor_sync(0xFFFFFFFFu, sum1, o2);
+        }
+        if (qd == 0) {
+            sm.red_sum[warp][g] = sum0;
+            sm.red_sum[warp][g + 8] = sum1;
+        }
+        __syncthreads();
+        if (tid < kH) {
+            float mt = fmaxf(fmaxf(sm.red_max[0][tid], sm.red_max[1][tid]), fmaxf(sm.red_max[2][tid], sm.red_max[3][tid]));
+            float mo = sm.m_run[tid];
+            float mn = fmaxf(mo, mt);
+            float al = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
+            sm.alpha[tid] = al;
+            sm.l_run[tid] = sm.l_run[tid] * al +
+                            ((sm.red_sum[0][tid] + sm.red_sum[1][tid]) + (sm.red_sum[2][tid] + sm.red_sum[3][tid]));
+            sm.m_run[tid] = mn;
+        }
+        __syncthreads();
+
+        // ---- O[:, 128 warp .. +127] = alpha O + P V ----
+        {
+            float al0 = sm.alpha[g], al1 = sm.alpha[g + 8];
+#pragma unroll
+            for (int n = 0; n < 16; ++n) {
+                o[n][0] *= al0;
+                o[n][1] *= al0;
+                o[n][2] *= al1;
+                o[n][3] *= al1;
+            }
+#pragma unroll
+            for (int kk = 0; kk < kKT / 16; ++kk) {
+                uint32_t a0, a1, a2, a3, l0, l1, l2, l3;
+                {
+                    int row = lane & 15, chunk = 2 * kk + (lane >> 4);
+                    uint32_t off = (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+                    ldsm_x4(sP + off, a0, a1, a2, a3);
+                    ldsm_x4(sPl + off, l0, l1, l2, l3);
+                }
+                const int mi = lane >> 3;
+                const int key = 16 * kk + (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+                for (int np = 0; np < 8; ++np) {
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_t(sK + swz(key, 16 * warp + 2 * np + (mi >> 1)), b0, b1, b2, b3);
+                    mma_bf16(o[2 * np], a0, a1, a2, a3, b0, b1);
+                    mma_bf16(o[2 * np + 1], a0, a1, a2, a3, b2, b3);
+                    mma_bf16(o[2 * np], l0, l1, l2, l3, b0, b1);
+                    mma_bf16(o[2 * np + 1], l0, l1, l2, l3, b2, b3);
+                }
+            }
+        }
+        __syncthreads();
+    }
+
+    // ---- write the split's partial, or the final output ----
+    const float LN2 = 0.6931471805599453f;
+    if (S == 1) {
+        float l0 = sm.l_run[g], l1 = sm.l_run[g + 8];
+        float inv0 = l0 > 0.0f ? 1.0f / l0 : 0.0f, inv1 = l1 > 0.0f ? 1.0f / l1 : 0.0f;
+        uint16_t* out = p.out + (int64_t)bq * kH * kD;
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+            int d = 128 * warp + 8 * n + 2 * qd;
+            *reinterpret_cast<uint32_t*>(out + g * kD + d) = pack_bf16(o[n][0] * inv0, o[n][1] * inv0);
+            *reinterpret_cast<uint32_t*>(out + (g + 8) * kD + d) = pack_bf16(o[n][2] * inv1, o[n][3] * inv1);
+        }
+        if (p.lse && tid < kH) {
+            float l = sm.l_run[tid];
+            p.lse[(int64_t)bq * kH + tid] = l > 0.0f ? (sm.m_run[tid] + log2f(l)) * LN2 : -INFINITY;
+        }
+        return;
+    }
+    {
+        float* po = p.part_o + ((int64_t)bq * S + split) * kH * kD;
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+            int d = 128 * warp + 8 * n + 2 * qd;
+            *reinterpret_cast<float2*>(po + g * kD + d) = make_float2(o[n][0], o[n][1]);
+            *reinterpret_cast<float2*>(po + (g + 8) * kD + d) = make_float2(o[n][2], o[n][3]);
+        }
+        if (tid < kH) {
+            float* pml = p.part_ml + (((int64_t)bq * S + split) * kH + tid) * 2;
+            pml[0] = sm.m_run[tid];
+            pml[1] = sm.l_run[tid];
+        }
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) sm.last = (atomicAdd(&p.counters[bq], 1) == S - 1);
+    __syncthreads();
+    if (!sm.last) return;
+    __threadfence();
+    // combine the S partials: weights 2^(m_s - M), normaliser sum_s l_s 2^(m_s - M)
+    if (tid < kH) {
+        float M = -INFINITY;
+        for (int c = 0; c < S; ++c) M = fmaxf(M, __ldcg(p.part_ml + (((int64_t)bq * S + c) * kH + tid) * 2));
+        float Mu = (M == -INFINITY) ? 0.0f : M;
+        float L = 0.0f;
+        for (int c = 0; c < S; ++c) {
+            const float* pml = p.part_ml + (((int64_t)bq * S + c) * kH + tid) * 2;
+            float wgt = exp2f(__ldcg(pml) - Mu);
+            L += __ldcg(pml + 1) * wgt;
+        }
+        sm.m_run[tid] = Mu;
+        sm.l_run[tid] = L;
+        if (p.lse) p.lse[(int64_t)bq * kH + tid] = L > 0.0f ? (Mu + log2f(L)) * LN2 : -INFINITY;
+    }
+    __syncthreads();
+    for (int e = tid; e < kH * kD / 2; e += kAT) {
+        int h = (2 * e) / kD, d = (2 * e) % kD;
+        float L = sm.l_run[h], Mu = sm.m_run[h];
+        float a0 = 0.0f, a1 = 0.0f;
+        for (int c = 0; c < S; ++c) {
+            float wgt = exp2f(__ldcg(p.part_ml + (((int64_t)bq * S + c) * kH + h) * 2) - Mu);
+            float2 v = __ldcg(reinterpret_cast<const float2*>(p.part_o + ((int64_t)bq * S + c) * kH * kD + h * kD + d));
+            a0 += v.x * wgt;
+            a1 += v.y * wgt;
+        }
+        float inv = L > 0.0f ? 1.0f / L : 0.0f;
+        *reinterpret_cast<uint32_t*>(p.out + (int64_t)bq * kH * kD + h * kD + d) = pack_bf16(a0 * inv, a1 * inv);
+    }
+    if (tid == 0) p.counters[bq] = 0;
+}
+
+int attn_splits(int B, int Q, int k, int window, int* tiles_per_split) {
+    int ntiles = (k + window + kKT - 1) / kKT;
+    if (ntiles < 1) ntiles = 1;
+    int64_t bq = (int64_t)B * Q;
+    int64_t want = (2 * kNumSMs) / (bq > 0 ? bq : 1);
+    if (want < 1) want = 1;
+    if (want > ntiles) want = ntiles;
+    int tps = (int)((ntiles + want - 1) / want);
+    int S = (ntiles + tps - 1) / tps;
+    if (tiles_per_split) *tiles_per_split = tps;
+    return S;
+}
+
+size_t attn_ws_bytes(int B, int Q, int k, int window) {
+    // bound the split count over every window <= CSA2_MAX_WINDOW: S <= min(tiles, CTA budget)
+    (void)window;
+    int64_t bq = (int64_t)B * Q;
+    int64_t want = (2 * kNumSMs) / (bq > 0 ? bq : 1);
+    if (want < 1) want = 1;
+    int64_t ntiles_max = (k + CSA2_MAX_WINDOW + kKT - 1) / kKT;
+    int64_t S = want < ntiles_max ? want : ntiles_max;
+    size_t ubq = (size_t)bq;
+    size_t bytes = align256(ubq * 4);
+    if (S > 1) bytes += align256(ubq * S * kH * kD * 4) + align256(ubq * S * kH * 2 * 4);
+    return bytes;
+}
+
+void attn_carve_ws(AttnParams& p, int S, void* ws) {
+    int64_t bq = (int64_t)p.B * p.Q;
+    int64_t want = (2 * kNumSMs) / (bq > 0 ? bq : 1);
+    if (want < 1) want = 1;
+    int64_t ntiles_max = (p.k + CSA2_MAX_WINDOW + kKT - 1) / kKT;
+    int64_t Sb = want < ntiles_max ? want : ntiles_max;
+    char* c = (char*)ws;
+    p.counters = (int32_t*)c;
+    c += align256((size_t)bq * 4);
+    if (S > 1) {
+        p.part_o = (float*)c;
+        c += align256((size_t)bq * Sb * kH * kD * 4);
+        p.part_ml = (float*)c;
+    }
+}
+
+cudaError_t launch_attn(AttnParams& p, int S, cudaStream_t st) {
+    static bool attr_set = false;
+    const int smem = (int)sizeof(AttnSmem);
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    dim3 grid(S, p.B * p.Q);
+    attn_kernel<<<grid, kAT, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace csa2

@@ -1,0 +1,260 @@
+// index.cu -- FP4 index scoring + exact Top-K (Full layers), pool Top-K
+// (Reindex layers) and pool build (hierarchical sparse indexer).
+//
+// One CTA scores a contiguous share of one query's candidates, keeps its local
+// best k in shared memory (topk.cuh) and writes them to the workspace; the
+// last CTA of the query (atomic ticket) merges the shares and writes the
+// ascending positions.  With one share per query the CTA writes directly.
+#include "common.cuh"
+#include "kernels.h"
+#include "topk.cuh"
+
+namespace csa2 {
+
+constexpr int kNT = 256;
+constexpr int kCap = 4096;
+using TK = TopK<kNT, kCap>;
+
+// The query side of the score, decoded once per CTA.
+struct QReg {
+    uint32_t q8[kIH][4][4];  // [head][block][word]: doubled E2M1 values as int8x4
+    float f[kIH][4];         // sq[h][b] / 4
+    float w[kIH];
+};
+
+__device__ __forceinline__ void load_query(QReg& R, const uint8_t* q, const uint8_t* qs, const float* w) {
+#pragma unroll
+    for (int h = 0; h < kIH; ++h) {
+        const uint4* src = reinterpret_cast<const uint4*>(q + 32 * h);
+        uint4 a = __ldg(src), c = __ldg(src + 1);
+        uint32_t cw[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int wi = 0; wi < 8; ++wi) e2m1x8_to_i8x2(cw[wi], R.q8[h][wi >> 1][2 * (wi & 1)], R.q8[h][wi >> 1][2 * (wi & 1) + 1]);
+        uint32_t sw = *reinterpret_cast<const uint32_t*>(qs + 4 * h);
+        float sf[4];
+        e4m3x4_to_f32(sw, sf);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) R.f[h][b] = sf[b] * 0.25f;
+        R.w[h] = __ldg(w + h);
+    }
+}
+
+// score = sum_h w_h ReLU(d_h) in the fixed order of csa2_index_topk.
+__device__ __forceinline__ float entry_score(const QReg& R, uint4 c0, uint4 c1, uint32_t skw) {
+    uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+    uint32_t k8[4][4];
+#pragma unroll
+    for (int wi = 0; wi < 8; ++wi) e2m1x8_to_i8x2(cw[wi], k8[wi >> 1][2 * (wi & 1)], k8[wi >> 1][2 * (wi & 1) + 1]);
+    float sk[4];
+    e4m3x4_to_f32(skw, sk);
+    float score = 0.0f;
+#pragma unroll
+    for (int h = 0; h < kIH; ++h) {
+        float d = 0.0f;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            int I = __dp4a((int)R.q8[h][b][0], (int)k8[b][0], 0);
+            I = __dp4a((int)R.q8[h][b][1], (int)k8[b][1], I);
+            I = __dp4a((int)R.q8[h][b][2], (int)k8[b][2], I);
+            I = __dp4a((int)R.q8[h][b][3], (int)k8[b][3], I);
+            float T = __fmul_rn((float)I, __fmul_rn(R.f[h][b], sk[b]));  // exact
+            d = (b == 0) ? T : __fadd_rn(d, T);
+        }
+        float r = d > 0.0f ? d : 0.0f;
+        float pr = __fmul_rn(R.w[h], r);
+        score = (h == 0) ? pr : __fadd_rn(score, pr);
+    }
+    return score;
+}
+
+__device__ __forceinline__ float entry_score_at(const QReg& R, const uint8_t* ik, const uint8_t* iks, int64_t e) {
+    const uint4* c = reinterpret_cast<const uint4*>(ik + e * 32);
+    uint4 c0 = __ldg(c), c1 = __ldg(c + 1);
+    uint32_t sw = __ldg(reinterpret_cast<const uint32_t*>(iks + e * 4));
+    return entry_score(R, c0, c1, sw);
+}
+
+enum { MODE_DENSE = 0, MODE_POOL = 1, MODE_BUILD = 2 };
+
+// Merge the S shares of query bq from the workspace (last CTA only), then write
+// the ascending positions.  Block-collective.
+__device__ void finalize(TK& tk, const SelectParams& p, int bq, int S, int k, int32_t* out) {
+    const int tid = threadIdx.x;
+    if (S > 1) {
+        TK::Smem& sm = tk.s;
+        int cnt = sm.count;
+        int64_t off = ((int64_t)bq * S + blockIdx.x) * k;
+        for (int i = tid; i < cnt; i += kNT) {
+            p.cand_key[off + i] = sm.key[i];
+            p.cand_pos[off + i] = sm.pos[i];
+        }
+        if (tid == 0) p.cand_cnt[(int64_t)bq * S + blockIdx.x] = cnt;
+        __threadfence();
+        __syncthreads();
+        __shared__ int s_last;
+        if (tid == 0) s_last = (atomicAdd(&p.counters[bq], 1) == S - 1);
+        __syncthreads();
+        if (!s_last) return;
+        __threadfence();
+        tk.init();
+        for (int c = 0; c < S; ++c) {
+            int n = __ldcg(&p.cand_cnt[(int64_t)bq * S + c]);
+            int64_t coff = ((int64_t)bq * S + c) * k;
+            for (int base = 0; base < n; base += kNT) {
+                tk.make_room(k, kNT);
+                int i = base + tid;
+                bool valid = i < n;
+                uint32_t key = valid ? __ldcg(&p.cand_key[coff + i]) : 0u;
+                int32_t pos = valid ? __ldcg(&p.cand_pos[coff + i]) : 0;
+                tk.offer(valid, key, pos);
+            }
+        }
+        tk.finish(k);
+        if (tid == 0) p.counters[bq] = 0;
+    }
+    int cnt = tk.s.count;
+    tk.sort_positions(cnt);
+    for (int i = tid; i < k; i += kNT) out[(int64_t)bq * k + i] = i < cnt ? tk.s.pos[i] : -1;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kNT, 2) select_kernel(SelectParams p) {
+    __shared__ TK::Smem sm;
+    TK tk(sm);
+    const int tid = threadIdx.x;
+    const int bq = blockIdx.y;
+    const int s = blockIdx.x, S = gridDim.x;
+    const int b = bq / p.Q;
+    const int nvis = n_visible(p.q_pos[bq], p.n_entries[b], p.m, p.cap);
+    const int k = p.k;
+    tk.init();
+
+    if (MODE == MODE_BUILD) {
+        const int64_t nbcap = p.nb_cap;
+        int nblk = (nvis + kBlk - 1) / kBlk;
+        if (nblk > nbcap) nblk = (int)nbcap;
+        int chunk = (nblk + S - 1) / S;
+        int lo = min(nblk, s * chunk), hi = min(nblk, lo + chunk);
+        const float* bm = p.blockmax + (int64_t)bq * nbcap;
+        for (int base = lo; base < hi; base += kNT) {
+            tk.make_room(k, kNT);
+            int j = base + tid;
+            bool valid = j < hi;
+            float v = valid ? __ldg(bm + j) : 0.0f;
+            tk.offer(valid, score_key(v), j);
+        }
+        tk.finish(k);
+        finalize(tk, p, bq, S, k, p.out);
+        return;
+    }
+
+    QReg R;
+    load_query(R, p.q + (int64_t)bq * 128, p.q_sc + (int64_t)bq * 16, p.w + (int64_t)bq * 4);
+    const uint8_t* ik = p.ik + (int64_t)b * p.cap * 32;
+    const uint8_t* iks = p.ik_sc + (int64_t)b * p.cap * 4;
+
+    if (MODE == MODE_DENSE) {
+        int chunk = (((nvis + S - 1) / S) + 7) & ~7;
+        int lo = min(nvis, s * chunk), hi = min(nvis, lo + chunk);
+        float* bm = p.blockmax ? p.blockmax + (int64_t)bq * p.nb_cap : nullptr;
+        for (int base = lo; base < hi; base += 2 * kNT) {
+            tk.make_room(k, 2 * kNT);
+            int e0 = base + tid, e1 = base + kNT + tid;
+            bool v0 = e0 < hi, v1 = e1 < hi;
+            float s0 = -INFINITY, s1 = -INFINITY;
+            if (v0) s0 = entry_score_at(R, ik, iks, e0);
+            if (v1) s1 = entry_score_at(R, ik, iks, e1);
+            if (bm) {
+                float m0 = s0, m1 = s1;
+#pragma unroll
+                for (int o = 1; o < 8; o <<= 1) {
+                    m0 = fmaxf(m0, __shfl_xor_sync(0xFFFFFFFFu, m0, o));
+                    m1 = fmaxf(m1, __shfl_xor_sync(0xFFFFFFFFu, m1, o));
+                }
+                if ((tid & 7) == 0) {
+                    if (v0) bm[e0 >> 3] = m0;
+                    if (v1) bm[e1 >> 3] = m1;
+                }
+            }
+            tk.offer(v0, score_key(s0), e0);
+            tk.offer(v1, score_key(s1), e1);
+        }
+        if (bm) {  // blocks with no visible position
+            int64_t jb = (nvis + kBlk - 1) / kBlk;
+            int64_t rest = p.nb_cap - jb;
+            if (rest > 0) {
+                int64_t cs = (rest + S - 1) / S;
+                int64_t j0 = jb + (int64_t)s * cs, j1 = min(p.nb_cap, j0 + cs);
+                for (int64_t j = j0 + tid; j < j1; j += kNT) bm[j] = -INFINITY;
+            }
+        }
+    } else {  // MODE_POOL
+        const int P = p.P;
+        int ps = (P + S - 1) / S;
+        int lo = min(P, s * ps), hi = min(P, lo + ps);
+        const int32_t* pool = p.pool + (int64_t)bq * P;
+        for (int sb = lo; sb < hi; sb += kNT / kBlk) {
+            tk.make_room(k, kNT);
+            int slot = sb + tid / kBlk;
+            int blk = slot < hi ? __ldg(pool + slot) : -1;
+            int64_t e = (int64_t)blk * kBlk + (tid & (kBlk - 1));
+            bool valid = blk >= 0 && e < nvis;
+            float sc = valid ? entry_score_at(R, ik, iks, e) : 0.0f;
+            tk.offer(valid, score_key(sc), (int32_t)e);
+        }
+    }
+    tk.finish(k);
+    finalize(tk, p, bq, S, k, p.out);
+}
+
+// ---- host side -------------------------------------------------------------
+
+static int slots() { return 2 * kNumSMs; }
+
+int select_splits(int op, int B, int Q, int64_t cap, int k, int P) {
+    int64_t bq = (int64_t)B * Q;
+    int64_t by_cta = slots() / (bq > 0 ? bq : 1);
+    int64_t want;
+    if (op == CSA2_OP_INDEX_TOPK) want = (cap + 2047) / 2048;
+    else if (op == CSA2_OP_POOL_TOPK) want = ((int64_t)P * kBlk + 4095) / 4096;
+    else want = ((cap + kBlk - 1) / kBlk + 16383) / 16384;
+    int64_t S = want < by_cta ? want : by_cta;
+    if (S < 1) S = 1;
+    if (S > 1024) S = 1024;
+    return (int)S;
+}
+
+size_t select_ws_bytes(int op, int B, int Q, int64_t cap, int k, int P) {
+    int S = select_splits(op, B, Q, cap, k, P);
+    size_t bq = (size_t)B * Q;
+    size_t bytes = align256(bq * 4);                 // counters
+    if (S > 1) {
+        bytes += align256(bq * S * 4);               // share counts
+        bytes += 2 * align256(bq * S * (size_t)k * 4);  // keys, positions
+    }
+    return bytes;
+}
+
+void select_carve_ws(SelectParams& p, int S, void* ws, int B, int Q, int k) {
+    size_t bq = (size_t)B * Q;
+    char* c = (char*)ws;
+    p.counters = (int32_t*)c;
+    c += align256(bq * 4);
+    if (S > 1) {
+        p.cand_cnt = (int32_t*)c;
+        c += align256(bq * S * 4);
+        p.cand_key = (uint32_t*)c;
+        c += align256(bq * S * (size_t)k * 4);
+        p.cand_pos = (int32_t*)c;
+    }
+}
+
+cudaError_t launch_select(int op, SelectParams& p, int S, cudaStream_t st) {
+    dim3 grid(S, p.B * p.Q);
+    if (op == CSA2_OP_INDEX_TOPK) select_kernel<MODE_DENSE><<<grid, kNT, 0, st>>>(p);
+    else if (op == CSA2_OP_POOL_TOPK) select_kernel<MODE_POOL><<<grid, kNT, 0, st>>>(p);
+    else select_kernel<MODE_BUILD><<<grid, kNT, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace csa2

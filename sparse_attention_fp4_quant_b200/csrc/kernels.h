@@ -1,0 +1,80 @@
+// kernels.h -- host-visible parameter blocks and launchers of the CSA2 kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/csa2.h"
+
+namespace csa2 {
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Index Top-K (Full), pool Top-K (Reindex) and pool build share one kernel.
+struct SelectParams {
+    const uint8_t* q;
+    const uint8_t* q_sc;
+    const float* w;
+    const uint8_t* ik;
+    const uint8_t* ik_sc;
+    const int32_t* n_entries;
+    int64_t cap;
+    int m;
+    const int32_t* q_pos;
+    int B, Q, k;
+    int32_t* out;          // idx_out or pool_out [B*Q][k]
+    float* blockmax;       // index: optional output; build: input
+    int64_t nb_cap;        // ceil(cap / 8)
+    const int32_t* pool;   // pool Top-K input [B*Q][P]
+    int P;
+    // workspace
+    int32_t* counters;     // [B*Q], zero between calls
+    int32_t* cand_cnt;     // [B*Q][S]
+    uint32_t* cand_key;    // [B*Q][S][k]
+    int32_t* cand_pos;     // [B*Q][S][k]
+};
+
+int select_splits(int op, int B, int Q, int64_t cap, int k, int P);
+size_t select_ws_bytes(int op, int B, int Q, int64_t cap, int k, int P);
+void select_carve_ws(SelectParams& p, int S, void* ws, int B, int Q, int k);
+cudaError_t launch_select(int op, SelectParams& p, int S, cudaStream_t st);
+
+// NVFP4 quantisation and the indexer-K projection.
+cudaError_t launch_quant(const void* x, int64_t rows, int ch, uint8_t* codes, uint8_t* scales,
+                         const int64_t* dst_rows, int64_t out_rows, cudaStream_t st);
+cudaError_t launch_index_k_proj(const void* x, int64_t rows, const float* W, uint8_t* k_codes, uint8_t* k_scales,
+                                const int64_t* dst_rows, int64_t out_rows, cudaStream_t st);
+
+// Sparse attention.
+struct AttnParams {
+    const uint16_t* q;        // bf16 [B*Q][16][512]
+    const uint8_t* lat;
+    const uint8_t* lat_sc;
+    const int32_t* n_entries;
+    int64_t cap;
+    const int32_t* idx;       // [B*Q][k]
+    int k;
+    const uint8_t* swa;       // [B][T][512]
+    const float* swa_sc;      // [B][T]
+    const int32_t* swa_pos0;  // [B]
+    int T, window;
+    const int32_t* replay_start;
+    const int32_t* q_pos;
+    int B, Q;
+    float sm_scale;
+    uint16_t* out;            // bf16 [B*Q][16][512]
+    float* lse;               // [B*Q][16] or null
+    int slots_total;          // k + window
+    int tiles_per_split;
+    // workspace
+    int32_t* counters;        // [B*Q]
+    float* part_o;            // [B*Q][S][16][512]
+    float* part_ml;           // [B*Q][S][16][2]
+};
+
+int attn_splits(int B, int Q, int k, int window, int* tiles_per_split);
+size_t attn_ws_bytes(int B, int Q, int k, int window);
+void attn_carve_ws(AttnParams& p, int S, void* ws);
+cudaError_t launch_attn(AttnParams& p, int S, cudaStream_t st);
+
+}  // namespace csa2

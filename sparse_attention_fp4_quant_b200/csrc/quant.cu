@@ -1,0 +1,156 @@
+// quant.cu -- NVFP4 quantisation of latent rows and the indexer-K projection.
+//
+// NVFP4 here: E2M1 codes, one E4M3 scale per 16 channels, no second-level
+// scale.  scale = E4M3_rne_satfinite(fp32(amax / 6)); each code rounds
+// |x| / scale to the nearest E2M1 magnitude, ties to the even code, by
+// comparing |x| with the exact fp32 midpoints m * scale.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace csa2 {
+
+__device__ __forceinline__ void quant16(const float v[16], uint32_t& scale_byte, uint32_t& lo, uint32_t& hi) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    const uint32_t sc = f32_to_e4m3_satfinite(__fdiv_rn(amax, 6.0f));
+    const float s = e4m3_to_f32(sc);
+    // midpoints between consecutive E2M1 magnitudes, times the scale (exact)
+    const float t0 = 0.25f * s, t1 = 0.75f * s, t2 = 1.25f * s, t3 = 1.75f * s;
+    const float t4 = 2.5f * s, t5 = 3.5f * s, t6 = 5.0f * s;
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        float a = fabsf(v[j]);
+        // a tie at a midpoint goes to the even code: strict for 0.25/1.25/2.5/5, inclusive for 0.75/1.75/3.5
+        uint32_t mag = (uint32_t)(a > t0) + (uint32_t)(a >= t1) + (uint32_t)(a > t2) + (uint32_t)(a >= t3) +
+                       (uint32_t)(a > t4) + (uint32_t)(a >= t5) + (uint32_t)(a > t6);
+        uint32_t code = mag | ((__float_as_uint(v[j]) >> 31) << 3);
+        w[j >> 3] |= code << (4 * (j & 7));
+    }
+    if (s == 0.0f) w[0] = w[1] = 0u;
+    scale_byte = sc;
+    lo = w[0];
+    hi = w[1];
+}
+
+__global__ void __launch_bounds__(256) quant_kernel(const uint16_t* __restrict__ x, int64_t rows, int ch,
+                                                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                    const int64_t* __restrict__ dst_rows, int64_t out_rows) {
+    const int G = ch / 16;
+    int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= rows * G) return;
+    int64_t r = t / G;
+    int g = (int)(t - r * G);
+    const uint4* src = reinterpret_cast<const uint4*>(x + r * ch + 16 * g);
+    uint4 a = __ldg(src), b = __ldg(src + 1);
+    uint32_t u[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    float v[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        v[2 * j] = __uint_as_float(u[j] << 16);
+        v[2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
+    }
+    uint32_t sc, lo, hi;
+    quant16(v, sc, lo, hi);
+    int64_t orow = dst_rows ? __ldg(dst_rows + r) : r;
+    if (orow < 0 || orow >= out_rows) return;
+    *reinterpret_cast<uint2*>(codes + orow * (ch / 2) + 8 * g) = make_uint2(lo, hi);
+    scales[orow * G + g] = (uint8_t)sc;
+}
+
+cudaError_t launch_quant(const void* x, int64_t rows, int ch, uint8_t* codes, uint8_t* scales,
+                         const int64_t* dst_rows, int64_t out_rows, cudaStream_t st) {
+    int64_t n = rows * (ch / 16);
+    if (n == 0) return cudaSuccess;
+    int64_t blocks = (n + 255) / 256;
+    quant_kernel<<<(unsigned)blocks, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, ch, codes, scales, dst_rows,
+                                                  out_rows);
+    return cudaGetLastError();
+}
+
+// k = x W as fp32 fused multiply-add chains over the 512 channels in ascending
+// order; a 64-row x 64-output tile per CTA, 4 x 4 outputs per thread.
+constexpr int kPR = 64;   // rows per CTA
+constexpr int kPC = 32;   // channels per smem chunk
+
+__global__ void __launch_bounds__(256) index_k_proj_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                           const float* __restrict__ W, uint8_t* __restrict__ kc,
+                                                           uint8_t* __restrict__ ks,
+                                                           const int64_t* __restrict__ dst_rows, int64_t out_rows) {
+    __shared__ float xs[kPC][kPR + 4];
+    __shared__ float wsm[kPC][kID + 4];
+    __shared__ float outs[kPR][kID + 4];
+    const int tid = threadIdx.x;
+    const int ty = tid >> 4, tx = tid & 15;
+    const int64_t r0 = (int64_t)blockIdx.x * kPR;
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+
+    for (int c0 = 0; c0 < kD; c0 += kPC) {
+        // x chunk [64 rows][32 ch] -> transposed fp32
+#pragma unroll
+        for (int it = 0; it < (kPR * kPC) / 256; ++it) {
+            int e = it * 256 + tid;
+            int rr = e / kPC, cc = e % kPC;
+            int64_t row = r0 + rr;
+            float v = 0.0f;
+            if (row < rows) v = __uint_as_float(((uint32_t)__ldg(x + row * kD + c0 + cc)) << 16);
+            xs[cc][rr] = v;
+        }
+#pragma unroll
+        for (int it = 0; it < (kPC * kID) / 256; ++it) {
+            int e = it * 256 + tid;
+            int cc = e / kID, jj = e % kID;
+            wsm[cc][jj] = __ldg(W + (int64_t)(c0 + cc) * kID + jj);
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int cc = 0; cc < kPC; ++cc) {
+            float a[4], bw[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = xs[cc][ty * 4 + i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) bw[j] = wsm[cc][tx * 4 + j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = __fmaf_rn(a[i], bw[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) outs[ty * 4 + i][tx * 4 + j] = acc[i][j];
+    __syncthreads();
+    // one thread per (row, group of 16 outputs)
+    const int rr = tid >> 2, g = tid & 3;
+    const int64_t row = r0 + rr;
+    if (row < rows) {
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = outs[rr][16 * g + j];
+        uint32_t sc, lo, hi;
+        quant16(v, sc, lo, hi);
+        int64_t orow = dst_rows ? __ldg(dst_rows + row) : row;
+        if (orow >= 0 && orow < out_rows) {
+            *reinterpret_cast<uint2*>(kc + orow * 32 + 8 * g) = make_uint2(lo, hi);
+            ks[orow * 4 + g] = (uint8_t)sc;
+        }
+    }
+}
+
+cudaError_t launch_index_k_proj(const void* x, int64_t rows, const float* W, uint8_t* k_codes, uint8_t* k_scales,
+                                const int64_t* dst_rows, int64_t out_rows, cudaStream_t st) {
+    if (rows == 0) return cudaSuccess;
+    int64_t blocks = (rows + kPR - 1) / kPR;
+    index_k_proj_kernel<<<(unsigned)blocks, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, W, k_codes,
+                                                          k_scales, dst_rows, out_rows);
+    return cudaGetLastError();
+}
+
+}  // namespace csa2

@@ -1,0 +1,87 @@
+"""Shared helpers of the GPU parity tests: input builders on both sides of the boundary.
+
+Inputs come from the seeded generator (synth); the CUDA path receives them as
+device tensors and the oracle as numpy copies of the same bytes.  Nothing the
+CUDA path computes is fed to the oracle.
+"""
+import math
+
+import numpy as np
+import torch
+
+import oracle
+import synth
+
+TOL_ABS, TOL_REL = 2e-3, 1e-2   # attention: |gpu - ref| <= 2e-3 + 1e-2 |ref|
+
+
+def np_(t):
+    return t.detach().cpu().numpy()
+
+
+def bits(t):
+    return synth.bf16_bits(t)
+
+
+def attn_close(gpu_bf16, ref):
+    g = gpu_bf16.float().cpu().numpy().astype(np.float64)
+    err = np.abs(g - ref)
+    ok = err <= TOL_ABS + TOL_REL * np.abs(ref)
+    big = np.abs(ref) > 1e-2
+    stats = dict(max_abs=float(err.max()) if err.size else 0.0,
+                 max_rel=float((err[big] / np.abs(ref[big])).max()) if big.any() else 0.0)
+    return bool(ok.all()), stats
+
+
+class Group:
+    """A CSA2 layer group: bf16 latent rows (generator), the oracle's quantised
+    cache (numpy) and the CUDA path's own quantised cache (device)."""
+
+    def __init__(self, seed, B, cap, n_entries, m=1, device="cuda", latent_device=None):
+        import sparse_attention_fp4_quant_b200 as csa
+        self.B, self.cap, self.m = B, cap, m
+        latent_device = latent_device or device
+        self.latent = torch.stack([synth.latent(synth.seed_of("grp", seed, b), cap, 0, latent_device)
+                                   for b in range(B)])  # [B, cap, 512] bf16
+        self.W = synth.proj_w(seed).to(device)
+        self.n_entries = np.array(n_entries, np.int32)
+        # CUDA path: its own quantiser and projection write the cache
+        self.kv = csa.KV(B, cap, m, device)
+        lat_dev = self.latent.to(device).reshape(-1, 512)
+        csa.csa2_quant_nvfp4(lat_dev, self.kv.lat.view(-1, 256), self.kv.lat_sc.view(-1, 32))
+        csa.csa2_index_k_proj(lat_dev, self.W, self.kv.ik.view(-1, 32), self.kv.ik_sc.view(-1, 4))
+        self.kv.n_entries.copy_(torch.from_numpy(self.n_entries))
+        self._oracle = None
+
+    def oracle_cache(self):
+        if self._oracle is None:
+            lb = bits(self.latent.reshape(-1, 512))
+            lat, lat_sc = oracle.quant_nvfp4(lb)
+            ik, iks = oracle.index_k_proj(lb, np_(self.W))
+            B, cap = self.B, self.cap
+            self._oracle = dict(lat=lat.reshape(B, cap, 256), lat_sc=lat_sc.reshape(B, cap, 32),
+                                ik=ik.reshape(B, cap, 32), iks=iks.reshape(B, cap, 4))
+        return self._oracle
+
+
+def index_query(seed, B, Q, device="cuda"):
+    """Indexer query: bf16 from the generator, quantised by each side on its own."""
+    import sparse_attention_fp4_quant_b200 as csa
+    iq_bf = synth.index_q(seed, B, Q, device)
+    iq_d, iqs_d = csa.csa2_quant_nvfp4(iq_bf.reshape(-1, 64))
+    iq_o, iqs_o = oracle.quant_nvfp4(bits(iq_bf.reshape(-1, 64)))
+    w = synth.index_w(B, Q, device)
+    return (iq_d.reshape(B, Q, 128), iqs_d.reshape(B, Q, 16), w,
+            iq_o.reshape(B, Q, 128), iqs_o.reshape(B, Q, 16), np_(w))
+
+
+def swa_for(seed, B, T, pos0s, device="cuda"):
+    codes, scs = [], []
+    for b in range(B):
+        c, s = synth.swa_kv(synth.seed_of("swa", seed, b), T, int(pos0s[b]), device)
+        codes.append(c)
+        scs.append(s)
+    return torch.stack(codes), torch.stack(scs)
+
+
+SM_SCALE = 1.0 / math.sqrt(512)

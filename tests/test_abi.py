@@ -1,0 +1,71 @@
+"""The C-ABI library loads, exports every symbol include/csa2.h declares, and
+rejects invalid arguments on the host before launching anything (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "csa2.h")).read()
+    return sorted(set(re.findall(r"CSA2_API\s+[\w\s\*]+?\b(csa2_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from sparse_attention_fp4_quant_b200 import build
+    import sparse_attention_fp4_quant_b200 as csa
+    build.build()
+    return csa.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared()
+    assert len(names) >= 10
+    import sparse_attention_fp4_quant_b200 as csa
+    assert sorted(csa.EXPORTS) == names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    assert L.csa2_status_str(0) == b"CSA2_OK"
+    assert L.csa2_status_str(1) == b"CSA2_ERR_INVALID_ARG"
+    assert L.csa2_status_str(4) == b"CSA2_ERR_CUDA"
+
+
+def test_workspace_sizes_are_host_only(L):
+    import sparse_attention_fp4_quant_b200 as csa
+    for op in range(5):
+        assert L.csa2_workspace_bytes(op, 32, 1, 131072, 512, 2048) >= 256
+    assert L.csa2_workspace_bytes(0, 0, 1, 10, 512, 0) == 0
+    # one share per query needs only the counters
+    assert L.csa2_workspace_bytes(csa.OP_INDEX_TOPK, 4096, 1, 1000, 512, 0) == 4096 * 4
+
+
+def test_invalid_arguments_rejected_before_launch(L):
+    P = ctypes.c_void_p
+    fake = P(0x1000)
+    # channel count not a multiple of 16
+    assert L.csa2_quant_nvfp4(fake, 4, 15, fake, fake, None, 4, None) == 1
+    # misaligned input
+    assert L.csa2_quant_nvfp4(P(0x1001), 4, 16, fake, fake, None, 4, None) == 1
+    # output smaller than the input without a row map
+    assert L.csa2_quant_nvfp4(fake, 4, 16, fake, fake, None, 3, None) == 1
+    # rows == 0 is a no-op
+    assert L.csa2_quant_nvfp4(None, 0, 16, None, None, None, 0, None) == 0
+    import sparse_attention_fp4_quant_b200 as csa
+    kv = csa.csa2_kv(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 100, 3)  # m = 3 is invalid
+    assert L.csa2_index_topk(fake, fake, fake, ctypes.byref(kv), fake, 1, 1, 512, fake, None, fake, 1 << 20,
+                             None) == 1
+    kv.m = 1
+    assert L.csa2_index_topk(fake, fake, fake, ctypes.byref(kv), fake, 1, 1, 4096, fake, None, fake, 1 << 20,
+                             None) == 1   # k > CSA2_MAX_K
+    assert L.csa2_index_topk(fake, fake, fake, ctypes.byref(kv), fake, 1, 1, 512, fake, None, fake, 0,
+                             None) == 3   # workspace too small
+    assert L.csa2_sparse_attn(fake, ctypes.byref(kv), fake, 512, fake, fake, fake, 128, 129, None, fake, 1, 1,
+                              ctypes.c_float(0.04), fake, None, fake, 1 << 20, None) == 1   # window > 128
+    assert L.csa2_layer_step(None, None) == 1

@@ -1,0 +1,266 @@
+"""GPU parity of every call of the C ABI against the CPU oracle (small and ragged cases).
+
+Bit-exact: quantised bytes, indexer-K bytes, Top-K indices, block maxima, pools.
+Tolerance (attention, bf16 out): |gpu - ref| <= 2e-3 + 1e-2 |ref| elementwise.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_common import SM_SCALE, Group, attn_close, bits, index_query, np_, swa_for
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def csa():
+    import sparse_attention_fp4_quant_b200 as m
+    m.lib()
+    return m
+
+
+# ---------------------------------------------------------------- quantisation
+def test_quant_exhaustive_bf16(csa):
+    """Every finite bf16 pattern appears in some group, next to every kind of amax."""
+    allb = np.arange(0, 1 << 16, dtype=np.uint32)
+    finite = allb[((allb >> 7) & 0xFF) != 0xFF].astype(np.uint16)
+    rng = np.random.default_rng(0)
+    groups = []
+    for rot in range(3):
+        perm = rng.permutation(finite)
+        pad = (-perm.size) % 16
+        groups.append(np.concatenate([perm, perm[:pad]]).reshape(-1, 16))
+    x = np.concatenate(groups)
+    pad_rows = (-x.shape[0]) % 32
+    x = np.concatenate([x, x[:pad_rows]]).reshape(-1, 512)
+    xt = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    c, s = csa.csa2_quant_nvfp4(xt)
+    oc, os_ = oracle.quant_nvfp4(x)
+    assert np.array_equal(np_(s), os_)
+    assert np.array_equal(np_(c), oc)
+
+
+def test_quant_special_groups(csa):
+    vals = [0.0, -0.0, 1e-30, -1e-30, 448 * 6.0, 448 * 7.5, 3e38, -3e38, 0.25, 0.75, 1.25, 5.0, -5.0]
+    rows = []
+    for v in vals:
+        g = np.zeros(16, np.float32)
+        g[0] = v
+        g[1:] = np.float32(v) * np.array([0.5, 0.25, 0.125, 1.0, -1.0, 0.7, 0.1, 0, -0.0, 0.33, 0.9, 0.99, 0.6, 0.4,
+                                          0.2], np.float32)
+        rows.append(g)
+    x = torch.tensor(np.stack(rows)).to(torch.bfloat16).reshape(-1, 16)
+    x = torch.cat([x, torch.zeros((3, 16), dtype=torch.bfloat16)]).reshape(-1, 16)
+    xc = x.cuda().contiguous()
+    c, s = csa.csa2_quant_nvfp4(xc)
+    oc, os_ = oracle.quant_nvfp4(bits(x))
+    assert np.array_equal(np_(s), os_) and np.array_equal(np_(c), oc)
+
+
+@pytest.mark.parametrize("ch", [16, 64, 512, 4096])
+def test_quant_latents_and_dst_rows(csa, ch):
+    x = synth.normal(ch, (300, ch), "cuda").to(torch.bfloat16)
+    c, s = csa.csa2_quant_nvfp4(x)
+    oc, os_ = oracle.quant_nvfp4(bits(x))
+    assert np.array_equal(np_(c), oc) and np.array_equal(np_(s), os_)
+    # scatter into a larger buffer at given rows
+    dst = torch.randperm(1000, device="cuda")[:300].to(torch.int64)
+    big_c = torch.zeros((1000, ch // 2), dtype=torch.uint8, device="cuda")
+    big_s = torch.zeros((1000, ch // 16), dtype=torch.uint8, device="cuda")
+    csa.csa2_quant_nvfp4(x, big_c, big_s, dst)
+    assert np.array_equal(np_(big_c)[np_(dst)], oc) and np.array_equal(np_(big_s)[np_(dst)], os_)
+
+
+def test_index_k_proj_bit_exact(csa):
+    x = synth.latent(5, 1000, 0, "cuda")
+    W = synth.proj_w(3).cuda()
+    kc, ks = csa.csa2_index_k_proj(x, W)
+    oc, os_ = oracle.index_k_proj(bits(x), np_(W))
+    assert np.array_equal(np_(kc), oc) and np.array_equal(np_(ks), os_)
+    dst = (torch.arange(1000, device="cuda", dtype=torch.int64) * 3 + 1)
+    bc = torch.zeros((3001, 32), dtype=torch.uint8, device="cuda")
+    bs = torch.zeros((3001, 4), dtype=torch.uint8, device="cuda")
+    csa.csa2_index_k_proj(x, W, bc, bs, dst)
+    assert np.array_equal(np_(bc)[1::3][:1000], oc) and np.array_equal(np_(bs)[1::3][:1000], os_)
+
+
+# ---------------------------------------------------------------- index / Top-K
+def _index_case(seed, B, Q, cap, n_entries, m, q_pos, k):
+    grp = Group(seed, B, cap, n_entries, m)
+    o = grp.oracle_cache()
+    assert np.array_equal(np_(grp.kv.ik), o["ik"]) and np.array_equal(np_(grp.kv.ik_sc), o["iks"])
+    iq, iqs, w, oiq, oiqs, ow = index_query(seed + 1, B, Q)
+    assert np.array_equal(np_(iq), oiq) and np.array_equal(np_(iqs), oiqs)
+    qp = torch.tensor(q_pos, dtype=torch.int32, device="cuda")
+    return grp, o, iq, iqs, w, oiq, oiqs, ow, qp
+
+
+@pytest.mark.parametrize("m", [1, 2])
+@pytest.mark.parametrize("k", [1, 37, 512, 2048])
+def test_index_topk_ragged(csa, m, k):
+    B, Q, cap = 3, 2, 9000
+    n_entries = [9000, 4097, 1]
+    q_pos = [[9000 * m - 1, 3000], [4096 * m + 50, 511], [0, 77]]
+    grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(11 * m + k, B, Q, cap, n_entries, m, q_pos, k)
+    idx, bm = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, k, blockmax=True)
+    ridx, rbm = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, m, np.array(q_pos, np.int32), k,
+                                  blockmax=True)
+    assert np.array_equal(np_(idx), ridx)
+    assert np.array_equal(np_(bm), rbm)
+
+
+def test_index_topk_ties_and_zero_scores(csa):
+    B, Q, cap = 1, 3, 20000
+    grp = Group(21, B, cap, [20000])
+    # duplicate one key everywhere in a stripe: many exactly equal scores
+    grp.kv.ik[0, 1000:9000] = grp.kv.ik[0, 5]
+    grp.kv.ik_sc[0, 1000:9000] = grp.kv.ik_sc[0, 5]
+    o = grp.oracle_cache()
+    o = dict(o)
+    o["ik"] = o["ik"].copy()
+    o["iks"] = o["iks"].copy()
+    o["ik"][0, 1000:9000] = o["ik"][0, 5]
+    o["iks"][0, 1000:9000] = o["iks"][0, 5]
+    iq, iqs, w, oiq, oiqs, ow = index_query(22, B, Q)
+    iq[0, 2].zero_()   # query 2 scores every entry +0
+    oiq = oiq.copy()
+    oiq[0, 2] = 0
+    q_pos = np.array([[19999, 15000, 19999]], np.int32)
+    for k in (512, 2048):
+        idx = csa.csa2_index_topk(iq, iqs, w, grp.kv, torch.from_numpy(q_pos).cuda(), k)
+        ridx = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, 1, q_pos, k)
+        assert np.array_equal(np_(idx), ridx)
+        assert list(np_(idx)[0, 2]) == list(range(k))
+
+
+# ---------------------------------------------------------------- pool
+def test_pool_build_and_pool_topk(csa):
+    B, Q, cap = 2, 2, 30000
+    n_entries = [30000, 17001]
+    q_pos = [[29999, 20000], [17000, 9]]
+    grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(31, B, Q, cap, n_entries, 1, q_pos, 512)
+    idx, bm = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, 512, blockmax=True)
+    _, rbm = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, 1, np.array(q_pos, np.int32), 512,
+                               blockmax=True)
+    assert np.array_equal(np_(bm), rbm)
+    for P in (2048, 300):
+        pool = csa.csa2_pool_build(bm, grp.kv, qp, P)
+        rpool = oracle.pool_build(rbm, grp.n_entries, 1, np.array(q_pos, np.int32), P)
+        assert np.array_equal(np_(pool), rpool)
+        riq, riqs, rw, roiq, roiqs, row_ = index_query(32 + P, B, Q)
+        for k in (512, 64):
+            got = csa.csa2_pool_topk(riq, riqs, rw, grp.kv, pool, qp, k)
+            ref = oracle.pool_topk(roiq, roiqs, row_, o["ik"], o["iks"], grp.n_entries, 1, rpool,
+                                   np.array(q_pos, np.int32), k)
+            assert np.array_equal(np_(got), ref)
+
+
+# ---------------------------------------------------------------- attention
+def _attn_case(csa, seed, B, Q, cap, n_entries, k, T, window, q_pos, pos0, replay, idx_np):
+    grp = Group(seed, B, cap, n_entries)
+    o = grp.oracle_cache()
+    assert np.array_equal(np_(grp.kv.lat), o["lat"]) and np.array_equal(np_(grp.kv.lat_sc), o["lat_sc"])
+    q = synth.attn_q(seed, B, Q, "cuda")
+    swa, swa_sc = swa_for(seed, B, T, pos0)
+    qp = torch.tensor(q_pos, dtype=torch.int32, device="cuda")
+    p0 = torch.tensor(pos0, dtype=torch.int32, device="cuda")
+    rs = None if replay is None else torch.tensor(replay, dtype=torch.int32, device="cuda")
+    idx = torch.from_numpy(idx_np).cuda()
+    out, lse = csa.csa2_sparse_attn(q, grp.kv, idx, swa, swa_sc, p0, qp, window, rs, SM_SCALE, lse=True)
+    ref, rlse = oracle.sparse_attn(bits(q), o["lat"], o["lat_sc"], grp.n_entries, idx_np, np_(swa), np_(swa_sc),
+                                   np.array(pos0, np.int32), window, None if replay is None else np.array(replay, np.int32),
+                                   np.array(q_pos, np.int32), SM_SCALE)
+    ok, st = attn_close(out, ref)
+    assert ok, st
+    fin = np.isfinite(rlse)
+    assert np.array_equal(fin, np.isfinite(np_(lse)))
+    assert np.allclose(np_(lse)[fin], rlse[fin], rtol=1e-4, atol=1e-4)
+    return st
+
+
+@pytest.mark.parametrize("B,Q", [(1, 1), (3, 2), (32, 1)])
+def test_sparse_attn_decode(csa, B, Q):
+    cap, k, T = 5000, 512, 128
+    rng = np.random.default_rng(B * 10 + Q)
+    n_entries = [5000 - 7 * b for b in range(B)]
+    idx = np.sort(rng.integers(0, 4990, (B, Q, k)), axis=-1).astype(np.int32)
+    idx[:, :, -20:] = -1
+    q_pos = [[n_entries[b] - 1 - qi for qi in range(Q)] for b in range(B)]
+    pos0 = [n_entries[b] - T for b in range(B)]
+    _attn_case(csa, 40 + B, B, Q, cap, n_entries, k, T, 128, q_pos, pos0, None, idx)
+
+
+@pytest.mark.parametrize("window", [1, 2, 4, 77, 128])
+def test_sparse_attn_replay_mask(csa, window):
+    B, Q, cap, k, T = 2, 128, 3000, 64, 128
+    rng = np.random.default_rng(window)
+    s = [3000 - 128, 2500]
+    q_pos = [[s[b] + qi for qi in range(Q)] for b in range(B)]
+    pos0 = [s[0], s[1] - 3]
+    idx = np.sort(rng.integers(0, 2900, (B, Q, k)), axis=-1).astype(np.int32)
+    _attn_case(csa, 50 + window, B, Q, cap, [3000, 2900], k, T, window, q_pos, pos0, s, idx)
+
+
+def test_sparse_attn_edge_cases(csa):
+    B, Q, cap = 2, 3, 600
+    # k = 0 (SWA only); T = 0 (main only); query with nothing visible -> zeros
+    rng = np.random.default_rng(7)
+    idx = np.full((B, Q, 0), -1, np.int32)
+    _attn_case(csa, 60, B, Q, cap, [600, 600], 0, 16, 128, [[599, 598, 10], [599, 300, 599]], [584, 584], None, idx)
+    idx = rng.integers(-5, 700, (B, Q, 100)).astype(np.int32)   # padding and out-of-range ids
+    _attn_case(csa, 61, B, Q, cap, [600, 321], 100, 0, 128, [[599, 598, 10], [599, 300, 599]], [0, 0], None, idx)
+    idx = np.full((B, Q, 8), -1, np.int32)
+    _attn_case(csa, 62, B, Q, cap, [600, 600], 8, 4, 128, [[599, 5000, 599], [10, 300, 599]], [0, 0], None, idx)
+
+
+# ---------------------------------------------------------------- layer dispatch
+def test_layer_dispatch_decoder_pattern(csa):
+    """The decoder pattern F R R R (X R R R) x 4 through csa2_layer_step equals the
+    oracle's layer composition (bit-exact indices; attention within tolerance)."""
+    B, Q, cap, T = 2, 1, 6000, 128
+    n_before = [5000, 4321]
+    grp = Group(70, B, cap, n_before)
+    o = {kk: v.copy() for kk, v in grp.oracle_cache().items()}
+    # the new token of this step: appended by the Full layer at position n_before[b]
+    new_lat = torch.stack([synth.latent(synth.seed_of("new", 70, b), 1, n_before[b], "cuda")[0] for b in range(B)])
+    new_rows = torch.tensor([b * cap + n_before[b] for b in range(B)], dtype=torch.int64, device="cuda")
+    nb = bits(new_lat)
+    olat, olsc = oracle.quant_nvfp4(nb)
+    oik, oiks = oracle.index_k_proj(nb, np_(grp.W))
+    n_after = np.array(n_before, np.int32) + 1
+    for b in range(B):
+        o["lat"][b, n_before[b]] = olat[b]
+        o["lat_sc"][b, n_before[b]] = olsc[b]
+        o["ik"][b, n_before[b]] = oik[b]
+        o["iks"][b, n_before[b]] = oiks[b]
+    grp.kv.n_entries.copy_(torch.from_numpy(n_after))
+    q_pos_np = (n_after - 1).reshape(B, 1).astype(np.int32)
+    qp = torch.from_numpy(q_pos_np).cuda()
+    idx = torch.zeros((B, Q, 512), dtype=torch.int32, device="cuda")
+    pool = torch.zeros((B, Q, 2048), dtype=torch.int32, device="cuda")
+    bm = torch.zeros((B, Q, (cap + 7) // 8), dtype=torch.float32, device="cuda")
+    st = dict(lat=o["lat"], lat_sc=o["lat_sc"], ik=o["ik"], iks=o["iks"], n_entries=n_after, m=1, k=512,
+              build_pool=True, pool_blocks=2048)
+    for li, mode in enumerate(oracle.DECODER_PATTERN):
+        q = synth.attn_q(synth.seed_of("layer-q", li), B, Q, "cuda")
+        pos0 = n_after - T
+        swa, swa_sc = swa_for(synth.seed_of("layer-swa", li), B, T, pos0)
+        p0 = torch.from_numpy(pos0.astype(np.int32)).cuda()
+        iq = iqs = w = oiq = oiqs = ow = None
+        if mode != "reuse":
+            iq, iqs, w, oiq, oiqs, ow = index_query(synth.seed_of("layer-iq", li), B, Q)
+        first = li == 0
+        out = csa.csa2_layer_step(mode, grp.kv, qp, q, swa, swa_sc, p0, idx, 512, iq, iqs, w,
+                                  pool=pool, blockmax=bm, new_latent=new_lat if first else None,
+                                  new_rows=new_rows if first else None, k_proj=grp.W)
+        layer = dict(q=bits(q), iq=oiq, iqs=oiqs, w=ow, swa=np_(swa), swa_sc=np_(swa_sc), swa_pos0=pos0.astype(np.int32),
+                     window=128, q_pos=q_pos_np)
+        ref, _ = oracle.layer_step(mode, st, layer)
+        if first:
+            assert np.array_equal(np_(grp.kv.lat), o["lat"]) and np.array_equal(np_(grp.kv.ik), o["ik"])
+            assert np.array_equal(np_(pool), st["pool"])
+        assert np.array_equal(np_(idx), st["idx"]), (li, mode)
+        ok, stats = attn_close(out, ref)
+        assert ok, (li, mode, stats)
