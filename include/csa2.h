@@ -280,6 +280,36 @@ typedef struct csa2_layer_args {
 
 CSA2_API csa2_status csa2_layer_step(const csa2_layer_args* a, void* stream);
 
+/*
+ * csa2_index_topk without a caller-provided workspace.  The pages have no
+ * counterpart to this call: it exists for callers that cannot allocate device
+ * memory -- hosts whose device memory is owned by their own pool allocator and
+ * that hand out no scratch buffers, or latency-critical paths where a
+ * cudaMalloc (which can synchronise the device) is not allowed.
+ *
+ * Arguments, results and errors are those of csa2_index_topk, minus ws and
+ * ws_bytes.  The scratch the call needs (the merge counters and the candidate
+ * lists of the per-query shares) lives in one static device array of
+ * CSA2_NOALLOC_SCRATCH_BYTES inside this library; every GPU that loads the
+ * library holds that array until the process exits.  A call whose scratch would
+ * exceed the array (csa2_workspace_bytes(CSA2_OP_INDEX_TOPK, B, Q, cap, k, 0) >
+ * CSA2_NOALLOC_SCRATCH_BYTES) returns CSA2_ERR_WORKSPACE and launches nothing.
+ * The call allocates nothing: no cudaMalloc, cudaFree or allocating library
+ * routine; it clears the counters with cudaMemsetAsync on `stream` and then
+ * launches the same kernel as csa2_index_topk.
+ *
+ * The first call on each device looks up the array's device address with that
+ * device current (cudaGetSymbolAddress); make that first call before any stream
+ * capture.  All calls share the one array, which keeps the last call's contents:
+ * calls that overlap on the GPU (other streams, other host threads) race on it
+ * and must be ordered by the caller.
+ */
+#define CSA2_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+CSA2_API csa2_status csa2_index_topk_noalloc(const uint8_t* q, const uint8_t* q_sc, const float* w,
+                                             const csa2_kv* kv, const int32_t* q_pos, int32_t B, int32_t Q,
+                                             int32_t k, int32_t* idx_out, float* blockmax_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -45,7 +45,9 @@ class csa2_layer_args(ctypes.Structure):
 
 _lib = None
 EXPORTS = ["csa2_status_str", "csa2_last_cuda_error", "csa2_quant_nvfp4", "csa2_index_k_proj", "csa2_index_topk",
-           "csa2_pool_build", "csa2_pool_topk", "csa2_sparse_attn", "csa2_workspace_bytes", "csa2_layer_step"]
+           "csa2_pool_build", "csa2_pool_topk", "csa2_sparse_attn", "csa2_workspace_bytes", "csa2_layer_step",
+           "csa2_index_topk_noalloc"]
+NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 def lib():
@@ -70,6 +72,7 @@ def lib():
                                             P, P, P, sz, P]),
         "csa2_workspace_bytes": (sz, [ctypes.c_int, i32, i32, i64, i32, i32]),
         "csa2_layer_step": (ctypes.c_int, [ctypes.POINTER(csa2_layer_args), P]),
+        "csa2_index_topk_noalloc": (ctypes.c_int, [P, P, P, KVP, P, i32, i32, i32, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -194,6 +197,25 @@ def csa2_index_topk(q, q_sc, w, kv, q_pos, k, idx_out=None, blockmax=False, ws=N
     ws = _workspace(nbytes) if ws is None else ws
     _check(lib().csa2_index_topk(_ptr(q), _ptr(q_sc), _ptr(w), kv.c(), _ptr(q_pos), B, Q, k, _ptr(idx_out),
                                  _ptr(bm), _ptr(ws), ws.numel(), _stream()))
+    return (idx_out, bm) if bm is not None else idx_out
+
+
+def csa2_index_topk_noalloc(q, q_sc, w, kv, q_pos, k, idx_out=None, blockmax=False):
+    """csa2_index_topk for callers that cannot allocate device memory: the scratch is the
+    library's own static device array (CSA2_NOALLOC_SCRATCH_BYTES per GPU); calls that overlap
+    on the GPU race on it."""
+    B, Q = q_pos.shape
+    for t, dt, n in ((q, torch.uint8, "q"), (q_sc, torch.uint8, "q_sc"), (w, torch.float32, "w"),
+                     (q_pos, torch.int32, "q_pos")):
+        _dev(t, dt, n)
+    if idx_out is None:
+        idx_out = torch.empty((B, Q, k), dtype=torch.int32, device=q.device)
+    bm = None
+    if blockmax is not False:
+        bm = blockmax if isinstance(blockmax, torch.Tensor) else torch.empty(
+            (B, Q, (kv.cap + BLOCK - 1) // BLOCK), dtype=torch.float32, device=q.device)
+    _check(lib().csa2_index_topk_noalloc(_ptr(q), _ptr(q_sc), _ptr(w), kv.c(), _ptr(q_pos), B, Q, k, _ptr(idx_out),
+                                         _ptr(bm), _stream()))
     return (idx_out, bm) if bm is not None else idx_out
 
 

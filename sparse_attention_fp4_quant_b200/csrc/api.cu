@@ -46,6 +46,10 @@ SelectParams select_params(const csa2_kv* kv, const int32_t* q_pos, int B, int Q
 
 }  // namespace
 
+namespace csa2 {
+void record_cuda_error(int e) { g_last_cuda_error = e; }
+}  // namespace csa2
+
 extern "C" {
 
 const char* csa2_status_str(csa2_status s) {

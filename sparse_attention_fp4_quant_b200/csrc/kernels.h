@@ -10,6 +10,9 @@ namespace csa2 {
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Record a CUDA error for csa2_last_cuda_error() (this host thread).
+void record_cuda_error(int e);
+
 // Index Top-K (Full), pool Top-K (Reindex) and pool build share one kernel.
 struct SelectParams {
     const uint8_t* q;
