@@ -21,6 +21,7 @@ namespace csa2 {
 constexpr int kAT = 128;      // threads per CTA (4 warps)
 constexpr int kKT = 64;       // keys per tile
 constexpr int kRowB = kD * 2; // bytes per bf16 row of 512
+constexpr int kMaxSplits = (CSA2_MAX_K + CSA2_MAX_WINDOW + kKT - 1) / kKT;
 
 struct AttnSmem {
     uint8_t K[kKT * kRowB];   // 64 KB, 16-byte chunks XOR-swizzled by row & 7
@@ -32,6 +33,7 @@ struct AttnSmem {
     float red_max[4][kH];
     float red_sum[4][kH];
     float m_run[kH], l_run[kH], alpha[kH];
+    float cw[kMaxSplits][kH];  // combine weights 2^(m_s - M) / L per split and head
     int last;
 };
 
@@ -344,34 +346,48 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
     __syncthreads();
     if (!sm.last) return;
     __threadfence();
-    // combine the S partials: weights 2^(m_s - M), normaliser sum_s l_s 2^(m_s - M)
+    // combine the S partials: weight 2^(m_s - M) / L with L = sum_s l_s 2^(m_s - M)
     if (tid < kH) {
         float M = -INFINITY;
         for (int c = 0; c < S; ++c) M = fmaxf(M, __ldcg(p.part_ml + (((int64_t)bq * S + c) * kH + tid) * 2));
-        float Mu = (M == -INFINITY) ? 0.0f : M;
+        const float Mu = (M == -INFINITY) ? 0.0f : M;
         float L = 0.0f;
         for (int c = 0; c < S; ++c) {
             const float* pml = p.part_ml + (((int64_t)bq * S + c) * kH + tid) * 2;
-            float wgt = exp2f(__ldcg(pml) - Mu);
+            const float wgt = exp2f(__ldcg(pml) - Mu);
+            sm.cw[c][tid] = wgt;
             L += __ldcg(pml + 1) * wgt;
         }
-        sm.m_run[tid] = Mu;
-        sm.l_run[tid] = L;
+        const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+        for (int c = 0; c < S; ++c) sm.cw[c][tid] *= inv;
         if (p.lse) p.lse[(int64_t)bq * kH + tid] = L > 0.0f ? (Mu + log2f(L)) * LN2 : -INFINITY;
     }
     __syncthreads();
-    for (int e = tid; e < kH * kD / 2; e += kAT) {
-        int h = (2 * e) / kD, d = (2 * e) % kD;
-        float L = sm.l_run[h], Mu = sm.m_run[h];
-        float a0 = 0.0f, a1 = 0.0f;
+    {
+        // thread owns 16 float4 of the [16][512] output: element 4 (tid + 128 j)
+        constexpr int kV = kH * kD / 4 / kAT;   // 16
+        float4 acc[kV];
+#pragma unroll
+        for (int j = 0; j < kV; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int c = 0; c < S; ++c) {
-            float wgt = exp2f(__ldcg(p.part_ml + (((int64_t)bq * S + c) * kH + h) * 2) - Mu);
-            float2 v = __ldcg(reinterpret_cast<const float2*>(p.part_o + ((int64_t)bq * S + c) * kH * kD + h * kD + d));
-            a0 += v.x * wgt;
-            a1 += v.y * wgt;
+            const float4* src = reinterpret_cast<const float4*>(p.part_o + ((int64_t)bq * S + c) * kH * kD);
+#pragma unroll
+            for (int j = 0; j < kV; ++j) {
+                const int e4 = tid + kAT * j;
+                const float wgt = sm.cw[c][(4 * e4) / kD];
+                const float4 v = __ldcg(src + e4);
+                acc[j].x += v.x * wgt;
+                acc[j].y += v.y * wgt;
+                acc[j].z += v.z * wgt;
+                acc[j].w += v.w * wgt;
+            }
         }
-        float inv = L > 0.0f ? 1.0f / L : 0.0f;
-        *reinterpret_cast<uint32_t*>(p.out + (int64_t)bq * kH * kD + h * kD + d) = pack_bf16(a0 * inv, a1 * inv);
+        uint16_t* out = p.out + (int64_t)bq * kH * kD;
+#pragma unroll
+        for (int j = 0; j < kV; ++j) {
+            const int e4 = tid + kAT * j;
+            *reinterpret_cast<uint2*>(out + 4 * e4) = make_uint2(pack_bf16(acc[j].x, acc[j].y), pack_bf16(acc[j].z, acc[j].w));
+        }
     }
     if (tid == 0) p.counters[bq] = 0;
 }

@@ -81,12 +81,11 @@ enum { MODE_DENSE = 0, MODE_POOL = 1, MODE_BUILD = 2 };
 __device__ void finalize(TK& tk, const SelectParams& p, int bq, int S, int k, int32_t* out) {
     const int tid = threadIdx.x;
     if (S > 1) {
-        TK::Smem& sm = tk.s;
-        int cnt = sm.count;
+        int cnt = tk.count();
         int64_t off = ((int64_t)bq * S + blockIdx.x) * k;
         for (int i = tid; i < cnt; i += kNT) {
-            p.cand_key[off + i] = sm.key[i];
-            p.cand_pos[off + i] = sm.pos[i];
+            p.cand_key[off + i] = tk.key_at(i);
+            p.cand_pos[off + i] = tk.pos_at(i);
         }
         if (tid == 0) p.cand_cnt[(int64_t)bq * S + blockIdx.x] = cnt;
         __threadfence();
@@ -112,15 +111,15 @@ __device__ void finalize(TK& tk, const SelectParams& p, int bq, int S, int k, in
         tk.finish(k);
         if (tid == 0) p.counters[bq] = 0;
     }
-    int cnt = tk.s.count;
+    int cnt = tk.count();
     tk.sort_positions(cnt);
-    for (int i = tid; i < k; i += kNT) out[(int64_t)bq * k + i] = i < cnt ? tk.s.pos[i] : -1;
+    for (int i = tid; i < k; i += kNT) out[(int64_t)bq * k + i] = i < cnt ? tk.pos_at(i) : -1;
 }
 
 template <int MODE>
 __global__ void __launch_bounds__(kNT, 2) select_kernel(SelectParams p) {
-    __shared__ TK::Smem sm;
-    TK tk(sm);
+    extern __shared__ __align__(16) uint8_t select_smem[];
+    TK tk(*reinterpret_cast<TK::Smem*>(select_smem));
     const int tid = threadIdx.x;
     const int bq = blockIdx.y;
     const int s = blockIdx.x, S = gridDim.x;
@@ -228,6 +227,7 @@ size_t select_ws_bytes(int op, int B, int Q, int64_t cap, int k, int P) {
     int S = select_splits(op, B, Q, cap, k, P);
     size_t bq = (size_t)B * Q;
     size_t bytes = align256(bq * 4);                 // counters
+    bytes += 256;                                    // status word
     if (S > 1) {
         bytes += align256(bq * S * 4);               // share counts
         bytes += 2 * align256(bq * S * (size_t)k * 4);  // keys, positions
@@ -240,6 +240,8 @@ void select_carve_ws(SelectParams& p, int S, void* ws, int B, int Q, int k) {
     char* c = (char*)ws;
     p.counters = (int32_t*)c;
     c += align256(bq * 4);
+    p.status = (int32_t*)c;
+    c += 256;
     if (S > 1) {
         p.cand_cnt = (int32_t*)c;
         c += align256(bq * S * 4);
@@ -250,10 +252,21 @@ void select_carve_ws(SelectParams& p, int S, void* ws, int B, int Q, int k) {
 }
 
 cudaError_t launch_select(int op, SelectParams& p, int S, cudaStream_t st) {
+    if ((op == CSA2_OP_INDEX_TOPK || op == CSA2_OP_POOL_TOPK) && index_tc_supported(p)) return launch_index_tc(op, p, S, st);
     dim3 grid(S, p.B * p.Q);
-    if (op == CSA2_OP_INDEX_TOPK) select_kernel<MODE_DENSE><<<grid, kNT, 0, st>>>(p);
-    else if (op == CSA2_OP_POOL_TOPK) select_kernel<MODE_POOL><<<grid, kNT, 0, st>>>(p);
-    else select_kernel<MODE_BUILD><<<grid, kNT, 0, st>>>(p);
+    const int smem = (int)sizeof(TK::Smem);
+    static bool attr[3] = {false, false, false};
+    const int mode = op == CSA2_OP_INDEX_TOPK ? 0 : (op == CSA2_OP_POOL_TOPK ? 1 : 2);
+    if (!attr[mode]) {
+        cudaError_t e = mode == 0   ? cudaFuncSetAttribute(select_kernel<MODE_DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+                        : mode == 1 ? cudaFuncSetAttribute(select_kernel<MODE_POOL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+                                    : cudaFuncSetAttribute(select_kernel<MODE_BUILD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        attr[mode] = true;
+    }
+    if (mode == 0) select_kernel<MODE_DENSE><<<grid, kNT, smem, st>>>(p);
+    else if (mode == 1) select_kernel<MODE_POOL><<<grid, kNT, smem, st>>>(p);
+    else select_kernel<MODE_BUILD><<<grid, kNT, smem, st>>>(p);
     return cudaGetLastError();
 }
 

@@ -32,6 +32,7 @@ struct SelectParams {
     int P;
     // workspace
     int32_t* counters;     // [B*Q], zero between calls
+    int32_t* status;       // sticky: set to 1 if a device-side wait timed out
     int32_t* cand_cnt;     // [B*Q][S]
     uint32_t* cand_key;    // [B*Q][S][k]
     int32_t* cand_pos;     // [B*Q][S][k]
@@ -41,6 +42,8 @@ int select_splits(int op, int B, int Q, int64_t cap, int k, int P);
 size_t select_ws_bytes(int op, int B, int Q, int64_t cap, int k, int P);
 void select_carve_ws(SelectParams& p, int S, void* ws, int B, int Q, int k);
 cudaError_t launch_select(int op, SelectParams& p, int S, cudaStream_t st);
+bool index_tc_supported(const SelectParams& p);
+cudaError_t launch_index_tc(int op, SelectParams& p, int S, cudaStream_t st);
 
 // NVFP4 quantisation and the indexer-K projection.
 cudaError_t launch_quant(const void* x, int64_t rows, int ch, uint8_t* codes, uint8_t* scales,

@@ -144,9 +144,52 @@ __global__ void __launch_bounds__(256) index_k_proj_kernel(const uint16_t* __res
     }
 }
 
+// Few rows (a decode append): one thread per (row, output) runs its 512-long
+// FMA chain, 4 rows per CTA; the 64 outputs of a row are then quantised from
+// shared memory by 4 threads.
+__global__ void __launch_bounds__(256) index_k_proj_rows_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                                const float* __restrict__ W, uint8_t* __restrict__ kc,
+                                                                uint8_t* __restrict__ ks,
+                                                                const int64_t* __restrict__ dst_rows, int64_t out_rows) {
+    __shared__ float outs[4][kID];
+    const int tid = threadIdx.x;
+    const int rr = tid >> 6, j = tid & 63;
+    const int64_t row = (int64_t)blockIdx.x * 4 + rr;
+    if (row < rows) {
+        const uint16_t* xr = x + row * kD;
+        float acc = 0.0f;
+#pragma unroll 16
+        for (int c = 0; c < kD; ++c)
+            acc = __fmaf_rn(__uint_as_float(((uint32_t)__ldg(xr + c)) << 16), __ldg(W + c * kID + j), acc);
+        outs[rr][j] = acc;
+    }
+    __syncthreads();
+    if (tid < 16) {
+        const int r2 = tid >> 2, g = tid & 3;
+        const int64_t row2 = (int64_t)blockIdx.x * 4 + r2;
+        if (row2 < rows) {
+            float v[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) v[q] = outs[r2][16 * g + q];
+            uint32_t sc, lo, hi;
+            quant16(v, sc, lo, hi);
+            const int64_t orow = dst_rows ? __ldg(dst_rows + row2) : row2;
+            if (orow >= 0 && orow < out_rows) {
+                *reinterpret_cast<uint2*>(kc + orow * 32 + 8 * g) = make_uint2(lo, hi);
+                ks[orow * 4 + g] = (uint8_t)sc;
+            }
+        }
+    }
+}
+
 cudaError_t launch_index_k_proj(const void* x, int64_t rows, const float* W, uint8_t* k_codes, uint8_t* k_scales,
                                 const int64_t* dst_rows, int64_t out_rows, cudaStream_t st) {
     if (rows == 0) return cudaSuccess;
+    if (rows <= 2048) {
+        index_k_proj_rows_kernel<<<(unsigned)((rows + 3) / 4), 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, W,
+                                                                             k_codes, k_scales, dst_rows, out_rows);
+        return cudaGetLastError();
+    }
     int64_t blocks = (rows + kPR - 1) / kPR;
     index_k_proj_kernel<<<(unsigned)blocks, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, W, k_codes,
                                                           k_scales, dst_rows, out_rows);

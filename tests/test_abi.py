@@ -43,7 +43,7 @@ def test_workspace_sizes_are_host_only(L):
         assert L.csa2_workspace_bytes(op, 32, 1, 131072, 512, 2048) >= 256
     assert L.csa2_workspace_bytes(0, 0, 1, 10, 512, 0) == 0
     # one share per query needs only the counters
-    assert L.csa2_workspace_bytes(csa.OP_INDEX_TOPK, 4096, 1, 1000, 512, 0) == 4096 * 4
+    assert L.csa2_workspace_bytes(csa.OP_INDEX_TOPK, 4096, 1, 1000, 512, 0) == 4096 * 4 + 256  # counters + status word
 
 
 def test_invalid_arguments_rejected_before_launch(L):
