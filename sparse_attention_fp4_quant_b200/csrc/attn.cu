@@ -4,21 +4,23 @@
 // Key slots of a query: [0, k) are the main rows idx[0..k), [k, k + W) are the
 // window tokens i - W + 1 .. i.  A slot is live if its row exists and (for the
 // window) the token lies in [max(s, i - W + 1), i] and in the stored SWA rows.
-// A CTA takes a split of the slot range in tiles of 64 keys: the tile is
-// gathered and dequantised to bf16 in swizzled shared memory (K = V), S = Q K^T
-// and O += P V run on warp-level tensor-core MMAs with the 16 heads as the M
-// dimension, and the softmax is online across tiles.  FP4 rows dequantise
-// exactly to bf16; an SWA row is stored as its E4M3 values (exact in bf16) and
-// its fp32 token scale multiplies the logit and the probability instead.  P
-// enters the P V product as two bf16 terms (rounded value + remainder), so the
-// product carries about 16 bits of P rather than 8.
-// Splits of one query are merged by the last CTA to finish (atomic ticket).
+// A CTA (8 warps) takes a split of the slot range in tiles of 64 keys.  Each
+// tile is gathered into registers one tile ahead (its loads overlap the
+// previous tile's math), dequantised to bf16 in swizzled shared memory (K = V),
+// and S = Q K^T (8 keys per warp) and O += P V (64 dims per warp) run on
+// warp-level tensor-core MMAs with the 16 heads as the M dimension; the softmax
+// is online across tiles.  FP4 rows dequantise exactly to bf16 (byte-table
+// decode, then an exact bf16 multiply by the block scale); an SWA row is kept
+// as its E4M3 values (exact in bf16) and its fp32 token scale multiplies the
+// logit and the probability instead.  P enters P V as two bf16 terms (rounded
+// value + remainder), about 16 bits of P.  Splits of one query are merged by
+// the last CTA to finish (atomic ticket).
 #include "common.cuh"
 #include "kernels.h"
 
 namespace csa2 {
 
-constexpr int kAT = 128;      // threads per CTA (4 warps)
+constexpr int kAT = 256;      // threads per CTA (8 warps)
 constexpr int kKT = 64;       // keys per tile
 constexpr int kRowB = kD * 2; // bytes per bf16 row of 512
 constexpr int kMaxSplits = (CSA2_MAX_K + CSA2_MAX_WINDOW + kKT - 1) / kKT;
@@ -26,12 +28,12 @@ constexpr int kMaxSplits = (CSA2_MAX_K + CSA2_MAX_WINDOW + kKT - 1) / kKT;
 struct AttnSmem {
     uint8_t K[kKT * kRowB];   // 64 KB, 16-byte chunks XOR-swizzled by row & 7
     uint8_t Qs[kH * kRowB];   // 16 KB, same swizzle
-    uint8_t P[kH * kKT * 2];  // 2 KB, bf16 P (rounded), same swizzle over 8 chunks per row
+    uint8_t P[kH * kKT * 2];  // 2 KB, bf16 P (rounded), 8 chunks per row, same swizzle
     uint8_t Pl[kH * kKT * 2]; // 2 KB, bf16 remainder P - rounded(P)
     float kf[kKT];            // per-key factor (1 for FP4 rows, token scale for SWA)
     int kvalid[kKT];
-    float red_max[4][kH];
-    float red_sum[4][kH];
+    float red_max[8][kH];
+    float red_sum[8][kH];
     float m_run[kH], l_run[kH], alpha[kH];
     float cw[kMaxSplits][kH];  // combine weights 2^(m_s - M) / L per split and head
     int last;
@@ -44,12 +46,29 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// 8 E2M1 codes (nibble n = dim n) times the block scale -> 8 bf16 (exact).
-__device__ __forceinline__ uint4 fp4x8_to_bf16(uint32_t w, float s) {
-    uint32_t o[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) o[j] = pack_bf16(e2m1_to_f32(w >> (8 * j)) * s, e2m1_to_f32(w >> (8 * j + 4)) * s);
-    return make_uint4(o[0], o[1], o[2], o[3]);
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+    __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// 8 E2M1 codes (nibble n = dim n) times the block scale (bf16x2 s2) -> 8 bf16.
+// The magnitudes come from byte tables (high and low byte of the bf16 value),
+// the sign is moved to bit 15 of each half, and the product with the scale is
+// exact (at most 6 significant bits).
+__device__ __forceinline__ uint4 fp4x8_to_bf16(uint32_t w, uint32_t s2) {
+    const uint32_t HI0 = 0x3F3F3F00u, HI1 = 0x40404040u;   // 0 .5 1 1.5 | 2 3 4 6: high bytes
+    const uint32_t LO0 = 0xC0800000u, LO1 = 0xC0804000u;   //                     low bytes
+    const uint32_t m = w & 0x77777777u, mh = m >> 16;
+    const uint32_t hi_a = __byte_perm(HI0, HI1, m), lo_a = __byte_perm(LO0, LO1, m);
+    const uint32_t hi_b = __byte_perm(HI0, HI1, mh), lo_b = __byte_perm(LO0, LO1, mh);
+    uint32_t v0 = __byte_perm(lo_a, hi_a, 0x5140), v1 = __byte_perm(lo_a, hi_a, 0x7362);
+    uint32_t v2 = __byte_perm(lo_b, hi_b, 0x5140), v3 = __byte_perm(lo_b, hi_b, 0x7362);
+    // nibble signs (bits 3 and 7 of each byte) -> bits 15 and 31 of the bf16 pair
+    v0 |= ((w & 0x88u) * 0x1001000u) & 0x80008000u;
+    v1 |= (((w >> 8) & 0x88u) * 0x1001000u) & 0x80008000u;
+    v2 |= (((w >> 16) & 0x88u) * 0x1001000u) & 0x80008000u;
+    v3 |= (((w >> 24) & 0x88u) * 0x1001000u) & 0x80008000u;
+    return make_uint4(bf16x2_mul(v0, s2), bf16x2_mul(v1, s2), bf16x2_mul(v2, s2), bf16x2_mul(v3, s2));
 }
 
 // 4 E4M3 bytes -> 4 bf16 (exact).
@@ -65,6 +84,10 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r
                  : "r"(addr));
 }
 
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+
 __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
@@ -78,6 +101,76 @@ __device__ __forceinline__ void mma_bf16(float c[4], uint32_t a0, uint32_t a1, u
         "{%0,%1,%2,%3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One quarter (128 dims) of one key row, held in registers between its load
+// and its dequantisation.
+struct RowQuarter {
+    uint4 raw[8];   // FP4: raw[0..3] = 64 code bytes; FP8: raw[0..7] = 128 bytes
+    uint2 sc;       // FP4: the 8 block scales of the quarter
+    float fac;      // FP8: the token scale
+    int kind;       // 0 = dead slot, 1 = FP4 main row, 2 = FP8 window row
+};
+
+__device__ __forceinline__ void fetch_quarter(const AttnParams& p, int bq, int b, int tile, int r, int qq, int64_t i_pos,
+                                              int64_t lo, int64_t pos0, int64_t nmain, RowQuarter& q) {
+    q.kind = 0;
+    const int slot = tile * kKT + r;
+    if (slot < p.k) {
+        const int32_t e = __ldg(p.idx + (int64_t)bq * p.k + slot);
+        if (e >= 0 && e < nmain) {
+            q.kind = 1;
+            const int64_t row = (int64_t)b * p.cap + e;
+            const uint4* cs = reinterpret_cast<const uint4*>(p.lat + row * (kD / 2) + 64 * qq);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) q.raw[v] = __ldg(cs + v);
+            q.sc = __ldg(reinterpret_cast<const uint2*>(p.lat_sc + row * (kD / 16) + 8 * qq));
+        }
+    } else if (slot < p.slots_total) {
+        const int64_t tau = i_pos - p.window + 1 + (slot - p.k);
+        const int64_t rr = tau - pos0;
+        if (tau >= lo && tau <= i_pos && rr >= 0 && rr < p.T) {
+            q.kind = 2;
+            const int64_t row = (int64_t)b * p.T + rr;
+            q.fac = __ldg(p.swa_sc + row);
+            const uint4* cs = reinterpret_cast<const uint4*>(p.swa + row * kD + 128 * qq);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) q.raw[v] = __ldg(cs + v);
+        }
+    }
+}
+
+__device__ __forceinline__ void store_quarter(AttnSmem& sm, int r, int qq, const RowQuarter& q) {
+    if (q.kind == 1) {
+        const uint32_t scw[2] = {q.sc.x, q.sc.y};
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const uint32_t ws[4] = {q.raw[v].x, q.raw[v].y, q.raw[v].z, q.raw[v].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int word = 4 * v + j;             // 8 dims per word
+                const int sb = word >> 1;               // one scale per 16 dims
+                const float s = e4m3_to_f32((scw[sb >> 2] >> (8 * (sb & 3))) & 0xFFu);
+                const uint32_t s2 = pack_bf16(s, s);   // exact (E4M3 fits bf16)
+                *reinterpret_cast<uint4*>(sm.K + swz(r, 16 * qq + word)) = fp4x8_to_bf16(ws[j], s2);
+            }
+        }
+    } else if (q.kind == 2) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            const uint2 a = fp8x4_to_bf16(q.raw[v].x), bb = fp8x4_to_bf16(q.raw[v].y);
+            const uint2 c = fp8x4_to_bf16(q.raw[v].z), d = fp8x4_to_bf16(q.raw[v].w);
+            *reinterpret_cast<uint4*>(sm.K + swz(r, 16 * qq + 2 * v)) = make_uint4(a.x, a.y, bb.x, bb.y);
+            *reinterpret_cast<uint4*>(sm.K + swz(r, 16 * qq + 2 * v + 1)) = make_uint4(c.x, c.y, d.x, d.y);
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) *reinterpret_cast<uint4*>(sm.K + swz(r, 16 * qq + c)) = make_uint4(0, 0, 0, 0);
+    }
+    if (qq == 0) {
+        sm.kvalid[r] = q.kind != 0;
+        sm.kf[r] = q.kind == 2 ? q.fac : 1.0f;
+    }
 }
 
 __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
@@ -101,15 +194,24 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
     const uint32_t sP = (uint32_t)__cvta_generic_to_shared(sm.P);
     const uint32_t sPl = (uint32_t)__cvta_generic_to_shared(sm.Pl);
 
+    const int ntiles = (p.slots_total + kKT - 1) / kKT;
+    const int t0 = split * p.tiles_per_split;
+    const int t1 = min(ntiles, t0 + p.tiles_per_split);
+    // gather: key row and quarter of this thread; consecutive lanes take
+    // consecutive rows so their swizzled 16-byte stores hit distinct banks
+    const int gr = tid & (kKT - 1), gq = tid >> 6;
+
+    RowQuarter rq;
+    if (t0 < t1) fetch_quarter(p, bq, b, t0, gr, gq, i_pos, lo, pos0, nmain, rq);
+
     // Q [16][512] bf16 -> swizzled smem
     {
         const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (int64_t)bq * kH * kD);
 #pragma unroll
         for (int it = 0; it < (kH * kD / 8) / kAT; ++it) {
-            int c = it * kAT + tid;  // 16-byte chunk id
-            int row = c >> 6, ch = c & 63;
-            uint4 v = __ldg(qsrc + c);
-            *reinterpret_cast<uint4*>(sm.Qs + swz(row, ch)) = v;
+            const int c = it * kAT + tid;  // 16-byte chunk id
+            const int row = c >> 6, ch = c & 63;
+            *reinterpret_cast<uint4*>(sm.Qs + swz(row, ch)) = __ldg(qsrc + c);
         }
     }
     if (tid < kH) {
@@ -117,103 +219,34 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
         sm.l_run[tid] = 0.0f;
     }
 
-    float o[16][4];
+    float o[8][4];
 #pragma unroll
-    for (int n = 0; n < 16; ++n)
+    for (int n = 0; n < 8; ++n)
 #pragma unroll
         for (int j = 0; j < 4; ++j) o[n][j] = 0.0f;
 
-    const int ntiles = (p.slots_total + kKT - 1) / kKT;
-    const int t0 = split * p.tiles_per_split;
-    const int t1 = min(ntiles, t0 + p.tiles_per_split);
-
     for (int tile = t0; tile < t1; ++tile) {
-        // ---- gather + dequantise 64 key rows (2 threads per row) ----
-        {
-            const int r = tid >> 1, half = tid & 1;
-            const int slot = tile * kKT + r;
-            bool live = false;
-            float fac = 1.0f;
-            if (slot < p.k) {
-                int32_t e = __ldg(p.idx + (int64_t)bq * p.k + slot);
-                if (e >= 0 && e < nmain) {
-                    live = true;
-                    const int64_t row = (int64_t)b * p.cap + e;
-                    const uint4* cs = reinterpret_cast<const uint4*>(p.lat + row * (kD / 2) + 128 * half);
-                    uint4 scw = __ldg(reinterpret_cast<const uint4*>(p.lat_sc + row * (kD / 16) + 16 * half));
-                    uint32_t scb[4] = {scw.x, scw.y, scw.z, scw.w};
-#pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        uint4 cw = __ldg(cs + v);
-                        uint32_t ws[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            int word = 4 * v + j;                    // 8 dims per word, 32 words per half row
-                            int sbyte = word >> 1;                   // one scale per 16 dims
-                            float s = e4m3_to_f32((scb[sbyte >> 2] >> (8 * (sbyte & 3))) & 0xFFu);
-                            int chunk = 32 * half + word;
-                            *reinterpret_cast<uint4*>(sm.K + swz(r, chunk)) = fp4x8_to_bf16(ws[j], s);
-                        }
-                    }
-                }
-            } else if (slot < p.slots_total) {
-                int64_t tau = i_pos - p.window + 1 + (slot - p.k);
-                int64_t rr = tau - pos0;
-                if (tau >= lo && tau <= i_pos && rr >= 0 && rr < p.T) {
-                    live = true;
-                    const int64_t row = (int64_t)b * p.T + rr;
-                    fac = __ldg(p.swa_sc + row);
-                    const uint4* cs = reinterpret_cast<const uint4*>(p.swa + row * kD + 256 * half);
-#pragma unroll
-                    for (int v = 0; v < 16; ++v) {
-                        uint4 cw = __ldg(cs + v);
-                        uint2 a = fp8x4_to_bf16(cw.x), bb = fp8x4_to_bf16(cw.y);
-                        uint2 c = fp8x4_to_bf16(cw.z), d = fp8x4_to_bf16(cw.w);
-                        int chunk = 32 * half + 2 * v;
-                        *reinterpret_cast<uint4*>(sm.K + swz(r, chunk)) = make_uint4(a.x, a.y, bb.x, bb.y);
-                        *reinterpret_cast<uint4*>(sm.K + swz(r, chunk + 1)) = make_uint4(c.x, c.y, d.x, d.y);
-                    }
-                }
-            }
-            if (!live) {
-#pragma unroll
-                for (int c = 0; c < 32; ++c) *reinterpret_cast<uint4*>(sm.K + swz(r, 32 * half + c)) = make_uint4(0, 0, 0, 0);
-            }
-            if (half == 0) {
-                sm.kvalid[r] = live;
-                sm.kf[r] = fac;
-            }
-        }
+        store_quarter(sm, gr, gq, rq);
         __syncthreads();
+        if (tile + 1 < t1) fetch_quarter(p, bq, b, tile + 1, gr, gq, i_pos, lo, pos0, nmain, rq);   // in flight meanwhile
 
-        // ---- S = Q K^T for keys 16*warp .. +15 ----
-        float s[2][4];
-#pragma unroll
-        for (int n = 0; n < 2; ++n)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) s[n][j] = 0.0f;
-#pragma unroll 4
+        // ---- S = Q K^T for keys 8*warp .. +7 ----
+        float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 8
         for (int ks = 0; ks < kD / 16; ++ks) {
-            uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+            uint32_t a0, a1, a2, a3, b0, b1;
             ldsm_x4(sQ + swz(lane & 15, 2 * ks + (lane >> 4)), a0, a1, a2, a3);
-            const int mi = lane >> 3;
-            const int key = 16 * warp + (mi >> 1) * 8 + (lane & 7);
-            ldsm_x4(sK + swz(key, 2 * ks + (mi & 1)), b0, b1, b2, b3);
-            mma_bf16(s[0], a0, a1, a2, a3, b0, b1);
-            mma_bf16(s[1], a0, a1, a2, a3, b2, b3);
+            const int key = 8 * warp + (lane & 7);
+            ldsm_x2(sK + swz(key, 2 * ks + ((lane >> 3) & 1)), b0, b1);
+            mma_bf16(s4, a0, a1, a2, a3, b0, b1);
         }
-        // logits (log2 units), masked keys -> -inf
-        float z[2][4];
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-        for (int n = 0; n < 2; ++n)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                int key = 16 * warp + 8 * n + 2 * qd + (j & 1);
-                float v = sm.kvalid[key] ? s[n][j] * sm.kf[key] * scale_log2 : -INFINITY;
-                z[n][j] = v;
-                if (j < 2) mx0 = fmaxf(mx0, v); else mx1 = fmaxf(mx1, v);
-            }
+        // logits (log2 units); masked keys -> -inf
+        const int key0 = 8 * warp + 2 * qd;
+        const float f0 = sm.kf[key0], f1 = sm.kf[key0 + 1];
+        const bool v0 = sm.kvalid[key0] != 0, v1 = sm.kvalid[key0 + 1] != 0;
+        const float z00 = v0 ? s4[0] * f0 * scale_log2 : -INFINITY, z01 = v1 ? s4[1] * f1 * scale_log2 : -INFINITY;
+        const float z10 = v0 ? s4[2] * f0 * scale_log2 : -INFINITY, z11 = v1 ? s4[3] * f1 * scale_log2 : -INFINITY;
+        float mx0 = fmaxf(z00, z01), mx1 = fmaxf(z10, z11);
 #pragma unroll
         for (int o2 = 1; o2 < 4; o2 <<= 1) {
             mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, o2));
@@ -224,33 +257,27 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
             sm.red_max[warp][g + 8] = mx1;
         }
         __syncthreads();
-        float mt0 = fmaxf(fmaxf(sm.red_max[0][g], sm.red_max[1][g]), fmaxf(sm.red_max[2][g], sm.red_max[3][g]));
-        float mt1 = fmaxf(fmaxf(sm.red_max[0][g + 8], sm.red_max[1][g + 8]),
-                          fmaxf(sm.red_max[2][g + 8], sm.red_max[3][g + 8]));
-        float mn0 = fmaxf(sm.m_run[g], mt0), mn1 = fmaxf(sm.m_run[g + 8], mt1);
-        float mu0 = (mn0 == -INFINITY) ? 0.0f : mn0, mu1 = (mn1 == -INFINITY) ? 0.0f : mn1;
-        float sum0 = 0.0f, sum1 = 0.0f;
+        float mt0 = sm.red_max[0][g], mt1 = sm.red_max[0][g + 8];
 #pragma unroll
-        for (int n = 0; n < 2; ++n) {
-            int key0 = 16 * warp + 8 * n + 2 * qd;
-            float p00 = exp2f(z[n][0] - mu0), p01 = exp2f(z[n][1] - mu0);
-            float p10 = exp2f(z[n][2] - mu1), p11 = exp2f(z[n][3] - mu1);
-            sum0 += p00 + p01;
-            sum1 += p10 + p11;
-            float f0 = sm.kf[key0], f1 = sm.kf[key0 + 1];
-            // P row = head, column = key; 2 keys per 32-bit word
-            int chunk = key0 >> 3, within = (key0 & 7) * 2;
-            const uint32_t o0 = g * 128 + ((chunk ^ (g & 7)) << 4) + within;
-            const uint32_t o1 = (g + 8) * 128 + ((chunk ^ ((g + 8) & 7)) << 4) + within;
-            float v00 = p00 * f0, v01 = p01 * f1, v10 = p10 * f0, v11 = p11 * f1;
-            __nv_bfloat162 h0 = __floats2bfloat162_rn(v00, v01), h1 = __floats2bfloat162_rn(v10, v11);
-            *reinterpret_cast<__nv_bfloat162*>(sm.P + o0) = h0;
-            *reinterpret_cast<__nv_bfloat162*>(sm.P + o1) = h1;
-            *reinterpret_cast<uint32_t*>(sm.Pl + o0) =
-                pack_bf16(v00 - __low2float(h0), v01 - __high2float(h0));
-            *reinterpret_cast<uint32_t*>(sm.Pl + o1) =
-                pack_bf16(v10 - __low2float(h1), v11 - __high2float(h1));
+        for (int w = 1; w < 8; ++w) {
+            mt0 = fmaxf(mt0, sm.red_max[w][g]);
+            mt1 = fmaxf(mt1, sm.red_max[w][g + 8]);
         }
+        const float mn0 = fmaxf(sm.m_run[g], mt0), mn1 = fmaxf(sm.m_run[g + 8], mt1);
+        const float mu0 = (mn0 == -INFINITY) ? 0.0f : mn0, mu1 = (mn1 == -INFINITY) ? 0.0f : mn1;
+        const float p00 = exp2f(z00 - mu0), p01 = exp2f(z01 - mu0), p10 = exp2f(z10 - mu1), p11 = exp2f(z11 - mu1);
+        {
+            const int chunk = key0 >> 3, within = (key0 & 7) * 2;
+            const uint32_t off0 = g * 128 + ((chunk ^ (g & 7)) << 4) + within;
+            const uint32_t off1 = (g + 8) * 128 + ((chunk ^ ((g + 8) & 7)) << 4) + within;
+            const float u00 = p00 * f0, u01 = p01 * f1, u10 = p10 * f0, u11 = p11 * f1;
+            const __nv_bfloat162 h0 = __floats2bfloat162_rn(u00, u01), h1 = __floats2bfloat162_rn(u10, u11);
+            *reinterpret_cast<__nv_bfloat162*>(sm.P + off0) = h0;
+            *reinterpret_cast<__nv_bfloat162*>(sm.P + off1) = h1;
+            *reinterpret_cast<uint32_t*>(sm.Pl + off0) = pack_bf16(u00 - __low2float(h0), u01 - __high2float(h0));
+            *reinterpret_cast<uint32_t*>(sm.Pl + off1) = pack_bf16(u10 - __low2float(h1), u11 - __high2float(h1));
+        }
+        float sum0 = p00 + p01, sum1 = p10 + p11;
 #pragma unroll
         for (int o2 = 1; o2 < 4; o2 <<= 1) {
             sum0 += __shfl_xor_sync(0xFFFFFFFFu, sum0, o2);
@@ -262,22 +289,26 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
         }
         __syncthreads();
         if (tid < kH) {
-            float mt = fmaxf(fmaxf(sm.red_max[0][tid], sm.red_max[1][tid]), fmaxf(sm.red_max[2][tid], sm.red_max[3][tid]));
-            float mo = sm.m_run[tid];
-            float mn = fmaxf(mo, mt);
-            float al = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
+            float mt = sm.red_max[0][tid], ssum = 0.0f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                mt = fmaxf(mt, sm.red_max[w][tid]);
+                ssum += sm.red_sum[w][tid];
+            }
+            const float mo = sm.m_run[tid];
+            const float mn = fmaxf(mo, mt);
+            const float al = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
             sm.alpha[tid] = al;
-            sm.l_run[tid] = sm.l_run[tid] * al +
-                            ((sm.red_sum[0][tid] + sm.red_sum[1][tid]) + (sm.red_sum[2][tid] + sm.red_sum[3][tid]));
+            sm.l_run[tid] = sm.l_run[tid] * al + ssum;
             sm.m_run[tid] = mn;
         }
         __syncthreads();
 
-        // ---- O[:, 128 warp .. +127] = alpha O + P V ----
+        // ---- O[:, 64 warp .. +63] = alpha O + P V ----
         {
-            float al0 = sm.alpha[g], al1 = sm.alpha[g + 8];
+            const float al0 = sm.alpha[g], al1 = sm.alpha[g + 8];
 #pragma unroll
-            for (int n = 0; n < 16; ++n) {
+            for (int n = 0; n < 8; ++n) {
                 o[n][0] *= al0;
                 o[n][1] *= al0;
                 o[n][2] *= al1;
@@ -287,17 +318,17 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
             for (int kk = 0; kk < kKT / 16; ++kk) {
                 uint32_t a0, a1, a2, a3, l0, l1, l2, l3;
                 {
-                    int row = lane & 15, chunk = 2 * kk + (lane >> 4);
-                    uint32_t off = (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+                    const int row = lane & 15, chunk = 2 * kk + (lane >> 4);
+                    const uint32_t off = (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
                     ldsm_x4(sP + off, a0, a1, a2, a3);
                     ldsm_x4(sPl + off, l0, l1, l2, l3);
                 }
                 const int mi = lane >> 3;
                 const int key = 16 * kk + (mi & 1) * 8 + (lane & 7);
 #pragma unroll
-                for (int np = 0; np < 8; ++np) {
+                for (int np = 0; np < 4; ++np) {
                     uint32_t b0, b1, b2, b3;
-                    ldsm_x4_t(sK + swz(key, 16 * warp + 2 * np + (mi >> 1)), b0, b1, b2, b3);
+                    ldsm_x4_t(sK + swz(key, 8 * warp + 2 * np + (mi >> 1)), b0, b1, b2, b3);
                     mma_bf16(o[2 * np], a0, a1, a2, a3, b0, b1);
                     mma_bf16(o[2 * np + 1], a0, a1, a2, a3, b2, b3);
                     mma_bf16(o[2 * np], l0, l1, l2, l3, b0, b1);
@@ -311,17 +342,17 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
     // ---- write the split's partial, or the final output ----
     const float LN2 = 0.6931471805599453f;
     if (S == 1) {
-        float l0 = sm.l_run[g], l1 = sm.l_run[g + 8];
-        float inv0 = l0 > 0.0f ? 1.0f / l0 : 0.0f, inv1 = l1 > 0.0f ? 1.0f / l1 : 0.0f;
+        const float l0 = sm.l_run[g], l1 = sm.l_run[g + 8];
+        const float inv0 = l0 > 0.0f ? 1.0f / l0 : 0.0f, inv1 = l1 > 0.0f ? 1.0f / l1 : 0.0f;
         uint16_t* out = p.out + (int64_t)bq * kH * kD;
 #pragma unroll
-        for (int n = 0; n < 16; ++n) {
-            int d = 128 * warp + 8 * n + 2 * qd;
+        for (int n = 0; n < 8; ++n) {
+            const int d = 64 * warp + 8 * n + 2 * qd;
             *reinterpret_cast<uint32_t*>(out + g * kD + d) = pack_bf16(o[n][0] * inv0, o[n][1] * inv0);
             *reinterpret_cast<uint32_t*>(out + (g + 8) * kD + d) = pack_bf16(o[n][2] * inv1, o[n][3] * inv1);
         }
         if (p.lse && tid < kH) {
-            float l = sm.l_run[tid];
+            const float l = sm.l_run[tid];
             p.lse[(int64_t)bq * kH + tid] = l > 0.0f ? (sm.m_run[tid] + log2f(l)) * LN2 : -INFINITY;
         }
         return;
@@ -329,8 +360,8 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
     {
         float* po = p.part_o + ((int64_t)bq * S + split) * kH * kD;
 #pragma unroll
-        for (int n = 0; n < 16; ++n) {
-            int d = 128 * warp + 8 * n + 2 * qd;
+        for (int n = 0; n < 8; ++n) {
+            const int d = 64 * warp + 8 * n + 2 * qd;
             *reinterpret_cast<float2*>(po + g * kD + d) = make_float2(o[n][0], o[n][1]);
             *reinterpret_cast<float2*>(po + (g + 8) * kD + d) = make_float2(o[n][2], o[n][3]);
         }
@@ -364,8 +395,8 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
     }
     __syncthreads();
     {
-        // thread owns 16 float4 of the [16][512] output: element 4 (tid + 128 j)
-        constexpr int kV = kH * kD / 4 / kAT;   // 16
+        // thread owns 8 float4 of the [16][512] output: element 4 (tid + 256 j)
+        constexpr int kV = kH * kD / 4 / kAT;   // 8
         float4 acc[kV];
 #pragma unroll
         for (int j = 0; j < kV; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -145,28 +145,55 @@ __global__ void __launch_bounds__(256) index_k_proj_kernel(const uint16_t* __res
 }
 
 // Few rows (a decode append): one thread per (row, output) runs its 512-long
-// FMA chain, 4 rows per CTA; the 64 outputs of a row are then quantised from
-// shared memory by 4 threads.
+// FMA chain, 4 rows per CTA.  The rows and 64-channel chunks of W are staged in
+// shared memory (double-buffered), so the chain waits only on its own FMAs.
+// The 64 outputs of a row are then quantised from shared memory by 4 threads.
+constexpr int kRC = 64;   // channels per W chunk
+
 __global__ void __launch_bounds__(256) index_k_proj_rows_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                                 const float* __restrict__ W, uint8_t* __restrict__ kc,
                                                                 uint8_t* __restrict__ ks,
                                                                 const int64_t* __restrict__ dst_rows, int64_t out_rows) {
+    __shared__ float xs[4][kD];
+    __shared__ float4 wbuf[2][kRC * kID / 4];
     __shared__ float outs[4][kID];
     const int tid = threadIdx.x;
     const int rr = tid >> 6, j = tid & 63;
-    const int64_t row = (int64_t)blockIdx.x * 4 + rr;
-    if (row < rows) {
-        const uint16_t* xr = x + row * kD;
-        float acc = 0.0f;
-#pragma unroll 16
-        for (int c = 0; c < kD; ++c)
-            acc = __fmaf_rn(__uint_as_float(((uint32_t)__ldg(xr + c)) << 16), __ldg(W + c * kID + j), acc);
-        outs[rr][j] = acc;
+    const int64_t r0 = (int64_t)blockIdx.x * 4;
+    for (int e = tid; e < 4 * kD; e += 256) {
+        const int64_t row = r0 + e / kD;
+        xs[e / kD][e % kD] = row < rows ? __uint_as_float(((uint32_t)__ldg(x + row * kD + e % kD)) << 16) : 0.0f;
     }
+    const float4* W4 = reinterpret_cast<const float4*>(W);
+    float4 pre[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) pre[q] = __ldg(W4 + tid + 256 * q);   // chunk 0: 1024 float4
+#pragma unroll
+    for (int q = 0; q < 4; ++q) wbuf[0][tid + 256 * q] = pre[q];
+    __syncthreads();
+    float acc = 0.0f;
+    constexpr int kChunks = kD / kRC;
+    for (int ch = 0; ch < kChunks; ++ch) {
+        const int cur = ch & 1;
+        if (ch + 1 < kChunks) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) pre[q] = __ldg(W4 + (ch + 1) * (kRC * kID / 4) + tid + 256 * q);
+        }
+        const float* wc = reinterpret_cast<const float*>(wbuf[cur]);
+        const float* xr = xs[rr] + ch * kRC;
+#pragma unroll 16
+        for (int c = 0; c < kRC; ++c) acc = __fmaf_rn(xr[c], wc[c * kID + j], acc);
+        if (ch + 1 < kChunks) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) wbuf[cur ^ 1][tid + 256 * q] = pre[q];
+        }
+        __syncthreads();
+    }
+    outs[rr][j] = acc;
     __syncthreads();
     if (tid < 16) {
         const int r2 = tid >> 2, g = tid & 3;
-        const int64_t row2 = (int64_t)blockIdx.x * 4 + r2;
+        const int64_t row2 = r0 + r2;
         if (row2 < rows) {
             float v[16];
 #pragma unroll
