@@ -57,7 +57,7 @@ def _peaks():
 
 def _kernel_hash():
     h = hashlib.sha256()
-    for f in ("index.cu", "topk.cuh", "common.cuh"):
+    for f in ("index_cluster.cu", "index_pipe.cuh", "index_tc.cu", "tc.cuh", "common.cuh", "kernels.h"):
         with open(os.path.join(ROOT, "sparse_attention_fp4_quant_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -353,7 +353,7 @@ def run_ours(args, rank, world, local_rank):
         "step_algorithmic_bytes": STEP_BYTES,
         "segments_ms": {"front": float(np.mean([e[0].elapsed_time(e[1]) for e in all_ev])),
                         "index_topk": float(np.mean(index_ms)), "attention_x4": float(np.mean(attn_ms))},
-        "roofline": {"kernel": "csa2_index_topk (select_kernel<dense>)", "bound": "hbm", "achieved": achieved,
+        "roofline": {"kernel": "csa2_index_topk (index_cluster_kernel)", "bound": "hbm", "achieved": achieved,
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
                      "bytes_per_launch": INDEX_LAUNCH_BYTES},

@@ -130,7 +130,7 @@ CSA2_API csa2_status csa2_quant_nvfp4(const void* x, int64_t rows, int32_t ch, u
  * then NVFP4-quantised exactly as csa2_quant_nvfp4 does (64 channels -> 32 B
  * codes + 4 B scales).
  *   x        device bf16 [rows][512] (post-RoPE latent rows), 16-byte aligned
- *   W        device fp32 [512][64]
+ *   W        device fp32 [512][64], 16-byte aligned
  *   k_codes  device u8 [out_rows][32] (8-byte aligned), k_scales device u8 [out_rows][4];
  *            row mapping and out_rows as for csa2_quant_nvfp4
  */

@@ -109,6 +109,17 @@ def _dev(t, dtype, name):
     return t
 
 
+def _size(t, n, name):
+    if t.numel() != n:
+        raise ValueError(f"{name}: expected {n} elements, got {t.numel()} (shape {tuple(t.shape)})")
+    return t
+
+
+def _batch(kv, B):
+    if kv.B != B:
+        raise ValueError(f"q_pos has {B} batch rows but the KV has {kv.B}")
+
+
 class KV:
     """The shared global KV of a CSA2 layer group (device tensors) and its csa2_kv view."""
 
@@ -187,12 +198,16 @@ def csa2_index_topk(q, q_sc, w, kv, q_pos, k, idx_out=None, blockmax=False, ws=N
     for t, dt, n in ((q, torch.uint8, "q"), (q_sc, torch.uint8, "q_sc"), (w, torch.float32, "w"),
                      (q_pos, torch.int32, "q_pos")):
         _dev(t, dt, n)
+    _batch(kv, B)
+    _size(q, B * Q * 128, "q"), _size(q_sc, B * Q * 16, "q_sc"), _size(w, B * Q * 4, "w")
     if idx_out is None:
         idx_out = torch.empty((B, Q, k), dtype=torch.int32, device=q.device)
+    _size(_dev(idx_out, torch.int32, "idx_out"), B * Q * k, "idx_out")
     bm = None
     if blockmax is not False:
         bm = blockmax if isinstance(blockmax, torch.Tensor) else torch.empty(
             (B, Q, (kv.cap + BLOCK - 1) // BLOCK), dtype=torch.float32, device=q.device)
+        _size(_dev(bm, torch.float32, "blockmax"), B * Q * ((kv.cap + BLOCK - 1) // BLOCK), "blockmax")
     nbytes = csa2_workspace_bytes(OP_INDEX_TOPK, B, Q, kv.cap, k)
     ws = _workspace(nbytes) if ws is None else ws
     _check(lib().csa2_index_topk(_ptr(q), _ptr(q_sc), _ptr(w), kv.c(), _ptr(q_pos), B, Q, k, _ptr(idx_out),
@@ -208,12 +223,16 @@ def csa2_index_topk_noalloc(q, q_sc, w, kv, q_pos, k, idx_out=None, blockmax=Fal
     for t, dt, n in ((q, torch.uint8, "q"), (q_sc, torch.uint8, "q_sc"), (w, torch.float32, "w"),
                      (q_pos, torch.int32, "q_pos")):
         _dev(t, dt, n)
+    _batch(kv, B)
+    _size(q, B * Q * 128, "q"), _size(q_sc, B * Q * 16, "q_sc"), _size(w, B * Q * 4, "w")
     if idx_out is None:
         idx_out = torch.empty((B, Q, k), dtype=torch.int32, device=q.device)
+    _size(_dev(idx_out, torch.int32, "idx_out"), B * Q * k, "idx_out")
     bm = None
     if blockmax is not False:
         bm = blockmax if isinstance(blockmax, torch.Tensor) else torch.empty(
             (B, Q, (kv.cap + BLOCK - 1) // BLOCK), dtype=torch.float32, device=q.device)
+        _size(_dev(bm, torch.float32, "blockmax"), B * Q * ((kv.cap + BLOCK - 1) // BLOCK), "blockmax")
     _check(lib().csa2_index_topk_noalloc(_ptr(q), _ptr(q_sc), _ptr(w), kv.c(), _ptr(q_pos), B, Q, k, _ptr(idx_out),
                                          _ptr(bm), _stream()))
     return (idx_out, bm) if bm is not None else idx_out
@@ -223,8 +242,11 @@ def csa2_pool_build(blockmax, kv, q_pos, max_blocks=POOL_BLOCKS, pool_out=None, 
     B, Q = q_pos.shape
     _dev(blockmax, torch.float32, "blockmax")
     _dev(q_pos, torch.int32, "q_pos")
+    _batch(kv, B)
+    _size(blockmax, B * Q * ((kv.cap + BLOCK - 1) // BLOCK), "blockmax")
     if pool_out is None:
         pool_out = torch.empty((B, Q, max_blocks), dtype=torch.int32, device=blockmax.device)
+    _size(_dev(pool_out, torch.int32, "pool_out"), B * Q * max_blocks, "pool_out")
     nbytes = csa2_workspace_bytes(OP_POOL_BUILD, B, Q, kv.cap, max_blocks)
     ws = _workspace(nbytes) if ws is None else ws
     _check(lib().csa2_pool_build(_ptr(blockmax), kv.c(), _ptr(q_pos), B, Q, max_blocks, _ptr(pool_out), _ptr(ws),
@@ -238,8 +260,12 @@ def csa2_pool_topk(q, q_sc, w, kv, pool, q_pos, k, idx_out=None, ws=None):
     for t, dt, n in ((q, torch.uint8, "q"), (q_sc, torch.uint8, "q_sc"), (w, torch.float32, "w"),
                      (pool, torch.int32, "pool"), (q_pos, torch.int32, "q_pos")):
         _dev(t, dt, n)
+    _batch(kv, B)
+    _size(q, B * Q * 128, "q"), _size(q_sc, B * Q * 16, "q_sc"), _size(w, B * Q * 4, "w")
+    _size(pool, B * Q * P, "pool")
     if idx_out is None:
         idx_out = torch.empty((B, Q, k), dtype=torch.int32, device=q.device)
+    _size(_dev(idx_out, torch.int32, "idx_out"), B * Q * k, "idx_out")
     nbytes = csa2_workspace_bytes(OP_POOL_TOPK, B, Q, kv.cap, k, P)
     ws = _workspace(nbytes) if ws is None else ws
     _check(lib().csa2_pool_topk(_ptr(q), _ptr(q_sc), _ptr(w), kv.c(), _ptr(pool), P, _ptr(q_pos), B, Q, k,
@@ -262,8 +288,14 @@ def csa2_sparse_attn(q, kv, idx, swa, swa_sc, swa_pos0, q_pos, window=WINDOW, re
         _dev(replay_start, torch.int32, "replay_start")
     k = idx.shape[-1]
     T = swa.shape[1]
+    _batch(kv, B)
+    _size(q, B * Q * H * D, "q"), _size(idx, B * Q * k, "idx"), _size(swa, B * T * D, "swa")
+    _size(swa_sc, B * T, "swa_sc"), _size(swa_pos0, B, "swa_pos0")
+    if replay_start is not None:
+        _size(replay_start, B, "replay_start")
     if out is None:
         out = torch.empty((B, Q, H, D), dtype=torch.bfloat16, device=q.device)
+    _size(_dev(out, torch.bfloat16, "out"), B * Q * H * D, "out")
     lse_t = None
     if lse is not False:
         lse_t = lse if isinstance(lse, torch.Tensor) else torch.empty((B, Q, H), dtype=torch.float32,
@@ -281,6 +313,7 @@ def csa2_layer_step(mode, kv, q_pos, q, swa, swa_sc, swa_pos0, idx, k=TOPK, iq=N
                     window=WINDOW, replay_start=None, sm_scale=1.0 / math.sqrt(D), out=None, lse=None, ws=None):
     """One CSA2 layer dispatched by mode ('full' | 'reindex' | 'reuse'); returns the attention output."""
     B, Q = q_pos.shape
+    _batch(kv, B)
     if out is None:
         out = torch.empty((B, Q, H, D), dtype=torch.bfloat16, device=q.device)
     P = pool.shape[-1] if pool is not None else pool_blocks

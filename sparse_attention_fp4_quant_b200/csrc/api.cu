@@ -78,7 +78,8 @@ csa2_status csa2_index_k_proj(const void* x, int64_t rows, const float* W, uint8
                               const int64_t* dst_rows, int64_t out_rows, void* stream) {
     if (rows < 0) return CSA2_ERR_INVALID_ARG;
     if (rows == 0) return CSA2_OK;
-    if (!x || !W || !k_codes || !k_scales || !aligned16(x) || ((uintptr_t)k_codes & 7u)) return CSA2_ERR_INVALID_ARG;
+    if (!x || !W || !k_codes || !k_scales || !aligned16(x) || !aligned16(W) || ((uintptr_t)k_codes & 7u))
+        return CSA2_ERR_INVALID_ARG;
     if (out_rows < 0 || (!dst_rows && out_rows < rows)) return CSA2_ERR_INVALID_ARG;
     return cuda_status(launch_index_k_proj(x, rows, W, k_codes, k_scales, dst_rows, out_rows, (cudaStream_t)stream));
 }
@@ -189,6 +190,8 @@ csa2_status csa2_sparse_attn(const void* q, const csa2_kv* kv, const int32_t* id
     p.out = static_cast<uint16_t*>(out);
     p.lse = lse;
     p.slots_total = k + window;
+    const int C = attn_cluster_size(B, Q, p.slots_total, &p.keys_per_cta);
+    if (C > 0) return cuda_status(launch_attn_cluster(p, C, (cudaStream_t)stream));
     int S = attn_splits(B, Q, k, window, &p.tiles_per_split);
     attn_carve_ws(p, S, ws);
     return cuda_status(launch_attn(p, S, (cudaStream_t)stream));

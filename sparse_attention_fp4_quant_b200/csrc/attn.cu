@@ -1,28 +1,21 @@
 // attn.cu -- sparse attention over the Top-K FP4 main rows plus the layer's own
 // FP8 sliding-window KV, under the SWA Bounded Replay mask.
 //
-// Key slots of a query: [0, k) are the main rows idx[0..k), [k, k + W) are the
-// window tokens i - W + 1 .. i.  A slot is live if its row exists and (for the
-// window) the token lies in [max(s, i - W + 1), i] and in the stored SWA rows.
-// A CTA (8 warps) takes a split of the slot range in tiles of 64 keys.  Each
-// tile is gathered into registers one tile ahead (its loads overlap the
-// previous tile's math), dequantised to bf16 in swizzled shared memory (K = V),
-// and S = Q K^T (8 keys per warp) and O += P V (64 dims per warp) run on
-// warp-level tensor-core MMAs with the 16 heads as the M dimension; the softmax
-// is online across tiles.  FP4 rows dequantise exactly to bf16 (byte-table
-// decode, then an exact bf16 multiply by the block scale); an SWA row is kept
-// as its E4M3 values (exact in bf16) and its fp32 token scale multiplies the
-// logit and the probability instead.  P enters P V as two bf16 terms (rounded
-// value + remainder), about 16 bits of P.  Splits of one query are merged by
-// the last CTA to finish (atomic ticket).
-#include "common.cuh"
-#include "kernels.h"
+// Split-K form, for query counts too large for one cluster per query
+// (attn_cluster.cu serves the rest).  A CTA (8 warps) takes a split of the
+// slot range in tiles of 64 keys.  Each tile is gathered into registers one
+// tile ahead (its loads overlap the previous tile's math), dequantised to bf16
+// in swizzled shared memory (K = V), and S = Q K^T (8 keys per warp) and
+// O += P V (64 dims per warp) run on warp-level tensor-core MMAs with the 16
+// heads as the M dimension; the softmax is online across tiles.  P enters P V
+// as two bf16 terms (rounded value + remainder), about 16 bits of P.  Splits
+// of one query are merged by the last CTA to finish (atomic ticket).
+#include "attn_common.cuh"
 
 namespace csa2 {
 
 constexpr int kAT = 256;      // threads per CTA (8 warps)
 constexpr int kKT = 64;       // keys per tile
-constexpr int kRowB = kD * 2; // bytes per bf16 row of 512
 constexpr int kMaxSplits = (CSA2_MAX_K + CSA2_MAX_WINDOW + kKT - 1) / kKT;
 
 struct AttnSmem {
@@ -38,140 +31,6 @@ struct AttnSmem {
     float cw[kMaxSplits][kH];  // combine weights 2^(m_s - M) / L per split and head
     int last;
 };
-
-__device__ __forceinline__ uint32_t swz(int row, int chunk) { return (uint32_t)(row * kRowB + ((chunk ^ (row & 7)) << 4)); }
-
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t*>(&h);
-}
-
-__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
-    __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
-    return *reinterpret_cast<uint32_t*>(&r);
-}
-
-// 8 E2M1 codes (nibble n = dim n) times the block scale (bf16x2 s2) -> 8 bf16.
-// The magnitudes come from byte tables (high and low byte of the bf16 value),
-// the sign is moved to bit 15 of each half, and the product with the scale is
-// exact (at most 6 significant bits).
-__device__ __forceinline__ uint4 fp4x8_to_bf16(uint32_t w, uint32_t s2) {
-    const uint32_t HI0 = 0x3F3F3F00u, HI1 = 0x40404040u;   // 0 .5 1 1.5 | 2 3 4 6: high bytes
-    const uint32_t LO0 = 0xC0800000u, LO1 = 0xC0804000u;   //                     low bytes
-    const uint32_t m = w & 0x77777777u, mh = m >> 16;
-    const uint32_t hi_a = __byte_perm(HI0, HI1, m), lo_a = __byte_perm(LO0, LO1, m);
-    const uint32_t hi_b = __byte_perm(HI0, HI1, mh), lo_b = __byte_perm(LO0, LO1, mh);
-    uint32_t v0 = __byte_perm(lo_a, hi_a, 0x5140), v1 = __byte_perm(lo_a, hi_a, 0x7362);
-    uint32_t v2 = __byte_perm(lo_b, hi_b, 0x5140), v3 = __byte_perm(lo_b, hi_b, 0x7362);
-    // nibble signs (bits 3 and 7 of each byte) -> bits 15 and 31 of the bf16 pair
-    v0 |= ((w & 0x88u) * 0x1001000u) & 0x80008000u;
-    v1 |= (((w >> 8) & 0x88u) * 0x1001000u) & 0x80008000u;
-    v2 |= (((w >> 16) & 0x88u) * 0x1001000u) & 0x80008000u;
-    v3 |= (((w >> 24) & 0x88u) * 0x1001000u) & 0x80008000u;
-    return make_uint4(bf16x2_mul(v0, s2), bf16x2_mul(v1, s2), bf16x2_mul(v2, s2), bf16x2_mul(v3, s2));
-}
-
-// 4 E4M3 bytes -> 4 bf16 (exact).
-__device__ __forceinline__ uint2 fp8x4_to_bf16(uint32_t w) {
-    float f[4];
-    e4m3x4_to_f32(w, f);
-    return make_uint2(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]));
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-
-__device__ __forceinline__ void mma_bf16(float c[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
-                                         uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// One quarter (128 dims) of one key row, held in registers between its load
-// and its dequantisation.
-struct RowQuarter {
-    uint4 raw[8];   // FP4: raw[0..3] = 64 code bytes; FP8: raw[0..7] = 128 bytes
-    uint2 sc;       // FP4: the 8 block scales of the quarter
-    float fac;      // FP8: the token scale
-    int kind;       // 0 = dead slot, 1 = FP4 main row, 2 = FP8 window row
-};
-
-__device__ __forceinline__ void fetch_quarter(const AttnParams& p, int bq, int b, int tile, int r, int qq, int64_t i_pos,
-                                              int64_t lo, int64_t pos0, int64_t nmain, RowQuarter& q) {
-    q.kind = 0;
-    const int slot = tile * kKT + r;
-    if (slot < p.k) {
-        const int32_t e = __ldg(p.idx + (int64_t)bq * p.k + slot);
-        if (e >= 0 && e < nmain) {
-            q.kind = 1;
-            const int64_t row = (int64_t)b * p.cap + e;
-            const uint4* cs = reinterpret_cast<const uint4*>(p.lat + row * (kD / 2) + 64 * qq);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) q.raw[v] = __ldg(cs + v);
-            q.sc = __ldg(reinterpret_cast<const uint2*>(p.lat_sc + row * (kD / 16) + 8 * qq));
-        }
-    } else if (slot < p.slots_total) {
-        const int64_t tau = i_pos - p.window + 1 + (slot - p.k);
-        const int64_t rr = tau - pos0;
-        if (tau >= lo && tau <= i_pos && rr >= 0 && rr < p.T) {
-            q.kind = 2;
-            const int64_t row = (int64_t)b * p.T + rr;
-            q.fac = __ldg(p.swa_sc + row);
-            const uint4* cs = reinterpret_cast<const uint4*>(p.swa + row * kD + 128 * qq);
-#pragma unroll
-            for (int v = 0; v < 8; ++v) q.raw[v] = __ldg(cs + v);
-        }
-    }
-}
-
-__device__ __forceinline__ void store_quarter(AttnSmem& sm, int r, int qq, const RowQuarter& q) {
-    if (q.kind == 1) {
-        const uint32_t scw[2] = {q.sc.x, q.sc.y};
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-            const uint32_t ws[4] = {q.raw[v].x, q.raw[v].y, q.raw[v].z, q.raw[v].w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int word = 4 * v + j;             // 8 dims per word
-                const int sb = word >> 1;               // one scale per 16 dims
-                const float s = e4m3_to_f32((scw[sb >> 2] >> (8 * (sb & 3))) & 0xFFu);
-                const uint32_t s2 = pack_bf16(s, s);   // exact (E4M3 fits bf16)
-                *reinterpret_cast<uint4*>(sm.K + swz(r, 16 * qq + word)) = fp4x8_to_bf16(ws[j], s2);
-            }
-        }
-    } else if (q.kind == 2) {
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-            const uint2 a = fp8x4_to_bf16(q.raw[v].x), bb = fp8x4_to_bf16(q.raw[v].y);
-            const uint2 c = fp8x4_to_bf16(q.raw[v].z), d = fp8x4_to_bf16(q.raw[v].w);
-            *reinterpret_cast<uint4*>(sm.K + swz(r, 16 * qq + 2 * v)) = make_uint4(a.x, a.y, bb.x, bb.y);
-            *reinterpret_cast<uint4*>(sm.K + swz(r, 16 * qq + 2 * v + 1)) = make_uint4(c.x, c.y, d.x, d.y);
-        }
-    } else {
-#pragma unroll
-        for (int c = 0; c < 16; ++c) *reinterpret_cast<uint4*>(sm.K + swz(r, 16 * qq + c)) = make_uint4(0, 0, 0, 0);
-    }
-    if (qq == 0) {
-        sm.kvalid[r] = q.kind != 0;
-        sm.kf[r] = q.kind == 2 ? q.fac : 1.0f;
-    }
-}
 
 __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -202,7 +61,7 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
     const int gr = tid & (kKT - 1), gq = tid >> 6;
 
     RowQuarter rq;
-    if (t0 < t1) fetch_quarter(p, bq, b, t0, gr, gq, i_pos, lo, pos0, nmain, rq);
+    if (t0 < t1) fetch_quarter(p, bq, b, t0 * kKT + gr, gq, i_pos, lo, pos0, nmain, rq);
 
     // Q [16][512] bf16 -> swizzled smem
     {
@@ -226,9 +85,9 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
         for (int j = 0; j < 4; ++j) o[n][j] = 0.0f;
 
     for (int tile = t0; tile < t1; ++tile) {
-        store_quarter(sm, gr, gq, rq);
+        store_quarter(sm.K, sm.kf, sm.kvalid, gr, gq, rq);
         __syncthreads();
-        if (tile + 1 < t1) fetch_quarter(p, bq, b, tile + 1, gr, gq, i_pos, lo, pos0, nmain, rq);   // in flight meanwhile
+        if (tile + 1 < t1) fetch_quarter(p, bq, b, (tile + 1) * kKT + gr, gq, i_pos, lo, pos0, nmain, rq);   // in flight meanwhile
 
         // ---- S = Q K^T for keys 8*warp .. +7 ----
         float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};

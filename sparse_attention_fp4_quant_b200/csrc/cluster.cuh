@@ -1,0 +1,50 @@
+// cluster.cuh -- thread-block cluster primitives (sm_100a): rank, barrier over
+// the cluster, and loads from another CTA's shared memory.
+#pragma once
+#include <stdint.h>
+
+namespace csa2 {
+namespace cl {
+
+__device__ __forceinline__ uint32_t rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t ctas() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
+// Barrier over every thread of the cluster; orders shared-memory writes before
+// it with reads (local or remote) after it.
+__device__ __forceinline__ void sync() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// Address of the same shared-memory variable in CTA `r` of the cluster.
+__device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t r) {
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(saddr), "r"(r));
+    return a;
+}
+
+__device__ __forceinline__ uint4 ld_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint2 ld_v2(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared::cluster.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
+    return v;
+}
+
+}  // namespace cl
+}  // namespace csa2

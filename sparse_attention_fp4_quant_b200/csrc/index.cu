@@ -252,7 +252,13 @@ void select_carve_ws(SelectParams& p, int S, void* ws, int B, int Q, int k) {
 }
 
 cudaError_t launch_select(int op, SelectParams& p, int S, cudaStream_t st) {
-    if ((op == CSA2_OP_INDEX_TOPK || op == CSA2_OP_POOL_TOPK) && index_tc_supported(p)) return launch_index_tc(op, p, S, st);
+    if ((op == CSA2_OP_INDEX_TOPK || op == CSA2_OP_POOL_TOPK) && index_tc_supported(p)) {
+        if (op == CSA2_OP_INDEX_TOPK) {
+            const int C = index_cluster_size(p);
+            if (C > 0) return launch_index_cluster(p, C, st);
+        }
+        return launch_index_tc(op, p, S, st);
+    }
     dim3 grid(S, p.B * p.Q);
     const int smem = (int)sizeof(TK::Smem);
     static bool attr[3] = {false, false, false};

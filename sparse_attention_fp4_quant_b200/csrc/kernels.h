@@ -44,6 +44,9 @@ void select_carve_ws(SelectParams& p, int S, void* ws, int B, int Q, int k);
 cudaError_t launch_select(int op, SelectParams& p, int S, cudaStream_t st);
 bool index_tc_supported(const SelectParams& p);
 cudaError_t launch_index_tc(int op, SelectParams& p, int S, cudaStream_t st);
+// One cluster of C CTAs per query (index Top-K only); 0 = the shape does not fit.
+int index_cluster_size(const SelectParams& p);
+cudaError_t launch_index_cluster(SelectParams& p, int C, cudaStream_t st);
 
 // NVFP4 quantisation and the indexer-K projection.
 cudaError_t launch_quant(const void* x, int64_t rows, int ch, uint8_t* codes, uint8_t* scales,
@@ -71,7 +74,8 @@ struct AttnParams {
     uint16_t* out;            // bf16 [B*Q][16][512]
     float* lse;               // [B*Q][16] or null
     int slots_total;          // k + window
-    int tiles_per_split;
+    int tiles_per_split;      // split-K form: 64-key tiles per split
+    int keys_per_cta;         // cluster form: key slots per CTA
     // workspace
     int32_t* counters;        // [B*Q]
     float* part_o;            // [B*Q][S][16][512]
@@ -82,5 +86,8 @@ int attn_splits(int B, int Q, int k, int window, int* tiles_per_split);
 size_t attn_ws_bytes(int B, int Q, int k, int window);
 void attn_carve_ws(AttnParams& p, int S, void* ws);
 cudaError_t launch_attn(AttnParams& p, int S, cudaStream_t st);
+// One cluster of C CTAs per query; 0 = the shape does not fit.
+int attn_cluster_size(int B, int Q, int slots_total, int* keys_per_cta);
+cudaError_t launch_attn_cluster(AttnParams& p, int C, cudaStream_t st);
 
 }  // namespace csa2

@@ -145,53 +145,40 @@ __global__ void __launch_bounds__(256) index_k_proj_kernel(const uint16_t* __res
 }
 
 // Few rows (a decode append): one thread per (row, output) runs its 512-long
-// FMA chain, 4 rows per CTA.  The rows and 64-channel chunks of W are staged in
-// shared memory (double-buffered), so the chain waits only on its own FMAs.
-// The 64 outputs of a row are then quantised from shared memory by 4 threads.
-constexpr int kRC = 64;   // channels per W chunk
+// FMA chain, 4 rows per CTA.  All of W (128 KB) is copied into shared memory
+// with cp.async up front, so the copy costs one memory latency and the chain
+// then waits only on its own FMAs.  The 64 outputs of a row are quantised from
+// shared memory by 4 threads.
+constexpr int kProjRowsPerCTA = 4;
+constexpr int kProjSmem = (kD * kID + kProjRowsPerCTA * kD) * 4;
 
 __global__ void __launch_bounds__(256) index_k_proj_rows_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                                 const float* __restrict__ W, uint8_t* __restrict__ kc,
                                                                 uint8_t* __restrict__ ks,
                                                                 const int64_t* __restrict__ dst_rows, int64_t out_rows) {
-    __shared__ float xs[4][kD];
-    __shared__ float4 wbuf[2][kRC * kID / 4];
-    __shared__ float outs[4][kID];
+    extern __shared__ __align__(16) float wsm[];   // W [512][64], then the rows [4][512]
+    float* xs = wsm + kD * kID;
+    __shared__ float outs[kProjRowsPerCTA][kID];
     const int tid = threadIdx.x;
     const int rr = tid >> 6, j = tid & 63;
-    const int64_t r0 = (int64_t)blockIdx.x * 4;
-    for (int e = tid; e < 4 * kD; e += 256) {
+    const int64_t r0 = (int64_t)blockIdx.x * kProjRowsPerCTA;
+    const uint32_t wbase = (uint32_t)__cvta_generic_to_shared(wsm);
+    for (int i = tid; i < kD * kID / 4; i += 256)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(wbase + 16u * i), "l"(W + 4 * i) : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    for (int e = tid; e < kProjRowsPerCTA * kD; e += 256) {
         const int64_t row = r0 + e / kD;
-        xs[e / kD][e % kD] = row < rows ? __uint_as_float(((uint32_t)__ldg(x + row * kD + e % kD)) << 16) : 0.0f;
+        xs[e] = row < rows ? __uint_as_float(((uint32_t)__ldg(x + row * kD + e % kD)) << 16) : 0.0f;
     }
-    const float4* W4 = reinterpret_cast<const float4*>(W);
-    float4 pre[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) pre[q] = __ldg(W4 + tid + 256 * q);   // chunk 0: 1024 float4
-#pragma unroll
-    for (int q = 0; q < 4; ++q) wbuf[0][tid + 256 * q] = pre[q];
+    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
+    const float* xr = xs + rr * kD;
     float acc = 0.0f;
-    constexpr int kChunks = kD / kRC;
-    for (int ch = 0; ch < kChunks; ++ch) {
-        const int cur = ch & 1;
-        if (ch + 1 < kChunks) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) pre[q] = __ldg(W4 + (ch + 1) * (kRC * kID / 4) + tid + 256 * q);
-        }
-        const float* wc = reinterpret_cast<const float*>(wbuf[cur]);
-        const float* xr = xs[rr] + ch * kRC;
 #pragma unroll 16
-        for (int c = 0; c < kRC; ++c) acc = __fmaf_rn(xr[c], wc[c * kID + j], acc);
-        if (ch + 1 < kChunks) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) wbuf[cur ^ 1][tid + 256 * q] = pre[q];
-        }
-        __syncthreads();
-    }
+    for (int c = 0; c < kD; ++c) acc = __fmaf_rn(xr[c], wsm[c * kID + j], acc);
     outs[rr][j] = acc;
     __syncthreads();
-    if (tid < 16) {
+    if (tid < 4 * kProjRowsPerCTA) {
         const int r2 = tid >> 2, g = tid & 3;
         const int64_t row2 = r0 + r2;
         if (row2 < rows) {
@@ -213,8 +200,15 @@ cudaError_t launch_index_k_proj(const void* x, int64_t rows, const float* W, uin
                                 const int64_t* dst_rows, int64_t out_rows, cudaStream_t st) {
     if (rows == 0) return cudaSuccess;
     if (rows <= 2048) {
-        index_k_proj_rows_kernel<<<(unsigned)((rows + 3) / 4), 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, W,
-                                                                             k_codes, k_scales, dst_rows, out_rows);
+        static bool attr = false;
+        if (!attr) {
+            cudaError_t e = cudaFuncSetAttribute(index_k_proj_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 kProjSmem);
+            if (e != cudaSuccess) return e;
+            attr = true;
+        }
+        index_k_proj_rows_kernel<<<(unsigned)((rows + kProjRowsPerCTA - 1) / kProjRowsPerCTA), 256, kProjSmem, st>>>(
+            static_cast<const uint16_t*>(x), rows, W, k_codes, k_scales, dst_rows, out_rows);
         return cudaGetLastError();
     }
     int64_t blocks = (rows + kPR - 1) / kPR;

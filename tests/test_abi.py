@@ -57,6 +57,8 @@ def test_invalid_arguments_rejected_before_launch(L):
     assert L.csa2_quant_nvfp4(fake, 4, 16, fake, fake, None, 3, None) == 1
     # rows == 0 is a no-op
     assert L.csa2_quant_nvfp4(None, 0, 16, None, None, None, 0, None) == 0
+    # projection matrix not 16-byte aligned
+    assert L.csa2_index_k_proj(fake, 4, P(0x1004), fake, fake, None, 4, None) == 1
     import sparse_attention_fp4_quant_b200 as csa
     kv = csa.csa2_kv(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 100, 3)  # m = 3 is invalid
     assert L.csa2_index_topk(fake, fake, fake, ctypes.byref(kv), fake, 1, 1, 512, fake, None, fake, 1 << 20,

@@ -111,6 +111,50 @@ def test_index_topk_ragged(csa, m, k):
     assert np.array_equal(np_(bm), rbm)
 
 
+def test_index_topk_many_queries(csa):
+    # 160 queries: more than one cluster per query can hold at once, so the
+    # streaming per-share kernel serves them (prefill-like causal positions)
+    B, Q, cap, m, k = 2, 80, 3000, 2, 512
+    n_entries = [3000, 2100]
+    rng = np.random.default_rng(5)
+    q_pos = rng.integers(0, 6000, size=(B, Q)).astype(np.int32)
+    q_pos[0, :4] = [0, 1, 1023, 5999]
+    grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(77, B, Q, cap, n_entries, m, q_pos.tolist(), k)
+    idx = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, k)
+    ridx = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, m, q_pos, k)
+    assert np.array_equal(np_(idx), ridx)
+
+
+@pytest.mark.parametrize("cap", [1001, 1002, 1004])
+def test_index_topk_capacity_not_multiple_of_4(csa, cap):
+    # rows of the cache that are not a whole number of 4-row groups take the
+    # per-share kernel; multiples of 4 take the cluster kernel
+    B, Q, m = 2, 1, 1
+    n_entries = [cap, cap - 3]
+    q_pos = [[cap - 1], [cap - 4]]
+    for k in (64, 512):
+        grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(90 + cap % 7, B, Q, cap, n_entries, m, q_pos, k)
+        idx, bm = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, k, blockmax=True)
+        ridx, rbm = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, m, np.array(q_pos, np.int32),
+                                      k, blockmax=True)
+        assert np.array_equal(np_(idx), ridx)
+        assert np.array_equal(np_(bm), rbm)
+
+
+def test_index_blockmax_signed_zero_and_negative_weights(csa):
+    # negative head weights make scores <= 0, with -0 and +0 in the same block;
+    # a block maximum keeps the first of equal values in position order
+    B, Q, cap, m, k = 1, 2, 4000, 1, 512
+    q_pos = [[3999, 2500]]
+    grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(95, B, Q, cap, [4000], m, q_pos, k)
+    w = torch.tensor([[[-0.25, 0.5, -0.75, 0.125], [-1.0, -0.5, -0.25, -0.125]]], dtype=torch.float32, device="cuda")
+    idx, bm = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, k, blockmax=True)
+    ridx, rbm = oracle.index_topk(oiq, oiqs, np_(w), o["ik"], o["iks"], grp.n_entries, m, np.array(q_pos, np.int32),
+                                  k, blockmax=True)
+    assert np.array_equal(np_(idx), ridx)
+    assert np.array_equal(np_(bm).view(np.uint32), rbm.view(np.uint32))   # bits, so -0 != +0
+
+
 def test_index_topk_ties_and_zero_scores(csa):
     B, Q, cap = 1, 3, 20000
     grp = Group(21, B, cap, [20000])
@@ -133,6 +177,18 @@ def test_index_topk_ties_and_zero_scores(csa):
         ridx = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, 1, q_pos, k)
         assert np.array_equal(np_(idx), ridx)
         assert list(np_(idx)[0, 2]) == list(range(k))
+
+
+def test_binding_rejects_mismatched_shapes(csa):
+    kv = csa.KV(1, 64, 1, "cuda")
+    q = torch.zeros((2, 1, 128), dtype=torch.uint8, device="cuda")
+    qs = torch.zeros((2, 1, 16), dtype=torch.uint8, device="cuda")
+    w = torch.zeros((2, 1, 4), dtype=torch.float32, device="cuda")
+    qp = torch.zeros((2, 1), dtype=torch.int32, device="cuda")
+    with pytest.raises(ValueError):   # two query rows, one cache row
+        csa.csa2_index_topk(q, qs, w, kv, qp, 8)
+    with pytest.raises(ValueError):   # q of the wrong size
+        csa.csa2_index_topk(q[:1, :, :64].contiguous(), qs[:1], w[:1], kv, qp[:1], 8)
 
 
 # ---------------------------------------------------------------- pool
@@ -193,9 +249,10 @@ def test_sparse_attn_decode(csa, B, Q):
 
 
 @pytest.mark.parametrize("window", [1, 2, 4, 77, 128])
-def test_sparse_attn_replay_mask(csa, window):
-    B, Q, cap, k, T = 2, 128, 3000, 64, 128
-    rng = np.random.default_rng(window)
+@pytest.mark.parametrize("Q", [8, 128])   # 16 queries: one cluster each; 256: split-K kernel
+def test_sparse_attn_replay_mask(csa, window, Q):
+    B, cap, k, T = 2, 3000, 64, 128
+    rng = np.random.default_rng(window + Q)
     s = [3000 - 128, 2500]
     q_pos = [[s[b] + qi for qi in range(Q)] for b in range(B)]
     pos0 = [s[0], s[1] - 3]
