@@ -5,20 +5,19 @@
 // Each CTA scores a contiguous 1/C of the query's visible entries with the
 // tcgen05 pipeline of index_pipe.cuh (permuted tiles: TMEM row m of a tile is
 // entry 4 (m % 32) + m / 32, so a stage is one TMA box per tile plus one bulk
-// copy of its scales) and keeps every order key in shared memory (at most
-// 32,768 per CTA, in TMEM-row order), while the epilogue counts the keys' top
-// 11 bits into a 2,048-bin histogram.  The cluster then finds the K-th largest
-// key T exactly in three radix passes (bits 31..21, 20..10, 9..0): each pass
-// sums the CTAs' histograms through distributed shared memory and locates the
-// bin holding the K-th key from the top.  After the first pass one ordered
-// sweep over the CTA's keys copies every key at or above the first-pass bin
-// (with its position) into a short per-warp list, which the later passes and
-// the output read instead of the whole key array (a list that would overflow
-// sends its CTA back to the whole array; the results are the same).  The
+// copy of its scales; 8 stages in flight) and keeps every order key in TMEM
+// (lane m, one column per tile: up to 32,768 keys beside the pipeline's 256
+// columns), while the epilogue counts the keys' top 11 bits into a 2,048-bin
+// histogram.  The cluster then finds the K-th largest key T exactly in three
+// radix passes (bits 31..21, 20..10, 9..0): each pass sums the CTAs'
+// histograms through distributed shared memory and locates the bin holding
+// the K-th key from the top; passes 2 and 3 re-read the keys from TMEM.  The
 // selected set is every key above T plus the lowest-positioned keys equal to T
-// (ties go to the lower position).  CTA r covers positions below those of CTA
-// r + 1 and each warp a contiguous run of its CTA, so writing each run's
-// survivors at a prefix-summed offset yields the positions in ascending order.
+// (ties go to the lower position).  A last read marks both kinds in position
+// bitmaps; CTA r covers positions below those of CTA r + 1, so its quota of
+// ties and its output offset follow from the lower-ranked CTAs' counts, and
+// two block-wide prefix sums over the bitmap words give every selected
+// position its place in the ascending output.
 //
 // Every mbarrier wait of the scoring pipeline is bounded; every thread of
 // every CTA reaches each cluster barrier (and each named barrier of its warp
@@ -35,24 +34,27 @@ using namespace pipe;
 constexpr int kThreads = 320;              // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int kEpiN = 256;
 constexpr int kTPG = kTPS / 2;             // tiles of a stage per epilogue warp group
-constexpr int kMaxKeys = 32768;            // order keys one CTA keeps in shared memory
+constexpr int kRing = 8;                   // shared-memory stages in flight
+constexpr int kMaxTiles = 256;             // 32,768 entries per CTA
+constexpr uint32_t kColKeys = kPipeCols;   // key of tile g, row m: TMEM lane m, column kColKeys + g
+constexpr uint32_t kTmemCols = kPipeCols + kMaxTiles;
+constexpr int kWords = kMaxTiles * kTile / 32;          // bitmap words over the CTA's entries
 constexpr int kNB1 = 2048, kNB2 = 2048, kNB3 = 1024;   // radix digits: bits 31..21, 20..10, 9..0
-constexpr int kSel = 256;                  // threads of the select phase (warps 0-7)
+constexpr int kSel = 256;                  // threads of the scans (warps 0-7)
 constexpr int kSelWarps = kSel / 32;
-constexpr int kSegCap = 512;               // candidate list capacity per select warp
-static_assert((kNB2 + kNB3) * 4 + kSelWarps * kSegCap * 8 <= (int)sizeof(Pipe::A), "select scratch fits the ring");
+using ClPipe = Pipe<kRing>;
+static_assert((kNB2 + kNB3 + 2 * kWords) * 4 <= (int)sizeof(ClPipe::A), "select scratch fits the ring");
+static_assert(kTmemCols == 512, "TMEM");
 
 struct ClSmem {
-    Pipe pipe;                              // its A ring holds hist2, hist3 and the candidate lists after scoring
+    ClPipe pipe;                            // its A ring holds hist2, hist3 and two bitmaps after scoring
     alignas(16) uint32_t hist1[kNB1];
-    alignas(16) uint32_t keys[kMaxKeys];    // key of TMEM row m of tile g at g * 128 + m (0 past the CTA's range)
     float bmx[2][2][kTPG][kTile];           // block-max staging: [group][stage parity][tile][entry in tile]
     uint32_t wsum[kSelWarps];               // scan: per-warp totals
-    uint32_t res[2];                        // scan: (bin, keys above the bin)
-    uint32_t segn[kSelWarps];               // candidates found per select warp (may exceed kSegCap)
-    uint32_t wgt[kSelWarps], weq[kSelWarps];   // per-warp counts of keys > T and == T
+    uint32_t res[2];                        // find_bin: (bin, keys above the bin)
+    uint32_t wcnt[8][2];                    // per sweeping warp: keys > T, keys == T
     alignas(8) uint32_t pub[2];             // this CTA's (> T, == T) counts, read by the cluster
-    uint32_t wbase[kSelWarps][2];           // per-warp (tie rank, output offset) at the start of its run
+    uint32_t cbase[2];                      // this CTA's tie quota and output offset
 };
 
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
@@ -64,10 +66,26 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
     return v;
 }
 
-__device__ __forceinline__ uint32_t lanemask_lt(int lane) { return (1u << lane) - 1u; }
-
 __device__ __forceinline__ void group_bar(int group) {
     asm volatile("bar.sync %0, 128;" ::"r"(2 + group) : "memory");
+}
+
+// Exclusive prefix of v over threads 0..255 in thread order (threads 256+ pass
+// 0 and get nothing useful); *total = the sum.  All threads of the CTA call it.
+__device__ __forceinline__ uint32_t block_scan_excl(ClSmem& s, uint32_t v, int tid, uint32_t* total) {
+    const int warp = tid >> 5, lane = tid & 31;
+    const uint32_t inc = warp_incl_scan(v, lane);
+    if (lane == 31 && warp < kSelWarps) s.wsum[warp] = inc;
+    __syncthreads();
+    uint32_t pre = inc - v, tot = 0;
+#pragma unroll
+    for (int w = 0; w < kSelWarps; ++w) {
+        if (w < warp) pre += s.wsum[w];
+        tot += s.wsum[w];
+    }
+    *total = tot;
+    __syncthreads();
+    return pre;
 }
 
 // Sum the NB-bin histogram `hist` over the cluster's CTAs and find the bin b
@@ -136,6 +154,24 @@ __device__ __forceinline__ void find_bin(ClSmem& s, const uint32_t* hist, uint32
     __syncthreads();
 }
 
+// Visit every stored key of this CTA: warps 2-9, TMEM lane quarter warp % 4,
+// tile columns [128 h, 128 h + 128) with h = (warp - 2) / 4.  f(key, entry)
+// gets the CTA-local entry 128 c + 4 lane + quarter of column c.
+template <class F>
+__device__ __forceinline__ void sweep_keys(uint32_t tbase, int warp, int lane, int ntiles, F&& f) {
+    if (warp < 2) return;
+    const int quarter = warp & 3, half = (warp - 2) >> 2;
+    const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
+    for (int c0 = half * 128; c0 < min(ntiles, half * 128 + 128); c0 += 32) {
+        uint32_t v[32];
+        tc::tmem_ld_32x32b_x32(tbase + lanes + kColKeys + (uint32_t)c0, v);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (c0 + j < ntiles) f(v[j], (c0 + j) * kTile + 4 * lane + quarter);
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     index_cluster_kernel(SelectParams p, const __grid_constant__ CUtensorMap tmap) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -147,17 +183,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int k = p.k;
     const int nvis = n_visible(p.q_pos[bq], p.n_entries[b], p.m, p.cap);
     const int64_t row_base = (int64_t)b * p.cap;
-    // this CTA's entries [lo, hi); the host keeps the chunk within kMaxKeys
+    // this CTA's entries [lo, hi); the host keeps the chunk within kMaxTiles tiles
     const int chunk = ((nvis + (int)C - 1) / (int)C + kTile - 1) / kTile * kTile;
     const int lo = min(nvis, (int)rank * chunk), hi = min(nvis, lo + chunk);
     const int ntiles = (hi - lo + kTile - 1) / kTile;
     const int nstages = (ntiles + kTPS - 1) / kTPS;
-    const int npad = ntiles * kTile;
     int32_t* status = p.status;
     int32_t* out = p.out + (int64_t)bq * k;
 
     if (tid == 0) init_barriers(s.pipe, 1, kEpiN);
-    if (warp == 1) setup_query(s.pipe, p.q + (int64_t)bq * 128, p.q_sc + (int64_t)bq * 16, lane);
+    if (warp == 1) setup_query(s.pipe, p.q + (int64_t)bq * 128, p.q_sc + (int64_t)bq * 16, lane, kTmemCols);
     for (int i = tid; i < kNB1; i += kThreads) s.hist1[i] = 0;
     __syncthreads();
     const uint32_t tbase = s.pipe.tmem_base;
@@ -170,8 +205,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;             // TMEM lanes this warp may read
         const int group = (warp - 2) >> 2;        // tiles 2*group, 2*group+1 of each stage
-        const int m = quarter * 32 + lane;        // TMEM row
-        const int eo = 4 * lane + quarter;        // its entry within the tile
+        const int eo = 4 * lane + quarter;        // entry of this thread's TMEM row within a tile
+        const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
         const float w0 = __ldg(p.w + (int64_t)bq * 4 + 0), w1 = __ldg(p.w + (int64_t)bq * 4 + 1);
         const float w2 = __ldg(p.w + (int64_t)bq * 4 + 2), w3 = __ldg(p.w + (int64_t)bq * 4 + 3);
         float* bm = p.blockmax ? p.blockmax + (int64_t)bq * p.nb_cap : nullptr;
@@ -189,23 +224,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t v[kTPG][16];
 #pragma unroll
                 for (int j = 0; j < kTPG; ++j)
-                    tc::tmem_ld_32x32b_x16(tbase + ((uint32_t)(quarter * 32) << 16) + kColAcc +
-                                               (uint32_t)(a * kTPS + kTPG * group + j) * 16,
-                                           v[j]);
+                    tc::tmem_ld_32x32b_x16(tbase + lanes + kColAcc + (uint32_t)(a * kTPS + kTPG * group + j) * 16, v[j]);
                 tc::tmem_ld_wait();
                 tc::tc_fence_before();
                 tc::mbar_arrive(&s.pipe.accempty[a]);
+                const int g0 = t * kTPS + kTPG * group;
+                uint32_t key[kTPG];
 #pragma unroll
                 for (int j = 0; j < kTPG; ++j) {
-                    const int g = t * kTPS + kTPG * group + j;
-                    if (g >= ntiles) continue;   // warp-uniform
-                    const bool valid = lo + g * kTile + eo < hi;
+                    const int g = g0 + j;
+                    const bool valid = g < ntiles && lo + g * kTile + eo < hi;
                     const float score = valid ? score_of(v[j], w0, w1, w2, w3) : -INFINITY;
-                    const uint32_t key = valid ? score_key(score) : 0u;
-                    s.keys[g * kTile + m] = key;
-                    if (valid) atomicAdd(&s.hist1[key >> 21], 1u);
+                    key[j] = valid ? score_key(score) : 0u;
+                    if (valid) atomicAdd(&s.hist1[key[j] >> 21], 1u);
                     if (bm) s.bmx[group][t & 1][j][eo] = score;
                 }
+                if (g0 + 1 < ntiles) tc::tmem_st_32x32b_x2(tbase + lanes + kColKeys + (uint32_t)g0, key[0], key[1]);
+                else if (g0 < ntiles) tc::tmem_st_32x32b_x1(tbase + lanes + kColKeys + (uint32_t)g0, key[0]);
             }
             if (bm) {
                 // block maxima in position order: the first strictly larger score wins
@@ -224,6 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
+        tc::tmem_st_wait();
         if (bm) {  // blocks with no visible position, split over the cluster
             const int64_t jb = (nvis + kBlk - 1) / kBlk;
             const int64_t rest = p.nb_cap - jb;
@@ -234,115 +270,71 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     }
+    tc::tc_fence_before();
     __syncthreads();
-    if (warp == 1) tc::tmem_dealloc(tbase, kTmemCols);
+    tc::tc_fence_after();
 
     // ---------------------------------------------------------------- select
     const uint32_t K1 = (uint32_t)min(k, nvis);
     if (K1 == 0) {   // the same for every CTA of the cluster: nothing visible
         if (rank == 0)
             for (int i = tid; i < k; i += kThreads) out[i] = -1;
+        if (warp == 1) tc::tmem_dealloc(tbase, kTmemCols);
         return;
     }
     uint32_t* hist2 = reinterpret_cast<uint32_t*>(&s.pipe.A[0][0][0]);
     uint32_t* hist3 = hist2 + kNB2;
-    uint2* seg = reinterpret_cast<uint2*>(hist3 + kNB3) + (warp < kSelWarps ? warp : 0) * kSegCap;
-    for (int i = tid; i < kNB2 + kNB3; i += kThreads) hist2[i] = 0;
-    // warp w < 8 owns keys [wlo, whi) of this CTA (whole tiles), in position order
-    const int Lw = ((npad + kSelWarps - 1) / kSelWarps + kTile - 1) / kTile * kTile;
-    const int wlo = min(npad, warp * Lw), whi = min(npad, wlo + Lw);
+    uint32_t* selbm = hist3 + kNB3;   // entries above T (then also the ties taken)
+    uint32_t* tiebm = selbm + kWords; // entries equal to T
+    for (int i = tid; i < kNB2 + kNB3 + 2 * kWords; i += kThreads) hist2[i] = 0;
 
     cl::sync();                                   // every CTA's hist1 is complete
     find_bin<kNB1>(s, s.hist1, C, K1, tid);
     const uint32_t d1 = s.res[0];
     uint32_t R = K1 - s.res[1];
-
-    // one ordered sweep: the candidates (first digit >= d1) into this warp's list,
-    // the second-digit histogram of the keys whose first digit is d1
-    if (warp < kSelWarps) {
-        uint32_t n = 0;
-        for (int base = wlo; base < whi; base += kTile) {
-            uint32_t kk[4], c = 0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                kk[j] = s.keys[base + 32 * j + lane];   // entry base + 4 lane + j
-                const uint32_t d = kk[j] >> 21;
-                if (d == d1) atomicAdd(&hist2[(kk[j] >> 10) & (kNB2 - 1)], 1u);
-                c += (uint32_t)(d >= d1);
-            }
-            if (__ballot_sync(0xFFFFFFFFu, c != 0) == 0) continue;   // warp-uniform
-            const uint32_t inc = warp_incl_scan(c, lane);
-            uint32_t o = n + inc - c;
-            n += __shfl_sync(0xFFFFFFFFu, inc, 31);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                if ((kk[j] >> 21) >= d1) {
-                    if (o < (uint32_t)kSegCap) seg[o] = make_uint2(kk[j], (uint32_t)(base + 4 * lane + j));
-                    ++o;
-                }
-            }
-        }
-        if (lane == 0) s.segn[warp] = n;
-    }
+    sweep_keys(tbase, warp, lane, ntiles, [&](uint32_t key, int) {
+        if ((key >> 21) == d1) atomicAdd(&hist2[(key >> 10) & (kNB2 - 1)], 1u);
+    });
     cl::sync();
     find_bin<kNB2>(s, hist2, C, R, tid);
     const uint32_t p2 = (d1 << 11) | s.res[0];
     R -= s.res[1];
-    bool whole = false;   // some list overflowed: this CTA reads its whole key array
-#pragma unroll
-    for (int w = 0; w < kSelWarps; ++w) whole |= s.segn[w] > (uint32_t)kSegCap;
-    const uint32_t nseg = warp < kSelWarps ? min(s.segn[warp], (uint32_t)kSegCap) : 0u;
-
-    if (whole) {
-        for (int i = tid; i < npad; i += kThreads) {
-            const uint32_t key = s.keys[i];
-            if ((key >> 10) == p2) atomicAdd(&hist3[key & (kNB3 - 1)], 1u);
-        }
-    } else if (warp < kSelWarps) {
-        for (uint32_t i = lane; i < nseg; i += 32) {
-            const uint32_t key = seg[i].x;
-            if ((key >> 10) == p2) atomicAdd(&hist3[key & (kNB3 - 1)], 1u);
-        }
-    }
+    sweep_keys(tbase, warp, lane, ntiles, [&](uint32_t key, int) {
+        if ((key >> 10) == p2) atomicAdd(&hist3[key & (kNB3 - 1)], 1u);
+    });
     cl::sync();
     find_bin<kNB3>(s, hist3, C, R, tid);
     const uint32_t T = (p2 << 10) | s.res[0];
-    R -= s.res[1];   // ties at T still to take, in position order (1 <= R)
+    R -= s.res[1];   // ties at T still to take, lowest positions first (1 <= R)
 
     // ---------------------------------------------------------------- output
-    if (warp < kSelWarps) {
-        uint32_t gt = 0, eq = 0;
-        if (whole) {
-            for (int base = wlo; base < whi; base += kTile)
+    uint32_t gt = 0, eq = 0;
+    sweep_keys(tbase, warp, lane, ntiles, [&](uint32_t key, int e) {
+        if (key > T) {
+            atomicOr(&selbm[e >> 5], 1u << (e & 31));
+            ++gt;
+        } else if (key == T) {
+            atomicOr(&tiebm[e >> 5], 1u << (e & 31));
+            ++eq;
+        }
+    });
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t key = s.keys[base + 32 * j + lane];
-                    gt += (uint32_t)(key > T);
-                    eq += (uint32_t)(key == T);
-                }
-        } else {
-            for (uint32_t i = lane; i < nseg; i += 32) {
-                const uint32_t key = seg[i].x;
-                gt += (uint32_t)(key > T);
-                eq += (uint32_t)(key == T);
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            gt += __shfl_xor_sync(0xFFFFFFFFu, gt, o);
-            eq += __shfl_xor_sync(0xFFFFFFFFu, eq, o);
-        }
-        if (lane == 0) {
-            s.wgt[warp] = gt;
-            s.weq[warp] = eq;
-        }
+    for (int o = 16; o > 0; o >>= 1) {
+        gt += __shfl_xor_sync(0xFFFFFFFFu, gt, o);
+        eq += __shfl_xor_sync(0xFFFFFFFFu, eq, o);
     }
+    if (warp >= 2 && lane == 0) {
+        s.wcnt[warp - 2][0] = gt;
+        s.wcnt[warp - 2][1] = eq;
+    }
+    tc::tc_fence_before();
     __syncthreads();
+    if (warp == 1) tc::tmem_dealloc(tbase, kTmemCols);   // no TMEM reads past this point
     if (tid == 0) {
         uint32_t g = 0, e = 0;
-        for (int w = 0; w < kSelWarps; ++w) {
-            g += s.wgt[w];
-            e += s.weq[w];
+        for (int w = 0; w < 8; ++w) {
+            g += s.wcnt[w][0];
+            e += s.wcnt[w][1];
         }
         s.pub[0] = g;
         s.pub[1] = e;
@@ -358,69 +350,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tb = warp_incl_scan(e, lane) - e;             // ties in lower-ranked CTAs
         const uint32_t take = tb < R ? min(e, R - tb) : 0u;
         const uint32_t ob = warp_incl_scan(g + take, lane) - (g + take);
-        uint32_t t = __shfl_sync(0xFFFFFFFFu, tb, (int)rank), o = __shfl_sync(0xFFFFFFFFu, ob, (int)rank);
+        const uint32_t my_take = __shfl_sync(0xFFFFFFFFu, take, (int)rank);
+        const uint32_t my_ob = __shfl_sync(0xFFFFFFFFu, ob, (int)rank);
         if (lane == 0) {
-            for (int w = 0; w < kSelWarps; ++w) {
-                s.wbase[w][0] = t;
-                s.wbase[w][1] = o;
-                const uint32_t tw = t < R ? min(s.weq[w], R - t) : 0u;
-                t += s.weq[w];
-                o += s.wgt[w] + tw;
-            }
+            s.cbase[0] = my_take;
+            s.cbase[1] = my_ob;
         }
     }
     __syncthreads();
-    if (warp < kSelWarps) {
-        uint32_t tie = s.wbase[warp][0], ob = s.wbase[warp][1];
-        if (whole) {
-            for (int base = wlo; base < whi; base += kTile) {
-                uint32_t kk[4];
-                uint32_t ne = 0, any = 0;
+    // take the lowest-positioned `quota` ties: thread t owns bitmap words 4t .. 4t + 3
+    const uint32_t quota = s.cbase[0];
+    uint32_t tw[4] = {0u, 0u, 0u, 0u}, nt = 0;
+    if (tid < kSel) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    kk[j] = s.keys[base + 32 * j + lane];   // entry base + 4 lane + j
-                    ne += (uint32_t)(kk[j] == T);
-                    any |= (uint32_t)(kk[j] >= T);
-                }
-                if (__ballot_sync(0xFFFFFFFFu, any) == 0) continue;   // warp-uniform
-                const uint32_t ne_inc = warp_incl_scan(ne, lane);
-                uint32_t tr = tie + ne_inc - ne;
-                tie += __shfl_sync(0xFFFFFFFFu, ne_inc, 31);
-                uint32_t sel = 0, ns = 0;
+        for (int j = 0; j < 4; ++j) {
+            tw[j] = tiebm[4 * tid + j];
+            nt += __popc(tw[j]);
+        }
+    }
+    uint32_t total;
+    uint32_t tpre = block_scan_excl(s, nt, tid, &total);
+    uint32_t sw[4] = {0u, 0u, 0u, 0u}, ns = 0;
+    if (tid < kSel) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    if (kk[j] > T) {
-                        sel |= 1u << j;
-                    } else if (kk[j] == T) {
-                        if (tr < R) sel |= 1u << j;
-                        ++tr;
-                    }
-                    ns += (sel >> j) & 1u;
-                }
-                const uint32_t ns_inc = warp_incl_scan(ns, lane);
-                uint32_t o = ob + ns_inc - ns;
-                ob += __shfl_sync(0xFFFFFFFFu, ns_inc, 31);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    if ((sel >> j) & 1u) {
-                        if (o < (uint32_t)k) out[o] = lo + base + 4 * lane + j;
-                        ++o;
-                    }
-                }
+        for (int j = 0; j < 4; ++j) {
+            uint32_t m = tw[j], keep = 0;
+            while (m != 0u && tpre < quota) {
+                const uint32_t low = m & (0u - m);
+                keep |= low;
+                m ^= low;
+                ++tpre;
             }
-        } else {
-            for (uint32_t i0 = 0; i0 < nseg; i0 += 32) {
-                const uint32_t i = i0 + lane;
-                const uint2 ce = i < nseg ? seg[i] : make_uint2(0u, 0u);
-                const bool gt = i < nseg && ce.x > T, eq = i < nseg && ce.x == T;
-                const uint32_t eqb = __ballot_sync(0xFFFFFFFFu, eq);
-                const uint32_t tr = tie + __popc(eqb & lanemask_lt(lane));
-                tie += __popc(eqb);
-                const bool sel = gt || (eq && tr < R);
-                const uint32_t sb = __ballot_sync(0xFFFFFFFFu, sel);
-                const uint32_t o = ob + __popc(sb & lanemask_lt(lane));
-                ob += __popc(sb);
-                if (sel && o < (uint32_t)k) out[o] = lo + (int)ce.y;
+            sw[j] = selbm[4 * tid + j] | keep;
+            ns += __popc(sw[j]);
+        }
+    }
+    uint32_t o = s.cbase[1] + block_scan_excl(s, ns, tid, &total);
+    if (tid < kSel) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t m = sw[j];
+            while (m != 0u) {
+                const int bit = __ffs(m) - 1;
+                m &= m - 1u;
+                if (o < (uint32_t)k) out[o] = lo + 32 * (4 * tid + j) + bit;
+                ++o;
             }
         }
     }
@@ -484,7 +458,7 @@ int index_cluster_size(const SelectParams& p) {
     for (int C = g_nonportable ? 16 : 8; C >= 1; C >>= 1) {
         if ((int64_t)bq * C > kNumSMs) continue;
         const int64_t chunk = ((p.cap + C - 1) / C + kTile - 1) / kTile * kTile;
-        if (chunk > kMaxKeys) return 0;   // a smaller cluster only lengthens the chunk
+        if (chunk > (int64_t)kMaxTiles * kTile) return 0;   // a smaller cluster only lengthens the chunk
         if (max_active_clusters(C, bq, smem_bytes()) >= bq) return C;
     }
     return 0;

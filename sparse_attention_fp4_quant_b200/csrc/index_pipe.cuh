@@ -30,37 +30,42 @@ namespace pipe {
 
 constexpr int kTile = 128;       // rows per MMA (M)
 constexpr int kTPS = 4;          // tiles per pipeline stage
-constexpr int kStages = 4;       // smem stages
-constexpr int kAcc = 2;          // accumulator stages
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColAcc = 0, kColSfa = kAcc * kTPS * 16, kColSfb = kColSfa + kStages * kTPS * 4;
-static_assert(kColSfb + 4 <= kTmemCols, "TMEM columns");
+constexpr int kAcc = 2;          // accumulator stages (each with its own scale-factor slot)
+constexpr uint32_t kPipeCols = 256;   // TMEM columns of the pipeline (a power of two)
+constexpr uint32_t kColAcc = 0, kColSfa = kAcc * kTPS * 16, kColSfb = kColSfa + kAcc * kTPS * 4;
+static_assert(kColSfb + 4 <= kPipeCols, "TMEM columns");
 constexpr uint32_t kIdesc = tc::idesc_mxf4nvf4(128, 16);
 constexpr int kPoolPerTile = kTile / kBlk;   // 16 pool blocks of 8 rows per tile
 
-// Shared-memory part of the pipeline.  Must start on a 1024-byte boundary.
+// Shared-memory part of the pipeline with ST ring stages.  Must start on a
+// 1024-byte boundary.
+template <int ST>
 struct Pipe {
-    uint8_t A[kStages][kTPS][kTile * 32];   // K-major, 32-byte swizzle (written by TMA)
-    uint8_t SF[kStages][kTPS][512];         // scale bytes in the 32 x (4 x 4 B) TMEM-copy layout
-    uint8_t Bq[16 * 32];                    // block-diagonal query, no swizzle, K-major
-    uint8_t SFB[512];                       // its scales, TMEM-copy layout
-    uint64_t full[kStages], empty[kStages], accfull[kAcc], accempty[kAcc], done;
+    static constexpr int kStages = ST;
+    uint8_t A[ST][kTPS][kTile * 32];   // K-major, 32-byte swizzle (written by TMA)
+    uint8_t SF[ST][kTPS][512];         // scale bytes in the 32 x (4 x 4 B) TMEM-copy layout
+    uint8_t Bq[16 * 32];               // block-diagonal query, no swizzle, K-major
+    uint8_t SFB[512];                  // its scales, TMEM-copy layout
+    uint64_t full[ST], empty[ST], accfull[kAcc], accempty[kAcc], done;
     uint32_t tmem_base;
     int abort_flag;
 };
 
-__device__ __forceinline__ void raise_abort(Pipe& s, int32_t* status) {
+template <class P>
+__device__ __forceinline__ void raise_abort(P& s, int32_t* status) {
     *reinterpret_cast<volatile int*>(&s.abort_flag) = 1;
     if (status) atomicExch(status, 1);
 }
 
-__device__ __forceinline__ bool aborted(const Pipe& s) { return *reinterpret_cast<const volatile int*>(&s.abort_flag) != 0; }
+template <class P>
+__device__ __forceinline__ bool aborted(const P& s) { return *reinterpret_cast<const volatile int*>(&s.abort_flag) != 0; }
 
 // One thread: barrier init.  `full_arrivals` = arrivals that fill a stage (the
 // expect_tx arrive, plus 32 cp.async arrivals when the scales come by cp.async);
 // `epi_arrivals` = arrivals that free an accumulator stage.
-__device__ __forceinline__ void init_barriers(Pipe& s, uint32_t full_arrivals, uint32_t epi_arrivals) {
-    for (int i = 0; i < kStages; ++i) {
+template <class P>
+__device__ __forceinline__ void init_barriers(P& s, uint32_t full_arrivals, uint32_t epi_arrivals) {
+    for (int i = 0; i < P::kStages; ++i) {
         tc::mbar_init(&s.full[i], full_arrivals);
         tc::mbar_init(&s.empty[i], 1);       // MMA commit
     }
@@ -73,10 +78,12 @@ __device__ __forceinline__ void init_barriers(Pipe& s, uint32_t full_arrivals, u
     tc::fence_mbar_init();
 }
 
-// Warp 1: allocate TMEM and lay out the block-diagonal query operand.
-// Row n = 4h + b keeps head h's 8 code bytes of block b; all else zero.
-__device__ __forceinline__ void setup_query(Pipe& s, const uint8_t* q, const uint8_t* qs, int lane) {
-    tc::tmem_alloc(&s.tmem_base, kTmemCols);
+// Warp 1: allocate `cols` TMEM columns (the pipeline uses the first kPipeCols)
+// and lay out the block-diagonal query operand.  Row n = 4h + b keeps head h's
+// 8 code bytes of block b; all else zero.
+template <class P>
+__device__ __forceinline__ void setup_query(P& s, const uint8_t* q, const uint8_t* qs, int lane, uint32_t cols) {
+    tc::tmem_alloc(&s.tmem_base, cols);
     for (int i = lane; i < 16 * 32; i += 32) s.Bq[i] = 0;
     for (int i = lane; i < 512; i += 32) s.SFB[i] = 0;
     __syncwarp();
@@ -95,10 +102,11 @@ __device__ __forceinline__ void setup_query(Pipe& s, const uint8_t* q, const uin
 
 // Warp 0.  MODE 0: rows [lo, hi) of the query's batch row (tiles of 128);
 // MODE 1: the pool slots [lo, hi), 16 blocks of 8 rows per tile.
-template <int MODE>
-__device__ __forceinline__ void producer(Pipe& s, const CUtensorMap* tmap, const uint8_t* iks, int64_t row_base,
+template <int MODE, class P>
+__device__ __forceinline__ void producer(P& s, const CUtensorMap* tmap, const uint8_t* iks, int64_t row_base,
                                          int lo, int hi, int ntiles, int nstages, const int32_t* pool, int nvis,
                                          int32_t* status, int lane) {
+    constexpr int kStages = P::kStages;
     int issued = 0;
     for (int t = 0; t < nstages; ++t) {
         const int slot = t % kStages;
@@ -183,8 +191,10 @@ __device__ __forceinline__ void producer(Pipe& s, const CUtensorMap* tmap, const
 // tile (3-D map: 32 bytes x 32 groups of 4 rows x 4 rows) and one bulk copy of
 // its contiguous scale bytes.  Needs lo, the batch row base and the cache
 // capacity to be multiples of 4 and 16-byte aligned scales.
-__device__ __forceinline__ void producer_perm(Pipe& s, const CUtensorMap* tmap3, const uint8_t* iks, int64_t row_base,
+template <class P>
+__device__ __forceinline__ void producer_perm(P& s, const CUtensorMap* tmap3, const uint8_t* iks, int64_t row_base,
                                               int lo, int hi, int ntiles, int nstages, int32_t* status, int lane) {
+    constexpr int kStages = P::kStages;
     int issued = 0;
     if (lane == 0) {
         for (int t = 0; t < nstages; ++t) {
@@ -214,7 +224,9 @@ __device__ __forceinline__ void producer_perm(Pipe& s, const CUtensorMap* tmap3,
 }
 
 // Warp 1 (lane 0 issues).  Returns once every MMA it issued has completed.
-__device__ __forceinline__ void mma_issuer(Pipe& s, int ntiles, int nstages, int32_t* status, int lane) {
+template <class P>
+__device__ __forceinline__ void mma_issuer(P& s, int ntiles, int nstages, int32_t* status, int lane) {
+    constexpr int kStages = P::kStages;
     const uint32_t tbase = s.tmem_base;
     if (lane == 0) {
         tc::tc_fence_after();
@@ -235,7 +247,7 @@ __device__ __forceinline__ void mma_issuer(Pipe& s, int ntiles, int nstages, int
             tc::fence_proxy_async_smem();   // scale bytes came through cp.async (generic proxy)
             for (int i = 0; i < kTPS; ++i) {
                 if (t * kTPS + i >= ntiles) break;
-                const uint32_t sfa = tbase + kColSfa + (uint32_t)(slot * kTPS + i) * 4;
+                const uint32_t sfa = tbase + kColSfa + (uint32_t)(a * kTPS + i) * 4;   // free once stage t - kAcc is read
                 tc::tmem_cp_32x128_x4(sfa, tc::smem_desc(tc::smem_u32(s.SF[slot][i]), 16, 128, tc::kLayoutNone));
                 const uint64_t adesc = tc::smem_desc(tc::smem_u32(s.A[slot][i]), 16, 256, tc::kLayoutSw32);
                 tc::mma_mxf4nvf4(tbase + kColAcc + (uint32_t)(a * kTPS + i) * 16, adesc, bdesc, kIdesc, 0u, sfa,

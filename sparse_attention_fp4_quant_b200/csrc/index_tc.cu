@@ -20,7 +20,7 @@ constexpr int kTPG = kTPS / 2;   // tiles of a stage per epilogue warp group
 
 template <int CAP>
 struct TcSmem {
-    Pipe pipe;
+    Pipe<4> pipe;
     int last;
     typename TopK<kEpiN, CAP, 1, kEpiT0>::Smem topk;
 };
@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int32_t* pool = (MODE == 1) ? p.pool + (int64_t)bq * p.P : nullptr;
 
     if (tid == 0) init_barriers(s.pipe, 1 + 32, kEpiN);
-    if (warp == 1) setup_query(s.pipe, p.q + (int64_t)bq * 128, p.q_sc + (int64_t)bq * 16, lane);
+    if (warp == 1) setup_query(s.pipe, p.q + (int64_t)bq * 128, p.q_sc + (int64_t)bq * 16, lane, kPipeCols);
     __syncthreads();
     const uint32_t tbase = s.pipe.tmem_base;
     int32_t* status = p.status;
@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!stop) tk.finish(k);
     }
     __syncthreads();
-    if (warp == 1) tc::tmem_dealloc(tbase, kTmemCols);
+    if (warp == 1) tc::tmem_dealloc(tbase, kPipeCols);
     if (warp < 2 || aborted(s.pipe)) return;
 
     // ---------------------------------------------------------------- output
