@@ -154,13 +154,19 @@ class DecodeGroup:
         nbytes = max(csa.csa2_workspace_bytes(csa.OP_INDEX_TOPK, B, 1, N_CTX, TOPK),
                      csa.csa2_workspace_bytes(csa.OP_SPARSE_ATTN, B, 1, N_CTX, TOPK))
         self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        self.side = torch.cuda.Stream(device=device)
 
-    # the three segments of a step (each is captured into its own CUDA graph)
+    # the three segments of a step
     def front(self):
+        """Append the new tokens (latent + indexer K, one launch) while, on a second
+        branch, the indexer query is quantised (the two are independent)."""
         c = self.csa
-        c.csa2_quant_nvfp4(self.new_lat, self.kv.lat.view(-1, 256), self.kv.lat_sc.view(-1, 32), self.new_rows)
-        c.csa2_index_k_proj(self.new_lat, self.W, self.kv.ik.view(-1, 32), self.kv.ik_sc.view(-1, 4), self.new_rows)
-        c.csa2_quant_nvfp4(self.iq_bf.view(-1, 64), self.iq.view(-1, 32), self.iqs.view(-1, 4))
+        cur = torch.cuda.current_stream()
+        self.side.wait_stream(cur)
+        with torch.cuda.stream(self.side):
+            c.csa2_quant_nvfp4(self.iq_bf.view(-1, 64), self.iq.view(-1, 32), self.iqs.view(-1, 4))
+        c.csa2_append_tokens(self.new_lat, self.W, self.kv, self.new_rows)
+        cur.wait_stream(self.side)
 
     def index(self):
         self.csa.csa2_index_topk(self.iq, self.iqs, self.w, self.kv, self.q_pos, TOPK, self.idx, ws=self.ws)
@@ -171,7 +177,12 @@ class DecodeGroup:
             self.csa.csa2_sparse_attn(self.q[li], self.kv, self.idx, swa, swa_sc, self.swa_pos0, self.q_pos,
                                       out=self.out[li], ws=self.ws)
 
-    LAUNCHES_PER_STEP = 3 + 1 + len(LAYERS)
+    def step(self):
+        self.front()
+        self.index()
+        self.attention()
+
+    LAUNCHES_PER_STEP = 2 + 1 + len(LAYERS)
 
 
 def _graph(fn):
@@ -253,22 +264,14 @@ def run_ours(args, rank, world, local_rank):
     csa.lib()
     grp = DecodeGroup(csa, seed=9 + rank, device=device)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    g_step = _graph(grp.step)
     g_front, g_index, g_attn = _graph(grp.front), _graph(grp.index), _graph(grp.attention)
     st = torch.cuda.current_stream()
+    mk = lambda n: [torch.cuda.Event(enable_timing=True) for _ in range(n)]  # noqa: E731
 
-    def step(evs):
-        evs[0].record(st)
-        g_front.replay()
-        evs[1].record(st)
-        g_index.replay()
-        evs[2].record(st)
-        g_attn.replay()
-        evs[3].record(st)
-
-    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(4)]  # noqa: E731
     for _ in range(args.warmup):
         flush.zero_()
-        step(mk())
+        g_step.replay()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -282,22 +285,41 @@ def run_ours(args, rank, world, local_rank):
     t_wall = time.perf_counter()
     for _ in range(args.steps):
         flush.zero_()
-        evs = mk()
-        step(evs)
+        evs = mk(2)
+        evs[0].record(st)
+        g_step.replay()
+        evs[1].record(st)
         all_ev.append(evs)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     wall_s = time.perf_counter() - t_wall
     clocks = sampler.stop()
-    step_ms = [e[0].elapsed_time(e[3]) for e in all_ev]
-    index_ms = [e[1].elapsed_time(e[2]) for e in all_ev]
-    attn_ms = [e[2].elapsed_time(e[3]) for e in all_ev]
+    step_ms = [e[0].elapsed_time(e[1]) for e in all_ev]
     ms = float(np.mean(step_ms))
     t = torch.tensor([ms], dtype=torch.float64, device=device)
     if world > 1:
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     ms_max = float(t.item())
+
+    # breakdown (not the headline): the same step as three graphs with events between them
+    seg_ev = []
+    for it in range(args.warmup + args.steps):
+        flush.zero_()
+        evs = mk(4)
+        evs[0].record(st)
+        g_front.replay()
+        evs[1].record(st)
+        g_index.replay()
+        evs[2].record(st)
+        g_attn.replay()
+        evs[3].record(st)
+        if it >= args.warmup:
+            seg_ev.append(evs)
+    torch.cuda.synchronize()
+    index_ms = [e[1].elapsed_time(e[2]) for e in seg_ev]
+    attn_ms = [e[2].elapsed_time(e[3]) for e in seg_ev]
+    front_ms = [e[0].elapsed_time(e[1]) for e in seg_ev]
 
     # end to end through the public API with host buffers: pinned inputs copied in,
     # the step, the four outputs copied back, every step
@@ -318,9 +340,7 @@ def run_ours(args, rank, world, local_rank):
         grp.iq_bf.copy_(h_iq, non_blocking=True)
         for q, hq in zip(grp.q, h_q):
             q.copy_(hq, non_blocking=True)
-        g_front.replay()
-        g_index.replay()
-        g_attn.replay()
+        g_step.replay()
         for o, ho in zip(grp.out, h_out):
             ho.copy_(o, non_blocking=True)
         e1.record(st)
@@ -347,12 +367,13 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None, "dtype": "e2m1+bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "B_per_gpu": B, "ctx_entries": N_CTX, "topk": TOPK, "swa": T_SWA,
                    "l2": "flushed between timed steps (256 MiB write outside the step events)",
-                   "graphs": "3 CUDA graphs per step (front, index, attention)"},
+                   "graphs": "one CUDA graph per step (front with two branches, index, 4 attention layers)"},
         "index_attn_gbs": STEP_BYTES / (ms_max / 1000.0) / 1e9,
         "index_attn_frac_of_hbm": STEP_BYTES / (ms_max / 1000.0) / 1e9 / peak,
         "step_algorithmic_bytes": STEP_BYTES,
-        "segments_ms": {"front": float(np.mean([e[0].elapsed_time(e[1]) for e in all_ev])),
-                        "index_topk": float(np.mean(index_ms)), "attention_x4": float(np.mean(attn_ms))},
+        "segments_ms": {"front": float(np.mean(front_ms)), "index_topk": float(np.mean(index_ms)),
+                        "attention_x4": float(np.mean(attn_ms)),
+                        "how": "the step re-run as three graphs with events between them (diagnostic)"},
         "roofline": {"kernel": "csa2_index_topk (index_cluster_kernel)", "bound": "hbm", "achieved": achieved,
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",

@@ -138,6 +138,17 @@ CSA2_API csa2_status csa2_index_k_proj(const void* x, int64_t rows, const float*
                                        uint8_t* k_scales, const int64_t* dst_rows, int64_t out_rows, void* stream);
 
 /*
+ * Append of new tokens: csa2_quant_nvfp4 of each latent row (ch = 512) into
+ * the main-KV codes/scales and csa2_index_k_proj of the same row into the
+ * indexer-K codes/scales, in one launch (same bytes as the two calls).
+ * Arguments as for those two calls; x, W 16-byte aligned; lat_codes and
+ * k_codes 8-byte aligned; both outputs use the same row mapping.
+ */
+CSA2_API csa2_status csa2_append_tokens(const void* x, int64_t rows, const float* W, uint8_t* lat_codes,
+                                        uint8_t* lat_scales, uint8_t* k_codes, uint8_t* k_scales,
+                                        const int64_t* dst_rows, int64_t out_rows, void* stream);
+
+/*
  * Step 2 -- FP4 index scoring + Top-K ([Blog] "CSA2" section: a lightweight
  * indexer scores the causally visible compressed entries and keeps the Top-K,
  * K = 512; [Blog] FP4 section: FP4 indexer Q/K).

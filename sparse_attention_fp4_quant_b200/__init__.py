@@ -44,7 +44,8 @@ class csa2_layer_args(ctypes.Structure):
 
 
 _lib = None
-EXPORTS = ["csa2_status_str", "csa2_last_cuda_error", "csa2_quant_nvfp4", "csa2_index_k_proj", "csa2_index_topk",
+EXPORTS = ["csa2_status_str", "csa2_last_cuda_error", "csa2_quant_nvfp4", "csa2_index_k_proj", "csa2_append_tokens",
+           "csa2_index_topk",
            "csa2_pool_build", "csa2_pool_topk", "csa2_sparse_attn", "csa2_workspace_bytes", "csa2_layer_step",
            "csa2_index_topk_noalloc"]
 NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -65,6 +66,7 @@ def lib():
         "csa2_last_cuda_error": (ctypes.c_int, []),
         "csa2_quant_nvfp4": (ctypes.c_int, [P, i64, i32, P, P, P, i64, P]),
         "csa2_index_k_proj": (ctypes.c_int, [P, i64, P, P, P, P, i64, P]),
+        "csa2_append_tokens": (ctypes.c_int, [P, i64, P, P, P, P, P, P, i64, P]),
         "csa2_index_topk": (ctypes.c_int, [P, P, P, KVP, P, i32, i32, i32, P, P, P, sz, P]),
         "csa2_pool_build": (ctypes.c_int, [P, KVP, P, i32, i32, i32, P, P, sz, P]),
         "csa2_pool_topk": (ctypes.c_int, [P, P, P, KVP, P, i32, P, i32, i32, i32, P, P, sz, P]),
@@ -190,6 +192,33 @@ def csa2_index_k_proj(x, W, k_codes=None, k_scales=None, dst_rows=None):
     _check(lib().csa2_index_k_proj(_ptr(x), rows, _ptr(W), _ptr(k_codes), _ptr(k_scales), _ptr(dst_rows),
                                    k_codes.numel() // (ID // 2), _stream()))
     return k_codes, k_scales
+
+
+def csa2_append_tokens(x, W, kv_or_outs, dst_rows=None):
+    """Quantise new latent rows x (bf16 [rows, 512]) into the main KV and project + quantise their
+    indexer K, in one launch.  kv_or_outs: a KV (rows land at dst_rows of its [B*cap] cache) or a
+    tuple (lat_codes, lat_scales, k_codes, k_scales)."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(W, torch.float32, "W")
+    _size(W, D * ID, "W")
+    rows = x.reshape(-1, D).shape[0]
+    if isinstance(kv_or_outs, KV):
+        kv = kv_or_outs
+        lc, ls, kc, ks = kv.lat, kv.lat_sc, kv.ik, kv.ik_sc
+        out_rows = kv.B * kv.cap
+    else:
+        lc, ls, kc, ks = kv_or_outs
+        out_rows = lc.numel() // (D // 2)
+    if dst_rows is not None:
+        _dev(dst_rows, torch.int64, "dst_rows")
+        _size(dst_rows, rows, "dst_rows")
+    elif out_rows < rows:
+        raise ValueError("outputs have fewer rows than x")
+    for t, n, per in ((lc, "lat_codes", D // 2), (ls, "lat_scales", D // 16), (kc, "k_codes", ID // 2),
+                      (ks, "k_scales", ID // 16)):
+        _size(_dev(t, torch.uint8, n), out_rows * per, n)
+    _check(lib().csa2_append_tokens(_ptr(x), rows, _ptr(W), _ptr(lc), _ptr(ls), _ptr(kc), _ptr(ks), _ptr(dst_rows),
+                                    out_rows, _stream()))
 
 
 def csa2_index_topk(q, q_sc, w, kv, q_pos, k, idx_out=None, blockmax=False, ws=None):

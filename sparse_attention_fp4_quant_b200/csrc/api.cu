@@ -84,6 +84,19 @@ csa2_status csa2_index_k_proj(const void* x, int64_t rows, const float* W, uint8
     return cuda_status(launch_index_k_proj(x, rows, W, k_codes, k_scales, dst_rows, out_rows, (cudaStream_t)stream));
 }
 
+csa2_status csa2_append_tokens(const void* x, int64_t rows, const float* W, uint8_t* lat_codes, uint8_t* lat_scales,
+                               uint8_t* k_codes, uint8_t* k_scales, const int64_t* dst_rows, int64_t out_rows,
+                               void* stream) {
+    if (rows < 0) return CSA2_ERR_INVALID_ARG;
+    if (rows == 0) return CSA2_OK;
+    if (!x || !W || !lat_codes || !lat_scales || !k_codes || !k_scales || !aligned16(x) || !aligned16(W) ||
+        ((uintptr_t)lat_codes & 7u) || ((uintptr_t)k_codes & 7u))
+        return CSA2_ERR_INVALID_ARG;
+    if (out_rows < 0 || (!dst_rows && out_rows < rows)) return CSA2_ERR_INVALID_ARG;
+    return cuda_status(launch_append(x, rows, W, lat_codes, lat_scales, k_codes, k_scales, dst_rows, out_rows,
+                                     (cudaStream_t)stream));
+}
+
 size_t csa2_workspace_bytes(csa2_op op, int32_t B, int32_t Q, int64_t cap, int32_t k, int32_t P) {
     if (B < 1 || Q < 1) return 0;
     switch (op) {
@@ -206,11 +219,8 @@ csa2_status csa2_layer_step(const csa2_layer_args* a, void* stream) {
     if (a->mode == CSA2_MODE_FULL) {
         if (a->n_new > 0) {
             if (!a->new_latent || !a->new_rows || !a->k_proj) return CSA2_ERR_INVALID_ARG;
-            st = csa2_quant_nvfp4(a->new_latent, a->n_new, CSA2_D, kv->lat, kv->lat_sc, a->new_rows,
-                                 (int64_t)kv->cap * a->B, stream);
-            if (st != CSA2_OK) return st;
-            st = csa2_index_k_proj(a->new_latent, a->n_new, a->k_proj, kv->ik, kv->ik_sc, a->new_rows,
-                                  (int64_t)kv->cap * a->B, stream);
+            st = csa2_append_tokens(a->new_latent, a->n_new, a->k_proj, kv->lat, kv->lat_sc, kv->ik, kv->ik_sc,
+                                    a->new_rows, (int64_t)kv->cap * a->B, stream);
             if (st != CSA2_OK) return st;
         }
         bool build = a->pool != nullptr;

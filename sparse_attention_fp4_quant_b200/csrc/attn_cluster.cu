@@ -6,14 +6,15 @@
 // all at once, so a CTA waits on global memory once instead of once per tile.
 // The rows are dequantised to bf16 in swizzled shared memory (K = V); with the
 // 16 heads as the M dimension, S = Q K^T runs on warp-level tensor-core MMAs
-// (8 keys per warp and tile), then the CTA's own softmax (max and sum over its
-// keys), then O_r = P V (32 dims per warp; P as a rounded bf16 term plus its
-// bf16 remainder).  The partial results meet in distributed shared memory:
-// each CTA publishes O_r (fp32) and its per-head (max, sum); CTA r then forms
-// dims [r * 512 / C, (r + 1) * 512 / C) of the output as
-//   sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c,   M = max_c m_c,
-// and writes them as bf16.  No partials go to global memory and no CTA waits
-// for a ticket.
+// (each warp a quarter of the channels of a fifth of the keys), then the CTA's
+// own softmax (one warp per head: max and sum over its keys), then O_r = P V
+// (32 dims per warp; P as a rounded bf16 term plus its bf16 remainder).  The partial results meet in distributed shared memory:
+// each CTA stores, into CTA c's (by then idle) key buffer, its slice
+// [c * 512 / C, (c + 1) * 512 / C) of O_r (fp32) and its per-head (max, sum);
+// CTA c then forms its slice of the output as
+//   sum_r 2^(m_r - M) O_r / sum_r 2^(m_r - M) l_r,   M = max_r m_r,
+// from its own shared memory and writes it as bf16.  No partials go to global
+// memory and no CTA waits for a ticket.
 #include "attn_common.cuh"
 #include "cluster.cuh"
 
@@ -21,22 +22,23 @@ namespace csa2 {
 namespace {
 
 constexpr int kCT = 512;                      // threads per CTA (16 warps)
-constexpr int kCW = kCT / 32;
 constexpr int kMaxKeys = 160;                 // key slots per CTA
 constexpr int kPStride = kMaxKeys * 2 + 16;   // bytes per head row of P (conflict-free ldmatrix)
-constexpr int kOStride = kD + 4;              // floats per head row of the partial O (conflict-free stores)
-static_assert(kMaxKeys % 16 == 0, "keys per CTA");
-static_assert(kH * kOStride * 4 <= kMaxKeys * kRowB, "partial O fits the key buffer");
+constexpr int kQG = 4;                        // key-tile groups of the S warps (x 4 channel groups)
+constexpr int kQT = kMaxKeys / 8 / kQG;       // key tiles per S warp
+constexpr int kSStride = kMaxKeys + 4;        // floats per head row of a partial S
+static_assert(kMaxKeys % 32 == 0 && kMaxKeys % (8 * kQG) == 0, "keys per CTA");
+static_assert(kCT / 32 == kH, "one warp per head in the softmax");
+static_assert(2 * kH * kSStride * 4 <= kH * kRowB + 2 * kH * kPStride, "partial S fit the Q and P buffers");
+static_assert((16 * kH * (kD / 16 + 4) + 16 * kH * 2) * 4 <= kMaxKeys * kRowB, "received slices fit the key buffer");
 
 struct ClAttnSmem {
-    uint8_t K[kMaxKeys * kRowB];   // bf16 keys (= values), swizzled; afterwards the fp32 partial O [16][kOStride]
-    uint8_t Qs[kH * kRowB];        // bf16 query, swizzled
+    uint8_t K[kMaxKeys * kRowB];   // bf16 keys (= values), swizzled; afterwards the received output slices
+    uint8_t Qs[kH * kRowB];        // bf16 query, swizzled; then (with P) the two partial S arrays
     uint8_t P[kH * kPStride];      // bf16 P (rounded), [head][key]
     uint8_t Pl[kH * kPStride];     // bf16 remainder P - rounded(P)
     float kf[kMaxKeys];            // per-key factor (1 for FP4 rows, token scale for SWA)
     int kvalid[kMaxKeys];
-    float red[kCW][kH];
-    float m_loc[kH];
     alignas(16) float ml[kH][2];   // this CTA's (max, sum) per head (log2 units), read by the cluster
     float cw[16][kH];              // combine weight of rank c for head h (for this CTA's output slice)
 };
@@ -67,29 +69,44 @@ __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
     const uint32_t sP = (uint32_t)__cvta_generic_to_shared(sm.P);
     const uint32_t sPl = (uint32_t)__cvta_generic_to_shared(sm.Pl);
 
-    // ---- gather: row quarter u = r + n16 * qq (consecutive lanes, consecutive rows)
+    // ---- gather: row quarter u = r + n16 * qq (consecutive lanes, consecutive rows).
+    // Every load of the thread is in flight before any is used: the main-row
+    // ids first, then the rows, then the query.
     {
         constexpr int kPer = (kMaxKeys * 4 + kCT - 1) / kCT;   // 2
         RowQuarter rq[kPer];
-        int rr[kPer], qs[kPer];
+        int rr[kPer], qs[kPer], slot[kPer];
+        int32_t e[kPer];
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
             const int u = tid + kCT * j;
-            rq[j].kind = 0;
             rr[j] = -1;
+            e[j] = -1;
+            slot[j] = p.slots_total;
             if (u < 4 * n16) {
                 rr[j] = u % n16;
                 qs[j] = u / n16;
-                const int slot = rr[j] < nk ? s0 + rr[j] : p.slots_total;   // past nk: dead
-                fetch_quarter(p, bq, b, slot, qs[j], i_pos, lo, pos0, nmain, rq[j]);
+                if (rr[j] < nk) slot[j] = s0 + rr[j];   // past nk: dead
+                if (slot[j] < p.k) e[j] = (int32_t)ld_nc_u32(p.idx + (int64_t)bq * p.k + slot[j]);
             }
         }
-        const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (int64_t)bq * kH * kD);
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            rq[j].kind = 0;
+            if (rr[j] >= 0) {
+                int64_t row = 0;
+                const int kind = slot_row(p, b, slot[j], e[j], i_pos, lo, pos0, nmain, row);
+                issue_quarter(p, kind, row, qs[j], rq[j]);
+            }
+        }
+        const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q + (int64_t)bq * kH * kD);
+        uint4 qv[(kH * kD / 8) / kCT];
+#pragma unroll
+        for (int it = 0; it < (kH * kD / 8) / kCT; ++it) qv[it] = ld_nc_v4(qsrc + 16 * (it * kCT + tid));
 #pragma unroll
         for (int it = 0; it < (kH * kD / 8) / kCT; ++it) {
             const int c = it * kCT + tid;   // 16-byte chunk id
-            const int row = c >> 6, ch = c & 63;
-            *reinterpret_cast<uint4*>(sm.Qs + swz(row, ch)) = __ldg(qsrc + c);
+            *reinterpret_cast<uint4*>(sm.Qs + swz(c >> 6, c & 63)) = qv[it];
         }
 #pragma unroll
         for (int j = 0; j < kPer; ++j)
@@ -97,97 +114,99 @@ __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
     }
     __syncthreads();
 
-    // ---- S = Q K^T: warp w takes key tiles w and w + 16 (8 keys each)
+    // ---- S = Q K^T.  Warp (kg, ng) = (warp % 4, warp / 4) takes channels
+    // [128 kg, 128 kg + 128) (its Q fragments stay in registers) of key tiles
+    // ng, ng + 4, ..., ng + 16 (8 keys each); the four channel partials are
+    // added in the fixed order (p0 + p2) + (p1 + p3) in shared memory.
     const int nt = n16 >> 3;
-    const bool has0 = warp < nt, has1 = warp + kCW < nt;
-    float s4[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    if (has0) {
-        const int key = 8 * warp + (lane & 7);
-#pragma unroll 4
-        for (int ks = 0; ks < kD / 16; ++ks) {
-            uint32_t a0, a1, a2, a3, b0, b1;
-            ldsm_x4(sQ + swz(lane & 15, 2 * ks + (lane >> 4)), a0, a1, a2, a3);
-            ldsm_x2(sK + swz(key, 2 * ks + ((lane >> 3) & 1)), b0, b1);
-            mma_bf16(s4[0], a0, a1, a2, a3, b0, b1);
-            if (has1) {
-                ldsm_x2(sK + swz(key + 8 * kCW, 2 * ks + ((lane >> 3) & 1)), b0, b1);
-                mma_bf16(s4[1], a0, a1, a2, a3, b0, b1);
+    const int kg = warp & 3, ng = warp >> 2;
+    float s4[kQT][4];
+    {
+        uint32_t qa[8][4];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            ldsm_x4(sQ + swz(lane & 15, 2 * (8 * kg + j) + (lane >> 4)), qa[j][0], qa[j][1], qa[j][2], qa[j][3]);
+#pragma unroll
+        for (int i = 0; i < kQT; ++i) {
+            s4[i][0] = s4[i][1] = s4[i][2] = s4[i][3] = 0.0f;
+            const int tile = ng + kQG * i;
+            if (tile < nt) {   // warp-uniform
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint32_t b0, b1;
+                    ldsm_x2(sK + swz(8 * tile + (lane & 7), 2 * (8 * kg + j) + ((lane >> 3) & 1)), b0, b1);
+                    mma_bf16(s4[i], qa[j][0], qa[j][1], qa[j][2], qa[j][3], b0, b1);
+                }
             }
         }
     }
-    // logits (log2 units), masked keys -> -inf; z[t][0..3] = (g, key0), (g, key0+1), (g+8, key0), (g+8, key0+1)
-    float z[2][4], f[2][2];
-    float mx0 = -INFINITY, mx1 = -INFINITY;
+    __syncthreads();   // every warp holds its Q fragments: the Q and P buffers take the partial sums
+    float* S0 = reinterpret_cast<float*>(sm.Qs);   // [16][kSStride], then S1 right after
+    float* S1 = S0 + kH * kSStride;
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
-        const bool has = t == 0 ? has0 : has1;
-        const int key0 = 8 * (warp + kCW * t) + 2 * qd;
-        f[t][0] = has ? sm.kf[key0] : 0.0f;
-        f[t][1] = has ? sm.kf[key0 + 1] : 0.0f;
-        const bool v0 = has && sm.kvalid[key0] != 0, v1 = has && sm.kvalid[key0 + 1] != 0;
-        z[t][0] = v0 ? s4[t][0] * f[t][0] * scale_log2 : -INFINITY;
-        z[t][1] = v1 ? s4[t][1] * f[t][1] * scale_log2 : -INFINITY;
-        z[t][2] = v0 ? s4[t][2] * f[t][0] * scale_log2 : -INFINITY;
-        z[t][3] = v1 ? s4[t][3] * f[t][1] * scale_log2 : -INFINITY;
-        mx0 = fmaxf(mx0, fmaxf(z[t][0], z[t][1]));
-        mx1 = fmaxf(mx1, fmaxf(z[t][2], z[t][3]));
-    }
+    for (int pass = 0; pass < 2; ++pass) {
+        if ((kg >> 1) == pass) {
+            float* S = (kg & 1) ? S1 : S0;
 #pragma unroll
-    for (int o2 = 1; o2 < 4; o2 <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, o2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xFFFFFFFFu, mx1, o2));
+            for (int i = 0; i < kQT; ++i) {
+                const int tile = ng + kQG * i;
+                if (tile >= nt) continue;
+                const int key0 = 8 * tile + 2 * qd;
+                float2* r0 = reinterpret_cast<float2*>(S + g * kSStride + key0);
+                float2* r1 = reinterpret_cast<float2*>(S + (g + 8) * kSStride + key0);
+                if (pass == 0) {
+                    *r0 = make_float2(s4[i][0], s4[i][1]);
+                    *r1 = make_float2(s4[i][2], s4[i][3]);
+                } else {
+                    const float2 x0 = *r0, x1 = *r1;
+                    *r0 = make_float2(x0.x + s4[i][0], x0.y + s4[i][1]);
+                    *r1 = make_float2(x1.x + s4[i][2], x1.y + s4[i][3]);
+                }
+            }
+        }
+        __syncthreads();
     }
-    if (qd == 0) {
-        sm.red[warp][g] = mx0;
-        sm.red[warp][g + 8] = mx1;
-    }
-    __syncthreads();
-    if (tid < kH) {
-        float m = sm.red[0][tid];
-#pragma unroll
-        for (int w = 1; w < kCW; ++w) m = fmaxf(m, sm.red[w][tid]);
-        sm.m_loc[tid] = m;
-    }
-    __syncthreads();
+    // ---- softmax over the CTA's keys: warp h owns head h (keys lane + 32 j)
     {
-        const float m0 = sm.m_loc[g], m1 = sm.m_loc[g + 8];
-        const float mu0 = (m0 == -INFINITY) ? 0.0f : m0, mu1 = (m1 == -INFINITY) ? 0.0f : m1;
-        float sum0 = 0.0f, sum1 = 0.0f;
+        const int h = warp;
+        float z[kMaxKeys / 32], fk[kMaxKeys / 32];
+        float m = -INFINITY;
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            const bool has = t == 0 ? has0 : has1;
-            if (!has) continue;
-            const int key0 = 8 * (warp + kCW * t) + 2 * qd;
-            const float p00 = exp2f(z[t][0] - mu0), p01 = exp2f(z[t][1] - mu0);
-            const float p10 = exp2f(z[t][2] - mu1), p11 = exp2f(z[t][3] - mu1);
-            sum0 += p00 + p01;
-            sum1 += p10 + p11;
-            const float u00 = p00 * f[t][0], u01 = p01 * f[t][1], u10 = p10 * f[t][0], u11 = p11 * f[t][1];
-            const __nv_bfloat162 h0 = __floats2bfloat162_rn(u00, u01), h1 = __floats2bfloat162_rn(u10, u11);
-            const uint32_t off0 = g * kPStride + key0 * 2, off1 = (g + 8) * kPStride + key0 * 2;
-            *reinterpret_cast<__nv_bfloat162*>(sm.P + off0) = h0;
-            *reinterpret_cast<__nv_bfloat162*>(sm.P + off1) = h1;
-            *reinterpret_cast<uint32_t*>(sm.Pl + off0) = pack_bf16(u00 - __low2float(h0), u01 - __high2float(h0));
-            *reinterpret_cast<uint32_t*>(sm.Pl + off1) = pack_bf16(u10 - __low2float(h1), u11 - __high2float(h1));
+        for (int j = 0; j < kMaxKeys / 32; ++j) {
+            const int t = lane + 32 * j;
+            const bool v = t < n16 && sm.kvalid[t] != 0;
+            fk[j] = t < n16 ? sm.kf[t] : 0.0f;
+            z[j] = v ? (S0[h * kSStride + t] + S1[h * kSStride + t]) * fk[j] * scale_log2 : -INFINITY;
+            m = fmaxf(m, z[j]);
         }
 #pragma unroll
-        for (int o2 = 1; o2 < 4; o2 <<= 1) {
-            sum0 += __shfl_xor_sync(0xFFFFFFFFu, sum0, o2);
-            sum1 += __shfl_xor_sync(0xFFFFFFFFu, sum1, o2);
-        }
-        if (qd == 0) {   // red's maxima were consumed before the last barrier
-            sm.red[warp][g] = sum0;
-            sm.red[warp][g + 8] = sum1;
-        }
-    }
-    __syncthreads();
-    if (tid < kH) {
+        for (int o2 = 16; o2 > 0; o2 >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o2));
+        const float mu = (m == -INFINITY) ? 0.0f : m;
         float l = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kCW; ++w) l += sm.red[w][tid];
-        sm.ml[tid][0] = sm.m_loc[tid];
-        sm.ml[tid][1] = l;
+        for (int j = 0; j < kMaxKeys / 32; ++j) {
+            z[j] = exp2f(z[j] - mu);
+            l += z[j];
+        }
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, o2);
+        __syncthreads();   // every partial sum is read: P may overwrite them
+#pragma unroll
+        for (int j = 0; j < kMaxKeys / 32; ++j) {
+            const int t = lane + 32 * j;
+            if (t < n16) {
+                const float u = z[j] * fk[j];
+                const __nv_bfloat16 hi = __float2bfloat16_rn(u);
+                *reinterpret_cast<__nv_bfloat16*>(sm.P + h * kPStride + 2 * t) = hi;
+                *reinterpret_cast<__nv_bfloat16*>(sm.Pl + h * kPStride + 2 * t) = __float2bfloat16_rn(u - __bfloat162float(hi));
+            }
+        }
+        if (lane == 0) {
+            sm.ml[h][0] = m;
+            sm.ml[h][1] = l;
+        }
     }
+    __syncthreads();
 
     // ---- O_r[:, 32 warp .. +31] = P V over the CTA's keys
     float o[4][4];
@@ -212,33 +231,44 @@ __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
             mma_bf16(o[2 * np + 1], l0, l1, l2, l3, b2, b3);
         }
     }
-    __syncthreads();   // every warp is done with K: its buffer now takes the partial O
-    float* Of = reinterpret_cast<float*>(sm.K);
-#pragma unroll
-    for (int n = 0; n < 4; ++n) {
-        const int d = 32 * warp + 8 * n + 2 * qd;
-        *reinterpret_cast<float2*>(Of + g * kOStride + d) = make_float2(o[n][0], o[n][1]);
-        *reinterpret_cast<float2*>(Of + (g + 8) * kOStride + d) = make_float2(o[n][2], o[n][3]);
-    }
-    cl::sync();   // every CTA's partial O and (max, sum) are published
 
-    // ---- combine: this CTA's slice of the output dims
+    // ---- combine: every CTA pushes the slice of O_r and its (max, sum) that CTA c
+    // owns (dims [c DS, (c + 1) DS)) into c's key buffer, which is free once every
+    // CTA has finished P V
     const int DS = kD / (int)C;
-    if (tid < kH) {
-        float mc[16], lc[16];
-        float M = -INFINITY;
-        for (uint32_t c = 0; c < C; ++c) {
-            const uint2 x = cl::ld_v2(cl::map_rank((uint32_t)__cvta_generic_to_shared(&sm.ml[tid][0]), c));
-            mc[c] = __uint_as_float(x.x);
-            lc[c] = __uint_as_float(x.y);
-            M = fmaxf(M, mc[c]);
+    const int rstride = DS + 4;   // floats per head row of a received slice
+    float* Rf = reinterpret_cast<float*>(sm.K);                 // [C][16][rstride]
+    float* MLf = Rf + (int)C * kH * rstride;                    // [C][16][2]
+    cl::sync();   // #1: every CTA is done with its key buffer
+    {
+        const uint32_t sR = (uint32_t)__cvta_generic_to_shared(Rf);
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            const int d = 32 * warp + 8 * n + 2 * qd;
+            const uint32_t owner = (uint32_t)(d / DS);
+            const int dd = d - (int)owner * DS;
+            const uint32_t a0 = sR + (uint32_t)(((int)rank * kH + g) * rstride + dd) * 4u;
+            const uint32_t a1 = sR + (uint32_t)(((int)rank * kH + g + 8) * rstride + dd) * 4u;
+            cl::st_v2f(cl::map_rank(a0, owner), o[n][0], o[n][1]);
+            cl::st_v2f(cl::map_rank(a1, owner), o[n][2], o[n][3]);
         }
+        if (tid < kH * (int)C) {
+            const uint32_t owner = (uint32_t)(tid / kH);
+            const int h = tid % kH;
+            const uint32_t a = (uint32_t)__cvta_generic_to_shared(MLf + ((int)rank * kH + h) * 2);
+            cl::st_v2f(cl::map_rank(a, owner), sm.ml[h][0], sm.ml[h][1]);
+        }
+    }
+    cl::sync();   // #2: every slice has arrived; nothing reads another CTA's memory after this
+    if (tid < kH) {
+        float M = -INFINITY;
+        for (uint32_t c = 0; c < C; ++c) M = fmaxf(M, MLf[((int)c * kH + tid) * 2]);
         const float Mu = (M == -INFINITY) ? 0.0f : M;
         float L = 0.0f;
         for (uint32_t c = 0; c < C; ++c) {
-            const float wgt = exp2f(mc[c] - Mu);
+            const float wgt = exp2f(MLf[((int)c * kH + tid) * 2] - Mu);
             sm.cw[c][tid] = wgt;
-            L += lc[c] * wgt;
+            L += MLf[((int)c * kH + tid) * 2 + 1] * wgt;
         }
         const float inv = L > 0.0f ? 1.0f / L : 0.0f;
         for (uint32_t c = 0; c < C; ++c) sm.cw[c][tid] *= inv;
@@ -247,25 +277,23 @@ __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
     __syncthreads();
     {
         const int per_head = DS / 4;   // float4 per head in the slice
-        const uint32_t sOf = (uint32_t)__cvta_generic_to_shared(Of);
         uint16_t* out = p.out + (int64_t)bq * kH * kD;
         for (int e4 = tid; e4 < kH * per_head; e4 += kCT) {
             const int h = e4 / per_head;
-            const int d = (int)rank * DS + 4 * (e4 - h * per_head);
-            const uint32_t la = sOf + (uint32_t)(h * kOStride + d) * 4u;
+            const int dd = 4 * (e4 - h * per_head);
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
             for (uint32_t c = 0; c < C; ++c) {
-                const uint4 x = cl::ld_v4(cl::map_rank(la, c));
+                const float4 x = *reinterpret_cast<const float4*>(Rf + ((int)c * kH + h) * rstride + dd);
                 const float wgt = sm.cw[c][h];
-                acc.x += __uint_as_float(x.x) * wgt;
-                acc.y += __uint_as_float(x.y) * wgt;
-                acc.z += __uint_as_float(x.z) * wgt;
-                acc.w += __uint_as_float(x.w) * wgt;
+                acc.x += x.x * wgt;
+                acc.y += x.y * wgt;
+                acc.z += x.z * wgt;
+                acc.w += x.w * wgt;
             }
-            *reinterpret_cast<uint2*>(out + h * kD + d) = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
+            *reinterpret_cast<uint2*>(out + h * kD + (int)rank * DS + dd) =
+                make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
         }
     }
-    cl::sync();   // no CTA leaves while the cluster may read it
 }
 
 int g_max_active[17];

@@ -117,19 +117,79 @@ __device__ __forceinline__ void fetch_quarter(const AttnParams& p, int bq, int b
     }
 }
 
+// Loads of read-only data as volatile asm: they issue in program order, so a
+// thread can put all of its loads in flight before it consumes any of them.
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint2 ld_nc_v2(const void* p) {
+    uint2 v;
+    asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ld_nc_u32(const void* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+// Which row a key slot reads (the main row id e of slot < k is given):
+// 1 = FP4 main row, 2 = FP8 window row, 0 = dead; `row` = its row in the cache.
+__device__ __forceinline__ int slot_row(const AttnParams& p, int b, int slot, int32_t e, int64_t i_pos, int64_t lo,
+                                        int64_t pos0, int64_t nmain, int64_t& row) {
+    if (slot < p.k) {
+        if (e >= 0 && e < nmain) {
+            row = (int64_t)b * p.cap + e;
+            return 1;
+        }
+    } else if (slot < p.slots_total) {
+        const int64_t tau = i_pos - p.window + 1 + (slot - p.k);
+        const int64_t rr = tau - pos0;
+        if (tau >= lo && tau <= i_pos && rr >= 0 && rr < p.T) {
+            row = (int64_t)b * p.T + rr;
+            return 2;
+        }
+    }
+    return 0;
+}
+
+// Issue the loads of quarter qq of a row chosen by slot_row.
+__device__ __forceinline__ void issue_quarter(const AttnParams& p, int kind, int64_t row, int qq, RowQuarter& q) {
+    q.kind = kind;
+    if (kind == 1) {
+        const uint8_t* cs = p.lat + row * (kD / 2) + 64 * qq;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) q.raw[v] = ld_nc_v4(cs + 16 * v);
+        q.sc = ld_nc_v2(p.lat_sc + row * (kD / 16) + 8 * qq);
+    } else if (kind == 2) {
+        q.fac = __uint_as_float(ld_nc_u32(p.swa_sc + row));
+        const uint8_t* cs = p.swa + row * kD + 128 * qq;
+#pragma unroll
+        for (int v = 0; v < 8; ++v) q.raw[v] = ld_nc_v4(cs + 16 * v);
+    }
+}
+
 __device__ __forceinline__ void store_quarter(uint8_t* K, float* kf, int* kvalid, int r, int qq, const RowQuarter& q) {
     if (q.kind == 1) {
-        const uint32_t scw[2] = {q.sc.x, q.sc.y};
+        uint32_t s2[8];   // the 8 block scales as bf16 pairs (exact: E4M3 fits bf16)
+        {
+            float f[8];
+            e4m3x4_to_f32(q.sc.x, f);
+            e4m3x4_to_f32(q.sc.y, f + 4);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) s2[i] = pack_bf16(f[i], f[i]);
+        }
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
             const uint32_t ws[4] = {q.raw[v].x, q.raw[v].y, q.raw[v].z, q.raw[v].w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const int word = 4 * v + j;             // 8 dims per word
-                const int sb = word >> 1;               // one scale per 16 dims
-                const float s = e4m3_to_f32((scw[sb >> 2] >> (8 * (sb & 3))) & 0xFFu);
-                const uint32_t s2 = pack_bf16(s, s);   // exact (E4M3 fits bf16)
-                *reinterpret_cast<uint4*>(K + swz(r, 16 * qq + word)) = fp4x8_to_bf16(ws[j], s2);
+                const int word = 4 * v + j;   // 8 dims per word, one scale per 16 dims
+                *reinterpret_cast<uint4*>(K + swz(r, 16 * qq + word)) = fp4x8_to_bf16(ws[j], s2[word >> 1]);
             }
         }
     } else if (q.kind == 2) {

@@ -46,5 +46,9 @@ __device__ __forceinline__ uint2 ld_v2(uint32_t addr) {
     return v;
 }
 
+__device__ __forceinline__ void st_v2f(uint32_t addr, float a, float b) {
+    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
+}
+
 }  // namespace cl
 }  // namespace csa2

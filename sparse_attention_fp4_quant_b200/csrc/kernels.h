@@ -53,6 +53,9 @@ cudaError_t launch_quant(const void* x, int64_t rows, int ch, uint8_t* codes, ui
                          const int64_t* dst_rows, int64_t out_rows, cudaStream_t st);
 cudaError_t launch_index_k_proj(const void* x, int64_t rows, const float* W, uint8_t* k_codes, uint8_t* k_scales,
                                 const int64_t* dst_rows, int64_t out_rows, cudaStream_t st);
+cudaError_t launch_append(const void* x, int64_t rows, const float* W, uint8_t* lat_codes, uint8_t* lat_scales,
+                          uint8_t* k_codes, uint8_t* k_scales, const int64_t* dst_rows, int64_t out_rows,
+                          cudaStream_t st);
 
 // Sparse attention.
 struct AttnParams {

@@ -196,6 +196,113 @@ __global__ void __launch_bounds__(256) index_k_proj_rows_kernel(const uint16_t* 
     }
 }
 
+// Append of a few new rows (a decode step): one launch quantises each latent
+// row into the main KV and projects + quantises its indexer K.  A projection
+// CTA takes 32 rows and one 16-output block of W (32 KB, staged with cp.async
+// next to the 32 bf16 rows): thread (row, output) runs the 512-long FMA chain
+// in ascending channel order, and since the 16 outputs of a row are exactly
+// one NVFP4 block, the CTA quantises its block alone.  The remaining CTAs
+// quantise the latent rows, one thread per 16 channels.
+constexpr int kAppRows = 32;
+constexpr int kAppThreads = kAppRows * 16;
+constexpr int kAppXStride = kD + 8;   // bf16 per staged row (16 bytes of padding: no bank conflicts)
+constexpr int kAppSmem = kD * 16 * 4 + kAppRows * kAppXStride * 2 + kAppRows * 16 * 4;
+
+__global__ void __launch_bounds__(kAppThreads) append_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                             const float* __restrict__ W, uint8_t* __restrict__ lc,
+                                                             uint8_t* __restrict__ ls, uint8_t* __restrict__ kc,
+                                                             uint8_t* __restrict__ ks,
+                                                             const int64_t* __restrict__ dst_rows, int64_t out_rows,
+                                                             int nproj) {
+    const int tid = threadIdx.x;
+    if ((int)blockIdx.x >= nproj) {
+        // latent rows -> NVFP4, one thread per 16 channels
+        const int64_t t = (int64_t)(blockIdx.x - nproj) * kAppThreads + tid;
+        if (t >= rows * (kD / 16)) return;
+        const int64_t r = t / (kD / 16);
+        const int g = (int)(t - r * (kD / 16));
+        const uint4* src = reinterpret_cast<const uint4*>(x + r * kD + 16 * g);
+        const uint4 a = __ldg(src), b = __ldg(src + 1);
+        const uint32_t u[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            v[2 * j] = __uint_as_float(u[j] << 16);
+            v[2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
+        }
+        uint32_t sc, lo, hi;
+        quant16(v, sc, lo, hi);
+        const int64_t orow = dst_rows ? __ldg(dst_rows + r) : r;
+        if (orow < 0 || orow >= out_rows) return;
+        *reinterpret_cast<uint2*>(lc + orow * (kD / 2) + 8 * g) = make_uint2(lo, hi);
+        ls[orow * (kD / 16) + g] = (uint8_t)sc;
+        return;
+    }
+    extern __shared__ __align__(16) uint8_t app_smem[];
+    float* Wb = reinterpret_cast<float*>(app_smem);                                 // [512][16]
+    uint16_t* xs = reinterpret_cast<uint16_t*>(app_smem + kD * 16 * 4);             // [32][kAppXStride]
+    float* outs = reinterpret_cast<float*>(app_smem + kD * 16 * 4 + kAppRows * kAppXStride * 2);   // [32][16]
+    const int cb = blockIdx.x & 3;                  // output block: outputs 16 cb .. 16 cb + 15
+    const int64_t r0 = (int64_t)(blockIdx.x >> 2) * kAppRows;
+    const uint32_t sW = (uint32_t)__cvta_generic_to_shared(Wb), sX = (uint32_t)__cvta_generic_to_shared(xs);
+    for (int i = tid; i < kD * 4; i += kAppThreads) {   // row c of the block: 4 x 16 B
+        const int c = i >> 2, q = i & 3;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sW + 16u * i), "l"(W + c * kID + 16 * cb + 4 * q)
+                     : "memory");
+    }
+    for (int i = tid; i < kAppRows * (kD / 8); i += kAppThreads) {   // 32 rows x 64 x 16 B
+        const int rr = i / (kD / 8), q = i % (kD / 8);
+        if (r0 + rr < rows)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sX + (uint32_t)(rr * kAppXStride * 2 + 16 * q)),
+                         "l"(x + (r0 + rr) * kD + 8 * q)
+                         : "memory");
+    }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
+    __syncthreads();
+    const int rr = tid >> 4, o = tid & 15;
+    const uint16_t* xr = xs + rr * kAppXStride;
+    float acc = 0.0f;
+#pragma unroll 16
+    for (int c = 0; c < kD; ++c) acc = __fmaf_rn(__uint_as_float((uint32_t)xr[c] << 16), Wb[c * 16 + o], acc);
+    outs[rr * 16 + o] = acc;
+    __syncthreads();
+    if (tid < kAppRows && r0 + tid < rows) {
+        float v[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) v[q] = outs[tid * 16 + q];
+        uint32_t sc, lo, hi;
+        quant16(v, sc, lo, hi);
+        const int64_t orow = dst_rows ? __ldg(dst_rows + r0 + tid) : r0 + tid;
+        if (orow >= 0 && orow < out_rows) {
+            *reinterpret_cast<uint2*>(kc + orow * 32 + 8 * cb) = make_uint2(lo, hi);
+            ks[orow * 4 + cb] = (uint8_t)sc;
+        }
+    }
+}
+
+cudaError_t launch_append(const void* x, int64_t rows, const float* W, uint8_t* lat_codes, uint8_t* lat_scales,
+                          uint8_t* k_codes, uint8_t* k_scales, const int64_t* dst_rows, int64_t out_rows,
+                          cudaStream_t st) {
+    if (rows == 0) return cudaSuccess;
+    if (rows > 2048) {
+        cudaError_t e = launch_quant(x, rows, kD, lat_codes, lat_scales, dst_rows, out_rows, st);
+        if (e != cudaSuccess) return e;
+        return launch_index_k_proj(x, rows, W, k_codes, k_scales, dst_rows, out_rows, st);
+    }
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAppSmem);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    const int nproj = (int)((rows + kAppRows - 1) / kAppRows) * 4;
+    const int nquant = (int)((rows * (kD / 16) + kAppThreads - 1) / kAppThreads);
+    append_kernel<<<nproj + nquant, kAppThreads, kAppSmem, st>>>(static_cast<const uint16_t*>(x), rows, W, lat_codes,
+                                                                   lat_scales, k_codes, k_scales, dst_rows, out_rows,
+                                                                   nproj);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_index_k_proj(const void* x, int64_t rows, const float* W, uint8_t* k_codes, uint8_t* k_scales,
                                 const int64_t* dst_rows, int64_t out_rows, cudaStream_t st) {
     if (rows == 0) return cudaSuccess;

@@ -86,6 +86,28 @@ def test_index_k_proj_bit_exact(csa):
     assert np.array_equal(np_(bc)[1::3][:1000], oc) and np.array_equal(np_(bs)[1::3][:1000], os_)
 
 
+@pytest.mark.parametrize("rows", [1, 32, 45, 2049])
+def test_append_tokens_bit_exact(csa, rows):
+    # one launch = csa2_quant_nvfp4 + csa2_index_k_proj of the same rows (2049: the two-launch path)
+    x = synth.latent(synth.seed_of("append", rows), rows, 100, "cuda")
+    W = synth.proj_w(rows).cuda()
+    lb = bits(x)
+    olc, ols = oracle.quant_nvfp4(lb)
+    okc, oks = oracle.index_k_proj(lb, np_(W))
+    out_rows = 3 * rows + 1
+    dst = torch.arange(rows, device="cuda", dtype=torch.int64) * 3 + 1
+    lc = torch.zeros((out_rows, 256), dtype=torch.uint8, device="cuda")
+    ls = torch.zeros((out_rows, 32), dtype=torch.uint8, device="cuda")
+    kc = torch.zeros((out_rows, 32), dtype=torch.uint8, device="cuda")
+    ks = torch.zeros((out_rows, 4), dtype=torch.uint8, device="cuda")
+    csa.csa2_append_tokens(x, W, (lc, ls, kc, ks), dst)
+    assert np.array_equal(np_(lc)[1::3][:rows], olc) and np.array_equal(np_(ls)[1::3][:rows], ols)
+    assert np.array_equal(np_(kc)[1::3][:rows], okc) and np.array_equal(np_(ks)[1::3][:rows], oks)
+    untouched = np.ones(out_rows, bool)
+    untouched[1::3][:rows] = False
+    assert not np_(lc)[untouched].any() and not np_(kc)[untouched].any()
+
+
 # ---------------------------------------------------------------- index / Top-K
 def _index_case(seed, B, Q, cap, n_entries, m, q_pos, k):
     grp = Group(seed, B, cap, n_entries, m)
