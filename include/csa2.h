@@ -172,7 +172,11 @@ CSA2_API csa2_status csa2_append_tokens(const void* x, int64_t rows, const float
  *   ws, ws_bytes  device workspace of at least csa2_workspace_bytes(CSA2_OP_INDEX_TOPK, ...)
  *                 bytes, zero-filled before its first use; every call leaves its
  *                 counters at zero again.  Calls that share a workspace must not
- *                 overlap on the GPU.
+ *                 overlap on the GPU.  The int32 at byte offset
+ *                 CSA2_STATUS_OFFSET(B, Q) of the workspace is a sticky error
+ *                 flag: a device-side wait that ran out of time (2 s) sets it to 1
+ *                 and the kernel winds down; the results of that call are not
+ *                 valid.  The caller may read it after the stream completes.
  */
 CSA2_API csa2_status csa2_index_topk(const uint8_t* q, const uint8_t* q_sc, const float* w, const csa2_kv* kv,
                             const int32_t* q_pos, int32_t B, int32_t Q, int32_t k, int32_t* idx_out,
@@ -244,6 +248,9 @@ typedef enum {
     CSA2_OP_LAYER = 4
 } csa2_op;
 CSA2_API size_t csa2_workspace_bytes(csa2_op op, int32_t B, int32_t Q, int64_t cap, int32_t k, int32_t P);
+
+/* Byte offset of the sticky device error flag in an index / pool workspace. */
+#define CSA2_STATUS_OFFSET(B, Q) ((((size_t)(B) * (size_t)(Q) * 4u) + 255u) & ~(size_t)255u)
 
 /*
  * Step 5 -- one CSA2 layer dispatched by its static mode ([Blog] "CSA2"

@@ -162,6 +162,17 @@ def _workspace(nbytes):
     return _ws[dev].get(nbytes)
 
 
+def status_offset(B, Q):
+    """Byte offset of the sticky device error flag in an index / pool workspace (CSA2_STATUS_OFFSET)."""
+    return (B * Q * 4 + 255) & ~255
+
+
+def device_error_flag(ws, B, Q):
+    """The workspace's sticky device error flag (1 after a device-side wait ran out of time)."""
+    off = status_offset(B, Q)
+    return int(ws[off:off + 4].view(torch.int32).item())
+
+
 def csa2_workspace_bytes(op, B, Q, cap, k, P=0):
     return int(lib().csa2_workspace_bytes(op, B, Q, cap, k, P))
 

@@ -154,11 +154,12 @@ __device__ __forceinline__ void find_bin(ClSmem& s, const uint32_t* hist, uint32
     __syncthreads();
 }
 
-// Visit every stored key of this CTA: warps 2-9, TMEM lane quarter warp % 4,
-// tile columns [128 h, 128 h + 128) with h = (warp - 2) / 4.  f(key, entry)
-// gets the CTA-local entry 128 c + 4 lane + quarter of column c.
+// Visit every stored key of this CTA, 32 tile columns at a time: warps 2-9,
+// TMEM lane quarter q = warp % 4, columns [128 h, 128 h + 128) with
+// h = (warp - 2) / 4.  f(v, c0, q) gets the keys of columns c0 .. c0 + 31 of
+// this lane; column c of lane l holds CTA-local entry 128 c + 4 l + q.
 template <class F>
-__device__ __forceinline__ void sweep_keys(uint32_t tbase, int warp, int lane, int ntiles, F&& f) {
+__device__ __forceinline__ void sweep_cols(uint32_t tbase, int warp, int ntiles, F&& f) {
     if (warp < 2) return;
     const int quarter = warp & 3, half = (warp - 2) >> 2;
     const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
@@ -166,9 +167,7 @@ __device__ __forceinline__ void sweep_keys(uint32_t tbase, int warp, int lane, i
         uint32_t v[32];
         tc::tmem_ld_32x32b_x32(tbase + lanes + kColKeys + (uint32_t)c0, v);
         tc::tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-            if (c0 + j < ntiles) f(v[j], (c0 + j) * kTile + 4 * lane + quarter);
+        f(v, c0, quarter);
     }
 }
 
@@ -292,15 +291,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     find_bin<kNB1>(s, s.hist1, C, K1, tid);
     const uint32_t d1 = s.res[0];
     uint32_t R = K1 - s.res[1];
-    sweep_keys(tbase, warp, lane, ntiles, [&](uint32_t key, int) {
-        if ((key >> 21) == d1) atomicAdd(&hist2[(key >> 10) & (kNB2 - 1)], 1u);
+    sweep_cols(tbase, warp, ntiles, [&](const uint32_t(&v)[32], int c0, int) {
+        uint32_t m = 0;   // bit j: column c0 + j matches (independent compares, then a short loop)
+#pragma unroll
+        for (int j = 0; j < 32; ++j) m |= (uint32_t)(c0 + j < ntiles && (v[j] >> 21) == d1) << j;
+        while (m != 0u) {
+            const int j = __ffs(m) - 1;
+            m &= m - 1u;
+            atomicAdd(&hist2[(v[j] >> 10) & (kNB2 - 1)], 1u);
+        }
     });
     cl::sync();
     find_bin<kNB2>(s, hist2, C, R, tid);
     const uint32_t p2 = (d1 << 11) | s.res[0];
     R -= s.res[1];
-    sweep_keys(tbase, warp, lane, ntiles, [&](uint32_t key, int) {
-        if ((key >> 10) == p2) atomicAdd(&hist3[key & (kNB3 - 1)], 1u);
+    sweep_cols(tbase, warp, ntiles, [&](const uint32_t(&v)[32], int c0, int) {
+        uint32_t m = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) m |= (uint32_t)(c0 + j < ntiles && (v[j] >> 10) == p2) << j;
+        while (m != 0u) {
+            const int j = __ffs(m) - 1;
+            m &= m - 1u;
+            atomicAdd(&hist3[v[j] & (kNB3 - 1)], 1u);
+        }
     });
     cl::sync();
     find_bin<kNB3>(s, hist3, C, R, tid);
@@ -308,14 +321,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     R -= s.res[1];   // ties at T still to take, lowest positions first (1 <= R)
 
     // ---------------------------------------------------------------- output
+    // keys > T and == T: counted, and marked in position bitmaps (column c of lane l
+    // is entry 128 c + 4 l + q: bitmap word 4 c + l / 8, bit 4 (l % 8) + q)
     uint32_t gt = 0, eq = 0;
-    sweep_keys(tbase, warp, lane, ntiles, [&](uint32_t key, int e) {
-        if (key > T) {
-            atomicOr(&selbm[e >> 5], 1u << (e & 31));
-            ++gt;
-        } else if (key == T) {
-            atomicOr(&tiebm[e >> 5], 1u << (e & 31));
-            ++eq;
+    sweep_cols(tbase, warp, ntiles, [&](const uint32_t(&v)[32], int c0, int q) {
+        uint32_t mg = 0, me = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const bool valid = c0 + j < ntiles;
+            mg |= (uint32_t)(valid && v[j] > T) << j;
+            me |= (uint32_t)(valid && v[j] == T) << j;
+        }
+        gt += __popc(mg);
+        eq += __popc(me);
+        const uint32_t bit = 1u << (4 * (lane & 7) + q);
+        const int w0 = 4 * c0 + (lane >> 3);
+        while (mg != 0u) {
+            const int j = __ffs(mg) - 1;
+            mg &= mg - 1u;
+            atomicOr(&selbm[w0 + 4 * j], bit);
+        }
+        while (me != 0u) {
+            const int j = __ffs(me) - 1;
+            me &= me - 1u;
+            atomicOr(&tiebm[w0 + 4 * j], bit);
         }
     });
 #pragma unroll

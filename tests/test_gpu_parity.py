@@ -201,6 +201,17 @@ def test_index_topk_ties_and_zero_scores(csa):
         assert list(np_(idx)[0, 2]) == list(range(k))
 
 
+def test_device_error_flag_stays_clear(csa):
+    B, Q, cap, k = 2, 1, 3000, 64
+    grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(31, B, Q, cap, [3000, 2000], 1, [[2999], [1999]], k)
+    ws = torch.zeros(csa.csa2_workspace_bytes(csa.OP_INDEX_TOPK, B, Q, cap, k), dtype=torch.uint8, device="cuda")
+    idx = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, k, ws=ws)
+    torch.cuda.synchronize()
+    assert csa.device_error_flag(ws, B, Q) == 0
+    ridx = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, 1, np.array([[2999], [1999]], np.int32), k)
+    assert np.array_equal(np_(idx), ridx)
+
+
 def test_binding_rejects_mismatched_shapes(csa):
     kv = csa.KV(1, 64, 1, "cuda")
     q = torch.zeros((2, 1, 128), dtype=torch.uint8, device="cuda")
