@@ -18,7 +18,6 @@ import hashlib
 import json
 import math
 import os
-import subprocess
 import sys
 import threading
 import time
@@ -94,45 +93,63 @@ def _ncu_traffic():
 
 
 class ClockSampler:
-    """nvidia-smi samples (200 ms) of the SM clock and throttle reasons during the timed region."""
+    """SM clock and clock-event (throttle) reasons of this GPU, read through NVML (the source
+    nvidia-smi reports from) every ~0.5 ms; only samples taken between mark() and stop() count,
+    so they cover the timed region, which lasts a few milliseconds (nvidia-smi's fastest loop,
+    200 ms, would see it once at most)."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
 
-    def __init__(self, index):
-        self.index, self.rows, self.proc = index, [], None
+    def __init__(self, device_index):
+        self.device_index, self.rows, self.t0, self.handle = device_index, [], None, None
+        self.stop_flag = threading.Event()
+
+    def _open(self):
+        import pynvml
+        pynvml.nvmlInit()
+        self.nvml = pynvml
+        try:
+            pr = torch.cuda.get_device_properties(self.device_index)
+            bus = "%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:  # noqa: BLE001 - fall back to the CUDA ordinal
+            return pynvml.nvmlDeviceGetHandleByIndex(self.device_index)
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except OSError:
-            self.proc = None
+            self.handle = self._open()
+        except Exception:  # noqa: BLE001 - no NVML: the record says so
+            self.handle = None
+            return
+        self.max_mhz = float(self.nvml.nvmlDeviceGetMaxClockInfo(self.handle, self.nvml.NVML_CLOCK_SM))
+        get_reasons = getattr(self.nvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            self.nvml.nvmlDeviceGetCurrentClocksThrottleReasons
 
-    def _read(self):
-        for line in self.proc.stdout:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) == 6:
-                self.rows.append(parts)
+        def run():
+            while not self.stop_flag.is_set():
+                t = time.perf_counter()
+                mhz = self.nvml.nvmlDeviceGetClockInfo(self.handle, self.nvml.NVML_CLOCK_SM)
+                self.rows.append((t, float(mhz), int(get_reasons(self.handle))))
+                time.sleep(0.0005)
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+
+    def mark(self):
+        self.t0 = time.perf_counter()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
+        if self.handle is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["NVML unavailable"], "samples": 0}
+        t1 = time.perf_counter()
+        self.stop_flag.set()
         self.thread.join(timeout=2)
-        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
-        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[2 + i].lower() == "active"})
-        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.rows)}
+        rows = [r for r in self.rows if self.t0 is None or self.t0 <= r[0] <= t1]
+        sm = [r[1] for r in rows]
+        reasons = sorted({name for r in rows for name, bit in self.REASONS if r[2] & bit})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(rows), "source": "NVML every ~0.5 ms during the timed region"}
 
 
 # ------------------------------------------------------------------ our arm
@@ -293,11 +310,12 @@ def run_ours(args, rank, world, local_rank):
         torch.distributed.barrier()
     sampler = ClockSampler(local_rank)
     sampler.start()
-    time.sleep(0.3)
+    time.sleep(0.05)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     all_ev = []
+    sampler.mark()
     t_wall = time.perf_counter()
     for _ in range(args.steps):
         flush.zero_()
