@@ -33,6 +33,7 @@ struct AttnSmem {
 };
 
 __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
+    pdl_enter();
     extern __shared__ __align__(128) uint8_t smem_raw[];
     AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -334,8 +335,7 @@ cudaError_t launch_attn(AttnParams& p, int S, cudaStream_t st) {
         attr_set = true;
     }
     dim3 grid(S, p.B * p.Q);
-    attn_kernel<<<grid, kAT, smem, st>>>(p);
-    return cudaGetLastError();
+    return launch_ex(attn_kernel, grid, dim3(kAT), smem, st, 0, p);
 }
 
 }  // namespace csa2

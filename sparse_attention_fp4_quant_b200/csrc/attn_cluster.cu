@@ -44,6 +44,7 @@ struct ClAttnSmem {
 };
 
 __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
+    pdl_enter();
     extern __shared__ __align__(128) uint8_t smem_raw[];
     ClAttnSmem& sm = *reinterpret_cast<ClAttnSmem*>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -365,9 +366,7 @@ int attn_cluster_size(int B, int Q, int slots_total, int* keys_per_cta) {
 
 cudaError_t launch_attn_cluster(AttnParams& p, int C, cudaStream_t st) {
     if (!set_attributes()) return cudaErrorInvalidValue;
-    cudaLaunchAttribute attr[1];
-    const cudaLaunchConfig_t cfg = make_config(C, p.B * p.Q, st, attr);
-    return cudaLaunchKernelEx(&cfg, attn_cluster_kernel, p);
+    return launch_ex(attn_cluster_kernel, dim3(C, p.B * p.Q), dim3(kCT), smem_bytes(), st, C, p);
 }
 
 }  // namespace csa2

@@ -91,4 +91,13 @@ __device__ __forceinline__ int n_visible(int64_t q_pos, int64_t n_entries, int m
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
+// Programmatic dependent launch: let the next kernel of the stream be scheduled
+// now (it waits in its own pdl_enter), then wait until the previous kernel of
+// the stream has completed and its writes are visible.  Every kernel calls it
+// before touching global memory; without a programmatic predecessor the wait
+// returns at once.
+__device__ __forceinline__ void pdl_enter() {
+    asm volatile("griddepcontrol.launch_dependents;\n\tgriddepcontrol.wait;" ::: "memory");
+}
+
 }  // namespace csa2

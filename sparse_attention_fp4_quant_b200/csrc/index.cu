@@ -118,6 +118,7 @@ __device__ void finalize(TK& tk, const SelectParams& p, int bq, int S, int k, in
 
 template <int MODE>
 __global__ void __launch_bounds__(kNT, 2) select_kernel(SelectParams p) {
+    pdl_enter();
     extern __shared__ __align__(16) uint8_t select_smem[];
     TK tk(*reinterpret_cast<TK::Smem*>(select_smem));
     const int tid = threadIdx.x;
@@ -270,10 +271,9 @@ cudaError_t launch_select(int op, SelectParams& p, int S, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         attr[mode] = true;
     }
-    if (mode == 0) select_kernel<MODE_DENSE><<<grid, kNT, smem, st>>>(p);
-    else if (mode == 1) select_kernel<MODE_POOL><<<grid, kNT, smem, st>>>(p);
-    else select_kernel<MODE_BUILD><<<grid, kNT, smem, st>>>(p);
-    return cudaGetLastError();
+    if (mode == 0) return launch_ex(select_kernel<MODE_DENSE>, grid, dim3(kNT), smem, st, 0, p);
+    if (mode == 1) return launch_ex(select_kernel<MODE_POOL>, grid, dim3(kNT), smem, st, 0, p);
+    return launch_ex(select_kernel<MODE_BUILD>, grid, dim3(kNT), smem, st, 0, p);
 }
 
 }  // namespace csa2

@@ -173,6 +173,7 @@ __device__ __forceinline__ void sweep_cols(uint32_t tbase, int warp, int ntiles,
 
 __global__ void __launch_bounds__(kThreads, 1)
     index_cluster_kernel(SelectParams p, const __grid_constant__ CUtensorMap tmap) {
+    pdl_enter();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     ClSmem& s = *reinterpret_cast<ClSmem*>(smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -497,19 +498,7 @@ cudaError_t launch_index_cluster(SelectParams& p, int C, cudaStream_t st) {
     CUtensorMap map;
     if (!pipe::encode_ik_map_perm(&map, p.ik, (int64_t)p.B * p.cap)) return cudaErrorInvalidValue;
     if (!set_attributes()) return cudaErrorInvalidValue;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(C, p.B * p.Q);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem_bytes();
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, index_cluster_kernel, p, map);
+    return launch_ex(index_cluster_kernel, dim3(C, p.B * p.Q), dim3(kThreads), smem_bytes(), st, C, p, map);
 }
 
 }  // namespace csa2

@@ -40,6 +40,7 @@ __device__ __forceinline__ bool epilogue_any(bool v) {
 template <int MODE, int CAP>  // MODE 0 = dense range (index Top-K), 1 = pool blocks (pool Top-K)
 __global__ void __launch_bounds__(kThreads, 2)
     index_tc_kernel(SelectParams p, const __grid_constant__ CUtensorMap tmap) {
+    pdl_enter();
     using TKE = TopK<kEpiN, CAP, 1, kEpiT0>;
     using TcSmem = csa2::TcSmem<CAP>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -211,8 +212,7 @@ cudaError_t launch_tc(SelectParams& p, int S, cudaStream_t st, const CUtensorMap
         attr = true;
     }
     dim3 grid(S, p.B * p.Q);
-    index_tc_kernel<MODE, CAP><<<grid, kThreads, smem, st>>>(p, map);
-    return cudaGetLastError();
+    return launch_ex(index_tc_kernel<MODE, CAP>, grid, dim3(kThreads), smem, st, 0, p, map);
 }
 
 namespace pipe {

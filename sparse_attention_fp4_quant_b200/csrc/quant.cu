@@ -37,6 +37,7 @@ __device__ __forceinline__ void quant16(const float v[16], uint32_t& scale_byte,
 __global__ void __launch_bounds__(256) quant_kernel(const uint16_t* __restrict__ x, int64_t rows, int ch,
                                                     uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                                                     const int64_t* __restrict__ dst_rows, int64_t out_rows) {
+    pdl_enter();
     const int G = ch / 16;
     int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= rows * G) return;
@@ -64,9 +65,8 @@ cudaError_t launch_quant(const void* x, int64_t rows, int ch, uint8_t* codes, ui
     int64_t n = rows * (ch / 16);
     if (n == 0) return cudaSuccess;
     int64_t blocks = (n + 255) / 256;
-    quant_kernel<<<(unsigned)blocks, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, ch, codes, scales, dst_rows,
-                                                  out_rows);
-    return cudaGetLastError();
+    return launch_ex(quant_kernel, dim3((unsigned)blocks), dim3(256), 0, st, 0, static_cast<const uint16_t*>(x), rows, ch,
+                     codes, scales, dst_rows, out_rows);
 }
 
 // k = x W as fp32 fused multiply-add chains over the 512 channels in ascending
@@ -78,6 +78,7 @@ __global__ void __launch_bounds__(256) index_k_proj_kernel(const uint16_t* __res
                                                            const float* __restrict__ W, uint8_t* __restrict__ kc,
                                                            uint8_t* __restrict__ ks,
                                                            const int64_t* __restrict__ dst_rows, int64_t out_rows) {
+    pdl_enter();
     __shared__ float xs[kPC][kPR + 4];
     __shared__ float wsm[kPC][kID + 4];
     __shared__ float outs[kPR][kID + 4];
@@ -156,6 +157,7 @@ __global__ void __launch_bounds__(256) index_k_proj_rows_kernel(const uint16_t* 
                                                                 const float* __restrict__ W, uint8_t* __restrict__ kc,
                                                                 uint8_t* __restrict__ ks,
                                                                 const int64_t* __restrict__ dst_rows, int64_t out_rows) {
+    pdl_enter();
     extern __shared__ __align__(16) float wsm[];   // W [512][64], then the rows [4][512]
     float* xs = wsm + kD * kID;
     __shared__ float outs[kProjRowsPerCTA][kID];
@@ -214,6 +216,7 @@ __global__ void __launch_bounds__(kAppThreads) append_kernel(const uint16_t* __r
                                                              uint8_t* __restrict__ ks,
                                                              const int64_t* __restrict__ dst_rows, int64_t out_rows,
                                                              int nproj) {
+    pdl_enter();
     const int tid = threadIdx.x;
     if ((int)blockIdx.x >= nproj) {
         // latent rows -> NVFP4, one thread per 16 channels
@@ -297,10 +300,9 @@ cudaError_t launch_append(const void* x, int64_t rows, const float* W, uint8_t* 
     }
     const int nproj = (int)((rows + kAppRows - 1) / kAppRows) * 4;
     const int nquant = (int)((rows * (kD / 16) + kAppThreads - 1) / kAppThreads);
-    append_kernel<<<nproj + nquant, kAppThreads, kAppSmem, st>>>(static_cast<const uint16_t*>(x), rows, W, lat_codes,
-                                                                   lat_scales, k_codes, k_scales, dst_rows, out_rows,
-                                                                   nproj);
-    return cudaGetLastError();
+    return launch_ex(append_kernel, dim3(nproj + nquant), dim3(kAppThreads), kAppSmem, st, 0,
+                     static_cast<const uint16_t*>(x), rows, W, lat_codes, lat_scales, k_codes, k_scales, dst_rows,
+                     out_rows, nproj);
 }
 
 cudaError_t launch_index_k_proj(const void* x, int64_t rows, const float* W, uint8_t* k_codes, uint8_t* k_scales,
@@ -314,14 +316,13 @@ cudaError_t launch_index_k_proj(const void* x, int64_t rows, const float* W, uin
             if (e != cudaSuccess) return e;
             attr = true;
         }
-        index_k_proj_rows_kernel<<<(unsigned)((rows + kProjRowsPerCTA - 1) / kProjRowsPerCTA), 256, kProjSmem, st>>>(
-            static_cast<const uint16_t*>(x), rows, W, k_codes, k_scales, dst_rows, out_rows);
-        return cudaGetLastError();
+        return launch_ex(index_k_proj_rows_kernel, dim3((unsigned)((rows + kProjRowsPerCTA - 1) / kProjRowsPerCTA)),
+                         dim3(256), kProjSmem, st, 0, static_cast<const uint16_t*>(x), rows, W, k_codes, k_scales,
+                         dst_rows, out_rows);
     }
     int64_t blocks = (rows + kPR - 1) / kPR;
-    index_k_proj_kernel<<<(unsigned)blocks, 256, 0, st>>>(static_cast<const uint16_t*>(x), rows, W, k_codes,
-                                                          k_scales, dst_rows, out_rows);
-    return cudaGetLastError();
+    return launch_ex(index_k_proj_kernel, dim3((unsigned)blocks), dim3(256), 0, st, 0, static_cast<const uint16_t*>(x),
+                     rows, W, k_codes, k_scales, dst_rows, out_rows);
 }
 
 }  // namespace csa2
