@@ -4,11 +4,11 @@
 // Split-K form, for query counts too large for one cluster per query
 // (attn_cluster.cu serves the rest).  A CTA (8 warps) takes a split of the
 // slot range in tiles of 64 keys.  Each tile is gathered into registers one
-// tile ahead (its loads overlap the previous tile's math), dequantised to bf16
+// tile ahead (its loads overlap the previous tile's math), dequantised to f16
 // in swizzled shared memory (K = V), and S = Q K^T (8 keys per warp) and
 // O += P V (64 dims per warp) run on warp-level tensor-core MMAs with the 16
 // heads as the M dimension; the softmax is online across tiles.  P enters P V
-// as two bf16 terms (rounded value + remainder), about 16 bits of P.  Splits
+// as two f16 terms (rounded value + remainder).  Splits
 // of one query are merged by the last CTA to finish (atomic ticket).
 #include "attn_common.cuh"
 
@@ -21,14 +21,15 @@ constexpr int kMaxSplits = (CSA2_MAX_K + CSA2_MAX_WINDOW + kKT - 1) / kKT;
 struct AttnSmem {
     uint8_t K[kKT * kRowB];   // 64 KB, 16-byte chunks XOR-swizzled by row & 7
     uint8_t Qs[kH * kRowB];   // 16 KB, same swizzle
-    uint8_t P[kH * kKT * 2];  // 2 KB, bf16 P (rounded), 8 chunks per row, same swizzle
-    uint8_t Pl[kH * kKT * 2]; // 2 KB, bf16 remainder P - rounded(P)
+    uint8_t P[kH * kKT * 2];  // 2 KB, f16 P (rounded), 8 chunks per row, same swizzle
+    uint8_t Pl[kH * kKT * 2]; // 2 KB, f16 remainder P - rounded(P)
     float kf[kKT];            // per-key factor (1 for FP4 rows, token scale for SWA)
     int kvalid[kKT];
     float red_max[8][kH];
     float red_sum[8][kH];
     float m_run[kH], l_run[kH], alpha[kH];
     float cw[kMaxSplits][kH];  // combine weights 2^(m_s - M) / L per split and head
+    float qmax[kAT / 32];      // per-warp max |q|
     int last;
 };
 
@@ -47,7 +48,7 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
     const int64_t pos0 = p.swa_pos0[b];
     int64_t nmain = p.n_entries[b];
     if (nmain > p.cap) nmain = p.cap;
-    const float scale_log2 = p.sm_scale * 1.4426950408889634f;
+    float scale_log2 = p.sm_scale * 1.4426950408889634f;
 
     const uint32_t sK = (uint32_t)__cvta_generic_to_shared(sm.K);
     const uint32_t sQ = (uint32_t)__cvta_generic_to_shared(sm.Qs);
@@ -64,14 +65,30 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
     RowQuarter rq;
     if (t0 < t1) fetch_quarter(p, bq, b, t0 * kKT + gr, gq, i_pos, lo, pos0, nmain, rq);
 
-    // Q [16][512] bf16 -> swizzled smem
+    // Q [16][512] bf16 -> f16 times a power-of-two prescale -> swizzled smem
     {
         const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (int64_t)bq * kH * kD);
+        uint4 qv[(kH * kD / 8) / kAT];
+        float qm = 0.0f;
+#pragma unroll
+        for (int it = 0; it < (kH * kD / 8) / kAT; ++it) {
+            qv[it] = __ldg(qsrc + it * kAT + tid);
+            qm = fmaxf(qm, bf16x8_maxabs(qv[it]));
+        }
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) qm = fmaxf(qm, __shfl_xor_sync(0xFFFFFFFFu, qm, o2));
+        if (lane == 0) sm.qmax[warp] = qm;
+        __syncthreads();
+        qm = sm.qmax[0];
+#pragma unroll
+        for (int w = 1; w < kAT / 32; ++w) qm = fmaxf(qm, sm.qmax[w]);
+        const int qe = q_prescale_exp(qm);
+        const float qmul = __uint_as_float((uint32_t)(127 - qe) << 23);   // 2^-qe
+        scale_log2 *= __uint_as_float((uint32_t)(127 + qe) << 23);       // the logits take 2^qe back
 #pragma unroll
         for (int it = 0; it < (kH * kD / 8) / kAT; ++it) {
             const int c = it * kAT + tid;  // 16-byte chunk id
-            const int row = c >> 6, ch = c & 63;
-            *reinterpret_cast<uint4*>(sm.Qs + swz(row, ch)) = __ldg(qsrc + c);
+            *reinterpret_cast<uint4*>(sm.Qs + swz(c >> 6, c & 63)) = bf16x8_to_f16(qv[it], qmul);
         }
     }
     if (tid < kH) {
@@ -98,7 +115,7 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
             ldsm_x4(sQ + swz(lane & 15, 2 * ks + (lane >> 4)), a0, a1, a2, a3);
             const int key = 8 * warp + (lane & 7);
             ldsm_x2(sK + swz(key, 2 * ks + ((lane >> 3) & 1)), b0, b1);
-            mma_bf16(s4, a0, a1, a2, a3, b0, b1);
+            mma_f16(s4, a0, a1, a2, a3, b0, b1);
         }
         // logits (log2 units); masked keys -> -inf
         const int key0 = 8 * warp + 2 * qd;
@@ -131,11 +148,11 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
             const uint32_t off0 = g * 128 + ((chunk ^ (g & 7)) << 4) + within;
             const uint32_t off1 = (g + 8) * 128 + ((chunk ^ ((g + 8) & 7)) << 4) + within;
             const float u00 = p00 * f0, u01 = p01 * f1, u10 = p10 * f0, u11 = p11 * f1;
-            const __nv_bfloat162 h0 = __floats2bfloat162_rn(u00, u01), h1 = __floats2bfloat162_rn(u10, u11);
-            *reinterpret_cast<__nv_bfloat162*>(sm.P + off0) = h0;
-            *reinterpret_cast<__nv_bfloat162*>(sm.P + off1) = h1;
-            *reinterpret_cast<uint32_t*>(sm.Pl + off0) = pack_bf16(u00 - __low2float(h0), u01 - __high2float(h0));
-            *reinterpret_cast<uint32_t*>(sm.Pl + off1) = pack_bf16(u10 - __low2float(h1), u11 - __high2float(h1));
+            const __half2 h0 = __floats2half2_rn(u00, u01), h1 = __floats2half2_rn(u10, u11);
+            *reinterpret_cast<__half2*>(sm.P + off0) = h0;
+            *reinterpret_cast<__half2*>(sm.P + off1) = h1;
+            *reinterpret_cast<uint32_t*>(sm.Pl + off0) = pack_f16(u00 - __low2float(h0), u01 - __high2float(h0));
+            *reinterpret_cast<uint32_t*>(sm.Pl + off1) = pack_f16(u10 - __low2float(h1), u11 - __high2float(h1));
         }
         float sum0 = p00 + p01, sum1 = p10 + p11;
 #pragma unroll
@@ -189,10 +206,10 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
                 for (int np = 0; np < 4; ++np) {
                     uint32_t b0, b1, b2, b3;
                     ldsm_x4_t(sK + swz(key, 8 * warp + 2 * np + (mi >> 1)), b0, b1, b2, b3);
-                    mma_bf16(o[2 * np], a0, a1, a2, a3, b0, b1);
-                    mma_bf16(o[2 * np + 1], a0, a1, a2, a3, b2, b3);
-                    mma_bf16(o[2 * np], l0, l1, l2, l3, b0, b1);
-                    mma_bf16(o[2 * np + 1], l0, l1, l2, l3, b2, b3);
+                    mma_f16(o[2 * np], a0, a1, a2, a3, b0, b1);
+                    mma_f16(o[2 * np + 1], a0, a1, a2, a3, b2, b3);
+                    mma_f16(o[2 * np], l0, l1, l2, l3, b0, b1);
+                    mma_f16(o[2 * np + 1], l0, l1, l2, l3, b2, b3);
                 }
             }
         }

@@ -4,11 +4,11 @@
 // CTA r of the cluster takes the key slots [r * n, (r + 1) * n) of its query
 // (n <= 160, a multiple of 16; slots as in attn_common.cuh) and gathers them
 // all at once, so a CTA waits on global memory once instead of once per tile.
-// The rows are dequantised to bf16 in swizzled shared memory (K = V); with the
+// The rows are dequantised to f16 in swizzled shared memory (K = V); with the
 // 16 heads as the M dimension, S = Q K^T runs on warp-level tensor-core MMAs
 // (each warp a quarter of the channels of a fifth of the keys), then the CTA's
 // own softmax (one warp per head: max and sum over its keys), then O_r = P V
-// (32 dims per warp; P as a rounded bf16 term plus its bf16 remainder).  The partial results meet in distributed shared memory:
+// (32 dims per warp; P as a rounded f16 term plus its f16 remainder).  The partial results meet in distributed shared memory:
 // each CTA stores, into CTA c's (by then idle) key buffer, its slice
 // [c * 512 / C, (c + 1) * 512 / C) of O_r (fp32) and its per-head (max, sum);
 // CTA c then forms its slice of the output as
@@ -33,14 +33,15 @@ static_assert(2 * kH * kSStride * 4 <= kH * kRowB + 2 * kH * kPStride, "partial 
 static_assert((16 * kH * (kD / 16 + 4) + 16 * kH * 2) * 4 <= kMaxKeys * kRowB, "received slices fit the key buffer");
 
 struct ClAttnSmem {
-    uint8_t K[kMaxKeys * kRowB];   // bf16 keys (= values), swizzled; afterwards the received output slices
-    uint8_t Qs[kH * kRowB];        // bf16 query, swizzled; then (with P) the two partial S arrays
-    uint8_t P[kH * kPStride];      // bf16 P (rounded), [head][key]
-    uint8_t Pl[kH * kPStride];     // bf16 remainder P - rounded(P)
+    uint8_t K[kMaxKeys * kRowB];   // f16 keys (= values), swizzled; afterwards the received output slices
+    uint8_t Qs[kH * kRowB];        // f16 query (prescaled), swizzled; then (with P) the two partial S arrays
+    uint8_t P[kH * kPStride];      // f16 P (rounded), [head][key]
+    uint8_t Pl[kH * kPStride];     // f16 remainder P - rounded(P)
     float kf[kMaxKeys];            // per-key factor (1 for FP4 rows, token scale for SWA)
     int kvalid[kMaxKeys];
     alignas(16) float ml[kH][2];   // this CTA's (max, sum) per head (log2 units), read by the cluster
     float cw[16][kH];              // combine weight of rank c for head h (for this CTA's output slice)
+    float qmax[kCT / 32];          // per-warp max |q|
 };
 
 __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
@@ -58,7 +59,7 @@ __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
     const int64_t pos0 = p.swa_pos0[b];
     int64_t nmain = p.n_entries[b];
     if (nmain > p.cap) nmain = p.cap;
-    const float scale_log2 = p.sm_scale * 1.4426950408889634f;
+    float scale_log2 = p.sm_scale * 1.4426950408889634f;
 
     // this CTA's slots [s0, s0 + nk), padded to n16 (dead slots past nk)
     const int s0 = min(p.slots_total, (int)rank * p.keys_per_cta);
@@ -104,14 +105,27 @@ __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
         uint4 qv[(kH * kD / 8) / kCT];
 #pragma unroll
         for (int it = 0; it < (kH * kD / 8) / kCT; ++it) qv[it] = ld_nc_v4(qsrc + 16 * (it * kCT + tid));
+        float qm = 0.0f;   // max |q| of the query, for its power-of-two prescale into f16
 #pragma unroll
-        for (int it = 0; it < (kH * kD / 8) / kCT; ++it) {
-            const int c = it * kCT + tid;   // 16-byte chunk id
-            *reinterpret_cast<uint4*>(sm.Qs + swz(c >> 6, c & 63)) = qv[it];
-        }
+        for (int it = 0; it < (kH * kD / 8) / kCT; ++it) qm = fmaxf(qm, bf16x8_maxabs(qv[it]));
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) qm = fmaxf(qm, __shfl_xor_sync(0xFFFFFFFFu, qm, o2));
+        if (lane == 0) sm.qmax[warp] = qm;
 #pragma unroll
         for (int j = 0; j < kPer; ++j)
             if (rr[j] >= 0) store_quarter(sm.K, sm.kf, sm.kvalid, rr[j], qs[j], rq[j]);
+        __syncthreads();
+        qm = sm.qmax[0];
+#pragma unroll
+        for (int w = 1; w < kCT / 32; ++w) qm = fmaxf(qm, sm.qmax[w]);
+        const int qe = q_prescale_exp(qm);
+        const float qmul = __uint_as_float((uint32_t)(127 - qe) << 23);   // 2^-qe
+        scale_log2 *= __uint_as_float((uint32_t)(127 + qe) << 23);       // the logits take 2^qe back
+#pragma unroll
+        for (int it = 0; it < (kH * kD / 8) / kCT; ++it) {
+            const int c = it * kCT + tid;   // 16-byte chunk id
+            *reinterpret_cast<uint4*>(sm.Qs + swz(c >> 6, c & 63)) = bf16x8_to_f16(qv[it], qmul);
+        }
     }
     __syncthreads();
 
@@ -136,7 +150,7 @@ __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
                 for (int j = 0; j < 8; ++j) {
                     uint32_t b0, b1;
                     ldsm_x2(sK + swz(8 * tile + (lane & 7), 2 * (8 * kg + j) + ((lane >> 3) & 1)), b0, b1);
-                    mma_bf16(s4[i], qa[j][0], qa[j][1], qa[j][2], qa[j][3], b0, b1);
+                    mma_f16(s4[i], qa[j][0], qa[j][1], qa[j][2], qa[j][3], b0, b1);
                 }
             }
         }
@@ -197,9 +211,9 @@ __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
             const int t = lane + 32 * j;
             if (t < n16) {
                 const float u = z[j] * fk[j];
-                const __nv_bfloat16 hi = __float2bfloat16_rn(u);
-                *reinterpret_cast<__nv_bfloat16*>(sm.P + h * kPStride + 2 * t) = hi;
-                *reinterpret_cast<__nv_bfloat16*>(sm.Pl + h * kPStride + 2 * t) = __float2bfloat16_rn(u - __bfloat162float(hi));
+                const __half hi = __float2half_rn(u);
+                *reinterpret_cast<__half*>(sm.P + h * kPStride + 2 * t) = hi;
+                *reinterpret_cast<__half*>(sm.Pl + h * kPStride + 2 * t) = __float2half_rn(u - __half2float(hi));
             }
         }
         if (lane == 0) {
@@ -226,10 +240,10 @@ __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
         for (int np = 0; np < 2; ++np) {
             uint32_t b0, b1, b2, b3;
             ldsm_x4_t(sK + swz(key, 4 * warp + 2 * np + (mi >> 1)), b0, b1, b2, b3);
-            mma_bf16(o[2 * np], a0, a1, a2, a3, b0, b1);
-            mma_bf16(o[2 * np + 1], a0, a1, a2, a3, b2, b3);
-            mma_bf16(o[2 * np], l0, l1, l2, l3, b0, b1);
-            mma_bf16(o[2 * np + 1], l0, l1, l2, l3, b2, b3);
+            mma_f16(o[2 * np], a0, a1, a2, a3, b0, b1);
+            mma_f16(o[2 * np + 1], a0, a1, a2, a3, b2, b3);
+            mma_f16(o[2 * np], l0, l1, l2, l3, b0, b1);
+            mma_f16(o[2 * np + 1], l0, l1, l2, l3, b2, b3);
         }
     }
 

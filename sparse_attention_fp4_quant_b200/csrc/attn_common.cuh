@@ -1,22 +1,24 @@
 // attn_common.cuh -- device pieces shared by the sparse-attention kernels:
-// exact FP4 / FP8 -> bf16 decoding, the row-quarter gather of one key slot,
-// ldmatrix / mma.sync wrappers, and the swizzled bf16 row layout.
+// exact FP4 / FP8 -> f16 decoding, the row-quarter gather of one key slot,
+// ldmatrix / mma.sync wrappers, and the swizzled 16-bit row layout.
 //
 // Key slots of a query: [0, k) are the main rows idx[0..k), [k, k + W) are the
 // window tokens i - W + 1 .. i.  A slot is live if its row exists and (for the
 // window) the token lies in [max(s, i - W + 1), i] and in the stored SWA rows.
-// FP4 rows dequantise exactly to bf16 (byte-table decode, then an exact bf16
-// multiply by the block scale); an SWA row is kept as its E4M3 values (exact in
-// bf16) and its fp32 token scale multiplies the logit and the probability.
+// Keys and values are f16 in shared memory: FP4 rows dequantise exactly (the
+// hardware E2M1 -> f16 conversion, then an exact f16 multiply by the block
+// scale); an SWA row is kept as its E4M3 values (exact in f16) and its fp32
+// token scale multiplies the logit and the probability.  The bf16 query is
+// brought into f16 range by a power of two that the logits take back.
 #pragma once
 #include "common.cuh"
 #include "kernels.h"
 
 namespace csa2 {
 
-constexpr int kRowB = kD * 2;   // bytes per bf16 row of 512
+constexpr int kRowB = kD * 2;   // bytes per 16-bit row of 512
 
-// 16-byte chunk `chunk` of bf16 row `row`, XOR-swizzled by row & 7.
+// 16-byte chunk `chunk` of 16-bit row `row`, XOR-swizzled by row & 7.
 __device__ __forceinline__ uint32_t swz(int row, int chunk) { return (uint32_t)(row * kRowB + ((chunk ^ (row & 7)) << 4)); }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -24,36 +26,68 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
-    __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+__device__ __forceinline__ uint32_t pack_f16(float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
+    __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
     return *reinterpret_cast<uint32_t*>(&r);
 }
 
-// 8 E2M1 codes (nibble n = dim n) times the block scale (bf16x2 s2) -> 8 bf16.
-// The magnitudes come from byte tables (high and low byte of the bf16 value),
-// the sign is moved to bit 15 of each half, and the product with the scale is
-// exact (at most 6 significant bits).
-__device__ __forceinline__ uint4 fp4x8_to_bf16(uint32_t w, uint32_t s2) {
-    const uint32_t HI0 = 0x3F3F3F00u, HI1 = 0x40404040u;   // 0 .5 1 1.5 | 2 3 4 6: high bytes
-    const uint32_t LO0 = 0xC0800000u, LO1 = 0xC0804000u;   //                     low bytes
-    const uint32_t m = w & 0x77777777u, mh = m >> 16;
-    const uint32_t hi_a = __byte_perm(HI0, HI1, m), lo_a = __byte_perm(LO0, LO1, m);
-    const uint32_t hi_b = __byte_perm(HI0, HI1, mh), lo_b = __byte_perm(LO0, LO1, mh);
-    uint32_t v0 = __byte_perm(lo_a, hi_a, 0x5140), v1 = __byte_perm(lo_a, hi_a, 0x7362);
-    uint32_t v2 = __byte_perm(lo_b, hi_b, 0x5140), v3 = __byte_perm(lo_b, hi_b, 0x7362);
-    // nibble signs (bits 3 and 7 of each byte) -> bits 15 and 31 of the bf16 pair
-    v0 |= ((w & 0x88u) * 0x1001000u) & 0x80008000u;
-    v1 |= (((w >> 8) & 0x88u) * 0x1001000u) & 0x80008000u;
-    v2 |= (((w >> 16) & 0x88u) * 0x1001000u) & 0x80008000u;
-    v3 |= (((w >> 24) & 0x88u) * 0x1001000u) & 0x80008000u;
-    return make_uint4(bf16x2_mul(v0, s2), bf16x2_mul(v1, s2), bf16x2_mul(v2, s2), bf16x2_mul(v3, s2));
+// 8 E2M1 codes (nibble n = dim n) times the block scale (f16x2 s2) -> 8 f16,
+// by the hardware E2M1 -> f16 conversion.  Every E2M1 x E4M3 product (at most
+// 5 significant bits, 2^-10 .. 2688) is exact in f16, so the multiply is exact.
+__device__ __forceinline__ uint4 fp4x8_to_f16(uint32_t w, uint32_t s2) {
+    uint32_t r0, r1, r2, r3;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\tcvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\tcvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+        : "r"(w));
+    return make_uint4(f16x2_mul(r0, s2), f16x2_mul(r1, s2), f16x2_mul(r2, s2), f16x2_mul(r3, s2));
 }
 
-// 4 E4M3 bytes -> 4 bf16 (exact).
-__device__ __forceinline__ uint2 fp8x4_to_bf16(uint32_t w) {
-    float f[4];
-    e4m3x4_to_f32(w, f);
-    return make_uint2(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]));
+// 4 E4M3 bytes -> 4 f16 (exact).
+__device__ __forceinline__ uint2 fp8x4_to_f16(uint32_t w) {
+    uint32_t lo, hi;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(lo) : "h"((uint16_t)(w & 0xFFFFu)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hi) : "h"((uint16_t)(w >> 16)));
+    return make_uint2(lo, hi);
+}
+
+// Power-of-two exponent e >= 0 that brings max |q| below 2^15, so q 2^-e fits f16
+// exactly (bf16 has 8 significant bits) except for values under 2^-14.
+__device__ __forceinline__ int q_prescale_exp(float maxabs) {
+    const int ex = (int)((__float_as_uint(maxabs) >> 23) & 0xFFu) - 127;
+    return max(0, ex - 14);
+}
+
+// 8 bf16 (a 16-byte chunk) times 2^-e -> 8 f16.
+__device__ __forceinline__ uint4 bf16x8_to_f16(uint4 v, float mul) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = pack_f16(__uint_as_float(w[i] << 16) * mul, __uint_as_float(w[i] & 0xFFFF0000u) * mul);
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ float bf16x8_maxabs(uint4 v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xFFFF0000u))));
+    return m;
+}
+
+__device__ __forceinline__ void mma_f16(float c[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                        uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -70,15 +104,6 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                  : "r"(addr));
-}
-
-__device__ __forceinline__ void mma_bf16(float c[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
-                                         uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 // One quarter (128 dims) of one key row, held in registers between its load
@@ -175,13 +200,15 @@ __device__ __forceinline__ void issue_quarter(const AttnParams& p, int kind, int
 
 __device__ __forceinline__ void store_quarter(uint8_t* K, float* kf, int* kvalid, int r, int qq, const RowQuarter& q) {
     if (q.kind == 1) {
-        uint32_t s2[8];   // the 8 block scales as bf16 pairs (exact: E4M3 fits bf16)
+        uint32_t s2[8];   // the 8 block scales as f16 pairs (exact: E4M3 fits f16)
         {
-            float f[8];
-            e4m3x4_to_f32(q.sc.x, f);
-            e4m3x4_to_f32(q.sc.y, f + 4);
+            const uint2 sp = fp8x4_to_f16(q.sc.x), sq = fp8x4_to_f16(q.sc.y);
+            const uint32_t pr[4] = {sp.x, sp.y, sq.x, sq.y};
 #pragma unroll
-            for (int i = 0; i < 8; ++i) s2[i] = pack_bf16(f[i], f[i]);
+            for (int i = 0; i < 4; ++i) {
+                s2[2 * i] = __byte_perm(pr[i], 0u, 0x1010);       // (low, low)
+                s2[2 * i + 1] = __byte_perm(pr[i], 0u, 0x3232);   // (high, high)
+            }
         }
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
@@ -189,14 +216,14 @@ __device__ __forceinline__ void store_quarter(uint8_t* K, float* kf, int* kvalid
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int word = 4 * v + j;   // 8 dims per word, one scale per 16 dims
-                *reinterpret_cast<uint4*>(K + swz(r, 16 * qq + word)) = fp4x8_to_bf16(ws[j], s2[word >> 1]);
+                *reinterpret_cast<uint4*>(K + swz(r, 16 * qq + word)) = fp4x8_to_f16(ws[j], s2[word >> 1]);
             }
         }
     } else if (q.kind == 2) {
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
-            const uint2 a = fp8x4_to_bf16(q.raw[v].x), bb = fp8x4_to_bf16(q.raw[v].y);
-            const uint2 c = fp8x4_to_bf16(q.raw[v].z), d = fp8x4_to_bf16(q.raw[v].w);
+            const uint2 a = fp8x4_to_f16(q.raw[v].x), bb = fp8x4_to_f16(q.raw[v].y);
+            const uint2 c = fp8x4_to_f16(q.raw[v].z), d = fp8x4_to_f16(q.raw[v].w);
             *reinterpret_cast<uint4*>(K + swz(r, 16 * qq + 2 * v)) = make_uint4(a.x, a.y, bb.x, bb.y);
             *reinterpret_cast<uint4*>(K + swz(r, 16 * qq + 2 * v + 1)) = make_uint4(c.x, c.y, d.x, d.y);
         }
