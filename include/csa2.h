@@ -68,7 +68,8 @@ typedef enum {
     CSA2_ERR_INVALID_ARG = 1,
     CSA2_ERR_UNSUPPORTED = 2,
     CSA2_ERR_WORKSPACE = 3,
-    CSA2_ERR_CUDA = 4
+    CSA2_ERR_CUDA = 4,
+    CSA2_ERR_TIMEOUT = 5
 } csa2_status;
 
 /* Human-readable name of a status (static storage, never NULL). */
@@ -251,6 +252,15 @@ CSA2_API size_t csa2_workspace_bytes(csa2_op op, int32_t B, int32_t Q, int64_t c
 
 /* Byte offset of the sticky device error flag in an index / pool workspace. */
 #define CSA2_STATUS_OFFSET(B, Q) ((((size_t)(B) * (size_t)(Q) * 4u) + 255u) & ~(size_t)255u)
+
+/*
+ * Reads the sticky device error flag of an index / pool workspace used with
+ * batch B and Q queries: waits for `stream` (this call synchronises, unlike the
+ * others), returns CSA2_ERR_TIMEOUT if a device-side wait of a call on that
+ * workspace ran out of time (its results are not valid), else CSA2_OK.  With
+ * clear != 0 the flag is reset to 0 on `stream`.
+ */
+CSA2_API csa2_status csa2_device_status(void* ws, int32_t B, int32_t Q, int32_t clear, void* stream);
 
 /*
  * Step 5 -- one CSA2 layer dispatched by its static mode ([Blog] "CSA2"

@@ -47,7 +47,7 @@ _lib = None
 EXPORTS = ["csa2_status_str", "csa2_last_cuda_error", "csa2_quant_nvfp4", "csa2_index_k_proj", "csa2_append_tokens",
            "csa2_index_topk",
            "csa2_pool_build", "csa2_pool_topk", "csa2_sparse_attn", "csa2_workspace_bytes", "csa2_layer_step",
-           "csa2_index_topk_noalloc"]
+           "csa2_index_topk_noalloc", "csa2_device_status"]
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -67,6 +67,7 @@ def lib():
         "csa2_quant_nvfp4": (ctypes.c_int, [P, i64, i32, P, P, P, i64, P]),
         "csa2_index_k_proj": (ctypes.c_int, [P, i64, P, P, P, P, i64, P]),
         "csa2_append_tokens": (ctypes.c_int, [P, i64, P, P, P, P, P, P, i64, P]),
+        "csa2_device_status": (ctypes.c_int, [P, i32, i32, i32, P]),
         "csa2_index_topk": (ctypes.c_int, [P, P, P, KVP, P, i32, i32, i32, P, P, P, sz, P]),
         "csa2_pool_build": (ctypes.c_int, [P, KVP, P, i32, i32, i32, P, P, sz, P]),
         "csa2_pool_topk": (ctypes.c_int, [P, P, P, KVP, P, i32, P, i32, i32, i32, P, P, sz, P]),
@@ -171,6 +172,12 @@ def device_error_flag(ws, B, Q):
     """The workspace's sticky device error flag (1 after a device-side wait ran out of time)."""
     off = status_offset(B, Q)
     return int(ws[off:off + 4].view(torch.int32).item())
+
+
+def csa2_device_status(ws, B, Q, clear=False):
+    """Waits for the current stream; raises CSA2Error (CSA2_ERR_TIMEOUT) if a call on this
+    workspace had a device-side wait run out of time."""
+    _check(lib().csa2_device_status(_ptr(ws), B, Q, 1 if clear else 0, _stream()))
 
 
 def csa2_workspace_bytes(op, B, Q, cap, k, P=0):

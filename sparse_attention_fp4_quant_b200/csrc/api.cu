@@ -59,6 +59,7 @@ const char* csa2_status_str(csa2_status s) {
         case CSA2_ERR_UNSUPPORTED: return "CSA2_ERR_UNSUPPORTED";
         case CSA2_ERR_WORKSPACE: return "CSA2_ERR_WORKSPACE";
         case CSA2_ERR_CUDA: return "CSA2_ERR_CUDA";
+        case CSA2_ERR_TIMEOUT: return "CSA2_ERR_TIMEOUT";
     }
     return "CSA2_ERR_UNKNOWN";
 }
@@ -95,6 +96,17 @@ csa2_status csa2_append_tokens(const void* x, int64_t rows, const float* W, uint
     if (out_rows < 0 || (!dst_rows && out_rows < rows)) return CSA2_ERR_INVALID_ARG;
     return cuda_status(launch_append(x, rows, W, lat_codes, lat_scales, k_codes, k_scales, dst_rows, out_rows,
                                      (cudaStream_t)stream));
+}
+
+csa2_status csa2_device_status(void* ws, int32_t B, int32_t Q, int32_t clear, void* stream) {
+    if (!ws || B < 1 || Q < 1) return CSA2_ERR_INVALID_ARG;
+    char* flag_ptr = static_cast<char*>(ws) + CSA2_STATUS_OFFSET(B, Q);
+    int32_t flag = 0;
+    cudaError_t e = cudaMemcpyAsync(&flag, flag_ptr, sizeof(flag), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e == cudaSuccess && flag && clear) e = cudaMemsetAsync(flag_ptr, 0, sizeof(flag), (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_status(e);
+    return flag ? CSA2_ERR_TIMEOUT : CSA2_OK;
 }
 
 size_t csa2_workspace_bytes(csa2_op op, int32_t B, int32_t Q, int64_t cap, int32_t k, int32_t P) {

@@ -35,6 +35,7 @@ def test_status_strings(L):
     assert L.csa2_status_str(0) == b"CSA2_OK"
     assert L.csa2_status_str(1) == b"CSA2_ERR_INVALID_ARG"
     assert L.csa2_status_str(4) == b"CSA2_ERR_CUDA"
+    assert L.csa2_status_str(5) == b"CSA2_ERR_TIMEOUT"
 
 
 def test_workspace_sizes_are_host_only(L):
@@ -71,3 +72,4 @@ def test_invalid_arguments_rejected_before_launch(L):
     assert L.csa2_sparse_attn(fake, ctypes.byref(kv), fake, 512, fake, fake, fake, 128, 129, None, fake, 1, 1,
                               ctypes.c_float(0.04), fake, None, fake, 1 << 20, None) == 1   # window > 128
     assert L.csa2_layer_step(None, None) == 1
+    assert L.csa2_device_status(None, 1, 1, 0, None) == 1   # no workspace

@@ -177,6 +177,29 @@ def test_index_blockmax_signed_zero_and_negative_weights(csa):
     assert np.array_equal(np_(bm).view(np.uint32), rbm.view(np.uint32))   # bits, so -0 != +0
 
 
+def test_index_scores_extreme_block_scales(csa):
+    # block scales at the ends of E4M3 (subnormal 2^-9 .. 448) on keys and queries, mixed within
+    # a row: each accumulator column of the block-scaled MMA holds one block, so the scores (seen
+    # directly through the block maxima) stay bit-exact whatever the exponent spread
+    B, Q, cap, k = 1, 2, 4096, 512
+    rng = np.random.default_rng(17)
+    grp = Group(18, B, cap, [cap])
+    o = {kk: v.copy() for kk, v in grp.oracle_cache().items()}
+    extremes = np.array([0x01, 0x02, 0x08, 0x30, 0x40, 0x77, 0x7E], np.uint8)
+    iks = extremes[rng.integers(0, len(extremes), size=(B, cap, 4))].astype(np.uint8)
+    o["iks"] = iks
+    grp.kv.ik_sc.copy_(torch.from_numpy(iks))
+    iq, iqs, w, oiq, oiqs, ow = index_query(19, B, Q)
+    qsc = extremes[rng.integers(0, len(extremes), size=(B, Q, 16))].astype(np.uint8)
+    oiqs = qsc
+    iqs.copy_(torch.from_numpy(qsc))
+    q_pos = np.array([[cap - 1, cap // 2]], np.int32)
+    idx, bm = csa.csa2_index_topk(iq, iqs, w, grp.kv, torch.from_numpy(q_pos).cuda(), k, blockmax=True)
+    ridx, rbm = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, 1, q_pos, k, blockmax=True)
+    assert np.array_equal(np_(bm).view(np.uint32), rbm.view(np.uint32))
+    assert np.array_equal(np_(idx), ridx)
+
+
 def test_index_topk_ties_and_zero_scores(csa):
     B, Q, cap = 1, 3, 20000
     grp = Group(21, B, cap, [20000])
@@ -208,6 +231,7 @@ def test_device_error_flag_stays_clear(csa):
     idx = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, k, ws=ws)
     torch.cuda.synchronize()
     assert csa.device_error_flag(ws, B, Q) == 0
+    csa.csa2_device_status(ws, B, Q)   # raises on CSA2_ERR_TIMEOUT
     ridx = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, 1, np.array([[2999], [1999]], np.int32), k)
     assert np.array_equal(np_(idx), ridx)
 
