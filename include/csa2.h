@@ -30,7 +30,16 @@
  *                      low nibble of byte j, 2j+1 in the high nibble) plus 32 B
  *                      of E4M3 scales, one per 16 channels (NVFP4 without the
  *                      second-level scale: [Blog] FP4 section, [Lsln] 4.3).
- *   indexer K row    : 64 channels -> 32 B codes + 4 B scales.
+ *   indexer K row    : 64 channels -> 32 B codes + 4 B scales; the codes are
+ *                      stored in the tiled order below (not row-major).
+ *   indexer K codes  : entries in tiles of 128 (entry e = tile e / 128, row
+ *                      e % 128); a tile's codes are 4096 contiguous bytes, and
+ *                      half h (channels 32h .. 32h + 31, 16 B) of entry e is at
+ *                        4096 (e / 128) + 256 ((e / 8) % 16) + 128 h + 16 (e % 8).
+ *                      This is the tensor cores' shared-memory operand image of
+ *                      a 128-row tile, so a tile moves with one bulk copy and a
+ *                      block of 8 entries is 256 contiguous bytes.
+ *   indexer K scales : row-major, 4 bytes per entry (blocks 0..3 in order).
  *   indexer Q        : per query [4 heads][32 B] codes + [4][4] scales.
  *   E2M1 code        : bit 3 sign, bits 2:1 exponent (bias 1), bit 0 mantissa.
  *   E4M3 byte        : "FN" variant, bias 7, no infinities, 0x7F/0xFF NaN
@@ -85,10 +94,12 @@ CSA2_API int csa2_last_cuda_error(void);
  * Reindex and Reuse layers ([Blog] "CSA2" section, Fig. 4).
  *   lat       device [B][cap][256]  E2M1 codes of the main latent
  *   lat_sc    device [B][cap][32]   E4M3 scales of the main latent
- *   ik        device [B][cap][32]   E2M1 codes of the indexer K
- *   ik_sc     device [B][cap][4]    E4M3 scales of the indexer K
+ *   ik        device [B][cap][32]   E2M1 codes of the indexer K (tiled order above;
+ *                                   entry e of batch row b is cache entry b cap + e)
+ *   ik_sc     device [B][cap][4]    E4M3 scales of the indexer K (row-major)
  *   n_entries device [B] int32      valid entries per batch row (clamped to [0, cap])
- *   cap       entries allocated per batch row (>= 1)
+ *   cap       entries allocated per batch row: a positive multiple of 128
+ *             (calls that read ik return CSA2_ERR_INVALID_ARG otherwise)
  *   m         tokens compressed into one entry: 1 (decoder) or 2 (encoder).
  *             Entry e covers tokens [m e, m e + m - 1] and is visible to the
  *             query at token p once complete: m e + m - 1 <= p.
@@ -132,8 +143,10 @@ CSA2_API csa2_status csa2_quant_nvfp4(const void* x, int64_t rows, int32_t ch, u
  * codes + 4 B scales).
  *   x        device bf16 [rows][512] (post-RoPE latent rows), 16-byte aligned
  *   W        device fp32 [512][64], 16-byte aligned
- *   k_codes  device u8 [out_rows][32] (8-byte aligned), k_scales device u8 [out_rows][4];
- *            row mapping and out_rows as for csa2_quant_nvfp4
+ *   k_codes  device u8 [out_rows][32] (8-byte aligned) in the tiled indexer-K
+ *            code order (output row r = cache entry r); k_scales device u8 [out_rows][4];
+ *            row mapping as for csa2_quant_nvfp4; out_rows a multiple of 128
+ *            (else CSA2_ERR_INVALID_ARG)
  */
 CSA2_API csa2_status csa2_index_k_proj(const void* x, int64_t rows, const float* W, uint8_t* k_codes,
                                        uint8_t* k_scales, const int64_t* dst_rows, int64_t out_rows, void* stream);

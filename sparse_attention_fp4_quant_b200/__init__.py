@@ -14,6 +14,7 @@ import os
 import torch
 
 D, H, IH, ID, BLOCK, MAX_K, MAX_WINDOW = 512, 16, 4, 64, 8, 2048, 128
+IK_TILE = 128   # entries per tile of the indexer-K cache order
 TOPK, POOL_BLOCKS, WINDOW = 512, 2048, 128
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -127,6 +128,8 @@ class KV:
     """The shared global KV of a CSA2 layer group (device tensors) and its csa2_kv view."""
 
     def __init__(self, B, cap, m=1, device="cuda"):
+        if cap <= 0 or cap % IK_TILE:
+            raise ValueError(f"cap must be a positive multiple of {IK_TILE} (the indexer-K tile), got {cap}")
         self.B, self.cap, self.m = B, cap, m
         self.lat = torch.zeros((B, cap, D // 2), dtype=torch.uint8, device=device)
         self.lat_sc = torch.zeros((B, cap, D // 16), dtype=torch.uint8, device=device)
@@ -202,9 +205,10 @@ def csa2_index_k_proj(x, W, k_codes=None, k_scales=None, dst_rows=None):
     _dev(x, torch.bfloat16, "x")
     _dev(W, torch.float32, "W")
     rows = x.reshape(-1, D).shape[0]
-    if k_codes is None:
-        k_codes = torch.empty((rows, ID // 2), dtype=torch.uint8, device=x.device)
-        k_scales = torch.empty((rows, ID // 16), dtype=torch.uint8, device=x.device)
+    if k_codes is None:   # whole tiles of the indexer-K order
+        out_rows = (rows + IK_TILE - 1) // IK_TILE * IK_TILE
+        k_codes = torch.empty((out_rows, ID // 2), dtype=torch.uint8, device=x.device)
+        k_scales = torch.empty((out_rows, ID // 16), dtype=torch.uint8, device=x.device)
     if dst_rows is not None:
         _dev(dst_rows, torch.int64, "dst_rows")
     _check(lib().csa2_index_k_proj(_ptr(x), rows, _ptr(W), _ptr(k_codes), _ptr(k_scales), _ptr(dst_rows),

@@ -23,7 +23,9 @@ bool kv_ok(const csa2_kv* kv) {
     return kv && kv->n_entries && kv->cap >= 1 && (kv->m == 1 || kv->m == 2) && kv->cap <= (int64_t(1) << 31) / 8;
 }
 
-bool kv_index_ok(const csa2_kv* kv) { return kv_ok(kv) && kv->ik && kv->ik_sc && aligned16(kv->ik) && aligned16(kv->ik_sc); }
+bool kv_index_ok(const csa2_kv* kv) {
+    return kv_ok(kv) && kv->ik && kv->ik_sc && aligned16(kv->ik) && aligned16(kv->ik_sc) && kv->cap % 128 == 0;
+}
 
 bool kv_latent_ok(const csa2_kv* kv) {
     return kv_ok(kv) && kv->lat && kv->lat_sc && aligned16(kv->lat) && aligned16(kv->lat_sc);
@@ -81,7 +83,7 @@ csa2_status csa2_index_k_proj(const void* x, int64_t rows, const float* W, uint8
     if (rows == 0) return CSA2_OK;
     if (!x || !W || !k_codes || !k_scales || !aligned16(x) || !aligned16(W) || ((uintptr_t)k_codes & 7u))
         return CSA2_ERR_INVALID_ARG;
-    if (out_rows < 0 || (!dst_rows && out_rows < rows)) return CSA2_ERR_INVALID_ARG;
+    if (out_rows < 0 || out_rows % 128 != 0 || (!dst_rows && out_rows < rows)) return CSA2_ERR_INVALID_ARG;
     return cuda_status(launch_index_k_proj(x, rows, W, k_codes, k_scales, dst_rows, out_rows, (cudaStream_t)stream));
 }
 
@@ -93,7 +95,7 @@ csa2_status csa2_append_tokens(const void* x, int64_t rows, const float* W, uint
     if (!x || !W || !lat_codes || !lat_scales || !k_codes || !k_scales || !aligned16(x) || !aligned16(W) ||
         ((uintptr_t)lat_codes & 7u) || ((uintptr_t)k_codes & 7u))
         return CSA2_ERR_INVALID_ARG;
-    if (out_rows < 0 || (!dst_rows && out_rows < rows)) return CSA2_ERR_INVALID_ARG;
+    if (out_rows < 0 || out_rows % 128 != 0 || (!dst_rows && out_rows < rows)) return CSA2_ERR_INVALID_ARG;
     return cuda_status(launch_append(x, rows, W, lat_codes, lat_scales, k_codes, k_scales, dst_rows, out_rows,
                                      (cudaStream_t)stream));
 }

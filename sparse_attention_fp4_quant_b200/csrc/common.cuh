@@ -81,6 +81,33 @@ __device__ __forceinline__ uint32_t score_key(float s) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// ---- indexer-K cache layout ---------------------------------------------
+// Codes: tiles of 128 entries stored as the tensor core reads its K-major
+// operand without swizzle: 8-row x 16-byte core matrices, the two 16-byte
+// halves of a row 128 bytes apart, row groups of 8 at 256 bytes.  For entry e
+// (counted over the whole [B][cap] cache, cap a multiple of 128), half kc of its
+// 32 code bytes starts at ik_code_off(e, kc).  Scales: row-major, 4 bytes per
+// entry at ik_scale_off(e).
+__host__ __device__ __forceinline__ int64_t ik_code_off(int64_t e, int kc) {
+    return ((e >> 7) << 12) + (((e >> 3) & 15) << 8) + ((int64_t)kc << 7) + ((e & 7) << 4);
+}
+
+__host__ __device__ __forceinline__ int64_t ik_scale_off(int64_t e) { return e * 4; }
+
+// Maximum over the 8 lanes of an aligned lane octet (one pool block of 8
+// consecutive entries), in position order: a later score replaces the running
+// maximum only when strictly larger, so of equal maxima (+0 and -0) the first wins.
+__device__ __forceinline__ float block_max8(float score, int lane) {
+    float mx = score;
+#pragma unroll
+    for (int o = 1; o < kBlk; o <<= 1) {
+        const float other = __shfl_xor_sync(0xFFFFFFFFu, mx, o);
+        const float earlier = (lane & o) ? other : mx, later = (lane & o) ? mx : other;
+        mx = later > earlier ? later : earlier;
+    }
+    return mx;
+}
+
 __device__ __forceinline__ int n_visible(int64_t q_pos, int64_t n_entries, int m, int64_t cap) {
     int64_t v = (q_pos + 1) / (m > 0 ? m : 1);
     if (n_entries > cap) n_entries = cap;

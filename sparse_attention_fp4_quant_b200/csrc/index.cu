@@ -68,9 +68,9 @@ __device__ __forceinline__ float entry_score(const QReg& R, uint4 c0, uint4 c1, 
 }
 
 __device__ __forceinline__ float entry_score_at(const QReg& R, const uint8_t* ik, const uint8_t* iks, int64_t e) {
-    const uint4* c = reinterpret_cast<const uint4*>(ik + e * 32);
-    uint4 c0 = __ldg(c), c1 = __ldg(c + 1);
-    uint32_t sw = __ldg(reinterpret_cast<const uint32_t*>(iks + e * 4));
+    const uint4 c0 = __ldg(reinterpret_cast<const uint4*>(ik + ik_code_off(e, 0)));
+    const uint4 c1 = __ldg(reinterpret_cast<const uint4*>(ik + ik_code_off(e, 1)));
+    const uint32_t sw = __ldg(reinterpret_cast<const uint32_t*>(iks + ik_scale_off(e)));
     return entry_score(R, c0, c1, sw);
 }
 
@@ -165,12 +165,7 @@ __global__ void __launch_bounds__(kNT, 2) select_kernel(SelectParams p) {
             if (v0) s0 = entry_score_at(R, ik, iks, e0);
             if (v1) s1 = entry_score_at(R, ik, iks, e1);
             if (bm) {
-                float m0 = s0, m1 = s1;
-#pragma unroll
-                for (int o = 1; o < 8; o <<= 1) {
-                    m0 = fmaxf(m0, __shfl_xor_sync(0xFFFFFFFFu, m0, o));
-                    m1 = fmaxf(m1, __shfl_xor_sync(0xFFFFFFFFu, m1, o));
-                }
+                const float m0 = block_max8(s0, tid & 31), m1 = block_max8(s1, tid & 31);
                 if ((tid & 7) == 0) {
                     if (v0) bm[e0 >> 3] = m0;
                     if (v1) bm[e1 >> 3] = m1;

@@ -3,9 +3,8 @@
 // over the whole cluster, no merge and no sort.
 //
 // Each CTA scores a contiguous 1/C of the query's visible entries with the
-// tcgen05 pipeline of index_pipe.cuh (permuted tiles: TMEM row m of a tile is
-// entry 4 (m % 32) + m / 32, so a stage is one TMA box per tile plus one bulk
-// copy of its scales; 8 stages in flight) and keeps every order key in TMEM
+// tcgen05 pipeline of index_pipe.cuh (a stage is one bulk copy of four tiles'
+// codes and one of their scales; 8 stages in flight) and keeps every order key in TMEM
 // (lane m, one column per tile: up to 32,768 keys beside the pipeline's 256
 // columns), while the epilogue counts the keys' top 11 bits into a 2,048-bin
 // histogram.  The cluster then finds the K-th largest key T exactly in three
@@ -31,7 +30,7 @@ namespace {
 
 using namespace pipe;
 
-constexpr int kThreads = 320;              // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+constexpr int kThreads = 320;              // warp 0 copies, warp 1 MMA, warps 2-9 epilogue
 constexpr int kEpiN = 256;
 constexpr int kTPG = kTPS / 2;             // tiles of a stage per epilogue warp group
 constexpr int kRing = 8;                   // shared-memory stages in flight
@@ -49,7 +48,6 @@ static_assert(kTmemCols == 512, "TMEM");
 struct ClSmem {
     ClPipe pipe;                            // its A ring holds hist2, hist3 and two bitmaps after scoring
     alignas(16) uint32_t hist1[kNB1];
-    float bmx[2][2][kTPG][kTile];           // block-max staging: [group][stage parity][tile][entry in tile]
     uint32_t wsum[kSelWarps];               // scan: per-warp totals
     uint32_t res[2];                        // find_bin: (bin, keys above the bin)
     uint32_t wcnt[8][2];                    // per sweeping warp: keys > T, keys == T
@@ -64,10 +62,6 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
         if (lane >= o) v += y;
     }
     return v;
-}
-
-__device__ __forceinline__ void group_bar(int group) {
-    asm volatile("bar.sync %0, 128;" ::"r"(2 + group) : "memory");
 }
 
 // Exclusive prefix of v over threads 0..255 in thread order (threads 256+ pass
@@ -157,7 +151,7 @@ __device__ __forceinline__ void find_bin(ClSmem& s, const uint32_t* hist, uint32
 // Visit every stored key of this CTA, 32 tile columns at a time: warps 2-9,
 // TMEM lane quarter q = warp % 4, columns [128 h, 128 h + 128) with
 // h = (warp - 2) / 4.  f(v, c0, q) gets the keys of columns c0 .. c0 + 31 of
-// this lane; column c of lane l holds CTA-local entry 128 c + 4 l + q.
+// this lane; column c of lane l holds CTA-local entry 128 c + 32 q + l.
 template <class F>
 __device__ __forceinline__ void sweep_cols(uint32_t tbase, int warp, int ntiles, F&& f) {
     if (warp < 2) return;
@@ -172,7 +166,7 @@ __device__ __forceinline__ void sweep_cols(uint32_t tbase, int warp, int ntiles,
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    index_cluster_kernel(SelectParams p, const __grid_constant__ CUtensorMap tmap) {
+    index_cluster_kernel(SelectParams p) {
     pdl_enter();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     ClSmem& s = *reinterpret_cast<ClSmem*>(smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u));
@@ -191,21 +185,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     int32_t* status = p.status;
     int32_t* out = p.out + (int64_t)bq * k;
 
-    if (tid == 0) init_barriers(s.pipe, 1, kEpiN);
+    if (tid == 0) init_barriers(s.pipe, kEpiN);
     if (warp == 1) setup_query(s.pipe, p.q + (int64_t)bq * 128, p.q_sc + (int64_t)bq * 16, lane, kTmemCols);
     for (int i = tid; i < kNB1; i += kThreads) s.hist1[i] = 0;
     __syncthreads();
     const uint32_t tbase = s.pipe.tmem_base;
 
     if (warp == 0) {
-        producer_perm(s.pipe, &tmap, p.ik_sc, row_base, lo, hi, ntiles, nstages, status, lane);
+        producer_dense(s.pipe, p.ik, p.ik_sc, row_base, lo, ntiles, nstages, status, lane);
     } else if (warp == 1) {
         mma_issuer(s.pipe, ntiles, nstages, status, lane);
     } else {
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;             // TMEM lanes this warp may read
         const int group = (warp - 2) >> 2;        // tiles 2*group, 2*group+1 of each stage
-        const int eo = 4 * lane + quarter;        // entry of this thread's TMEM row within a tile
+        const int eo = quarter * 32 + lane;       // this thread's TMEM row = its entry within a tile
         const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
         const float w0 = __ldg(p.w + (int64_t)bq * 4 + 0), w1 = __ldg(p.w + (int64_t)bq * 4 + 1);
         const float w2 = __ldg(p.w + (int64_t)bq * 4 + 2), w3 = __ldg(p.w + (int64_t)bq * 4 + 3);
@@ -228,35 +222,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::tmem_ld_wait();
                 tc::tc_fence_before();
                 tc::mbar_arrive(&s.pipe.accempty[a]);
+                if (!__all_sync(0xFFFFFFFFu, stage_landed(s.pipe, t))) {   // warp-uniform
+                    if (lane == 0) raise_abort(s.pipe, status);
+                    dead = true;
+                    continue;
+                }
+                uint32_t skw[kTPG];
+#pragma unroll
+                for (int j = 0; j < kTPG; ++j) skw[j] = stage_scales(s.pipe, t % kRing, kTPG * group + j, eo);
+                release_stage(s.pipe, t, lane);
                 const int g0 = t * kTPS + kTPG * group;
                 uint32_t key[kTPG];
 #pragma unroll
                 for (int j = 0; j < kTPG; ++j) {
                     const int g = g0 + j;
                     const bool valid = g < ntiles && lo + g * kTile + eo < hi;
-                    const float score = valid ? score_of(v[j], w0, w1, w2, w3) : -INFINITY;
+                    const float score = valid ? score_of(v[j], skw[j], w0, w1, w2, w3) : -INFINITY;
                     key[j] = valid ? score_key(score) : 0u;
                     if (valid) atomicAdd(&s.hist1[key[j] >> 21], 1u);
-                    if (bm) s.bmx[group][t & 1][j][eo] = score;
+                    if (bm) {
+                        const float mx = block_max8(score, lane);
+                        if ((lane & (kBlk - 1)) == 0 && valid) bm[(lo + g * kTile + eo) >> 3] = mx;
+                    }
                 }
                 if (g0 + 1 < ntiles) tc::tmem_st_32x32b_x2(tbase + lanes + kColKeys + (uint32_t)g0, key[0], key[1]);
                 else if (g0 < ntiles) tc::tmem_st_32x32b_x1(tbase + lanes + kColKeys + (uint32_t)g0, key[0]);
-            }
-            if (bm) {
-                // block maxima in position order: the first strictly larger score wins
-                group_bar(group);
-                if (!dead && warp == 2 + 4 * group) {   // one warp of the group
-                    const int j = lane >> 4, c = lane & 15;
-                    const int g = t * kTPS + kTPG * group + j;
-                    const int e0 = lo + g * kTile + 8 * c;
-                    if (g < ntiles && e0 < hi) {
-                        const float* sc = &s.bmx[group][t & 1][j][8 * c];
-                        float mx = sc[0];
-                        for (int e = 1; e < kBlk && e0 + e < hi; ++e)
-                            if (sc[e] > mx) mx = sc[e];
-                        bm[e0 >> 3] = mx;
-                    }
-                }
             }
         }
         tc::tmem_st_wait();
@@ -323,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---------------------------------------------------------------- output
     // keys > T and == T: counted, and marked in position bitmaps (column c of lane l
-    // is entry 128 c + 4 l + q: bitmap word 4 c + l / 8, bit 4 (l % 8) + q)
+    // is entry 128 c + 32 q + l: bitmap word 4 c + q, bit l)
     uint32_t gt = 0, eq = 0;
     sweep_cols(tbase, warp, ntiles, [&](const uint32_t(&v)[32], int c0, int q) {
         uint32_t mg = 0, me = 0;
@@ -335,8 +325,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         gt += __popc(mg);
         eq += __popc(me);
-        const uint32_t bit = 1u << (4 * (lane & 7) + q);
-        const int w0 = 4 * c0 + (lane >> 3);
+        const uint32_t bit = 1u << lane;
+        const int w0 = 4 * c0 + q;
         while (mg != 0u) {
             const int j = __ffs(mg) - 1;
             mg &= mg - 1u;
@@ -483,8 +473,7 @@ bool set_attributes() {
 
 int index_cluster_size(const SelectParams& p) {
     const int bq = p.B * p.Q;
-    // permuted tiles: rows in groups of 4, 16-byte aligned scale rows
-    if (bq <= 0 || (p.cap & 3) != 0 || (((uintptr_t)p.ik_sc) & 15u) != 0 || !set_attributes()) return 0;
+    if (bq <= 0 || !set_attributes()) return 0;
     for (int C = g_nonportable ? 16 : 8; C >= 1; C >>= 1) {
         if ((int64_t)bq * C > kNumSMs) continue;
         const int64_t chunk = ((p.cap + C - 1) / C + kTile - 1) / kTile * kTile;
@@ -495,10 +484,8 @@ int index_cluster_size(const SelectParams& p) {
 }
 
 cudaError_t launch_index_cluster(SelectParams& p, int C, cudaStream_t st) {
-    CUtensorMap map;
-    if (!pipe::encode_ik_map_perm(&map, p.ik, (int64_t)p.B * p.cap)) return cudaErrorInvalidValue;
     if (!set_attributes()) return cudaErrorInvalidValue;
-    return launch_ex(index_cluster_kernel, dim3(C, p.B * p.Q), dim3(kThreads), smem_bytes(), st, C, p, map);
+    return launch_ex(index_cluster_kernel, dim3(C, p.B * p.Q), dim3(kThreads), smem_bytes(), st, C, p);
 }
 
 }  // namespace csa2

@@ -18,9 +18,11 @@ constexpr int kEpiT0 = 64, kEpiN = 256;   // 8 epilogue warps: two per TMEM lane
 constexpr int kThreads = kEpiT0 + kEpiN;
 constexpr int kTPG = kTPS / 2;   // tiles of a stage per epilogue warp group
 
+constexpr int kRing = 4;   // shared-memory stages in flight
+
 template <int CAP>
 struct TcSmem {
-    Pipe<4> pipe;
+    Pipe<kRing> pipe;
     int last;
     typename TopK<kEpiN, CAP, 1, kEpiT0>::Smem topk;
 };
@@ -39,7 +41,7 @@ __device__ __forceinline__ bool epilogue_any(bool v) {
 
 template <int MODE, int CAP>  // MODE 0 = dense range (index Top-K), 1 = pool blocks (pool Top-K)
 __global__ void __launch_bounds__(kThreads, 2)
-    index_tc_kernel(SelectParams p, const __grid_constant__ CUtensorMap tmap) {
+    index_tc_kernel(SelectParams p) {
     pdl_enter();
     using TKE = TopK<kEpiN, CAP, 1, kEpiT0>;
     using TcSmem = csa2::TcSmem<CAP>;
@@ -70,14 +72,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int nstages = (ntiles + kTPS - 1) / kTPS;
     const int32_t* pool = (MODE == 1) ? p.pool + (int64_t)bq * p.P : nullptr;
 
-    if (tid == 0) init_barriers(s.pipe, 1 + 32, kEpiN);
+    if (tid == 0) init_barriers(s.pipe, kEpiN);
     if (warp == 1) setup_query(s.pipe, p.q + (int64_t)bq * 128, p.q_sc + (int64_t)bq * 16, lane, kPipeCols);
     __syncthreads();
     const uint32_t tbase = s.pipe.tmem_base;
     int32_t* status = p.status;
 
     if (warp == 0) {
-        producer<MODE>(s.pipe, &tmap, p.ik_sc, row_base, lo, hi, ntiles, nstages, pool, nvis, status, lane);
+        if (MODE == 0) producer_dense(s.pipe, p.ik, p.ik_sc, row_base, lo, ntiles, nstages, status, lane);
+        else producer_pool(s.pipe, p.ik, p.ik_sc, row_base, lo, hi, ntiles, nstages, pool, nvis, status, lane);
     } else if (warp == 1) {
         mma_issuer(s.pipe, ntiles, nstages, status, lane);
     } else {
@@ -109,6 +112,12 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (ok) tc::tmem_ld_wait();
             tc::tc_fence_before();
             tc::mbar_arrive(&s.pipe.accempty[a]);
+            const bool landed = ok && __all_sync(0xFFFFFFFFu, stage_landed(s.pipe, t));   // warp-uniform
+            if (ok && !landed && lane == 0) raise_abort(s.pipe, status);
+            uint32_t skw[kTPG];
+#pragma unroll
+            for (int j = 0; j < kTPG; ++j) skw[j] = landed ? stage_scales(s.pipe, t % kRing, kTPG * group + j, row) : 0u;
+            if (landed) release_stage(s.pipe, t, lane);
             if (epilogue_any(aborted(s.pipe))) {   // also the barrier that orders the previous offers
                 stop = true;
                 break;
@@ -133,11 +142,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                 }
                 const bool valid = e >= 0;
-                const float score = valid ? score_of(v[j], w0, w1, w2, w3) : -INFINITY;
+                const float score = valid ? score_of(v[j], skw[j], w0, w1, w2, w3) : -INFINITY;
                 if (MODE == 0 && bm && g < ntiles) {
-                    float m8 = score;
-#pragma unroll
-                    for (int o = 1; o < 8; o <<= 1) m8 = fmaxf(m8, __shfl_xor_sync(0xFFFFFFFFu, m8, o));
+                    const float m8 = block_max8(score, lane);
                     if ((lane & 7) == 0 && valid) bm[e >> 3] = m8;
                 }
                 tk.offer(th, valid, score_key(valid ? score : 0.0f), (int32_t)(valid ? e : 0));
@@ -199,11 +206,12 @@ __global__ void __launch_bounds__(kThreads, 2)
 }  // namespace
 
 bool index_tc_supported(const SelectParams& p) {
-    return (((uintptr_t)p.ik) & 15u) == 0 && (int64_t)p.B * p.cap < (int64_t(1) << 31);
+    return (((uintptr_t)p.ik) & 15u) == 0 && (((uintptr_t)p.ik_sc) & 15u) == 0 && p.cap % kTile == 0 &&
+           (int64_t)p.B * p.cap < (int64_t(1) << 31);
 }
 
 template <int MODE, int CAP>
-cudaError_t launch_tc(SelectParams& p, int S, cudaStream_t st, const CUtensorMap& map) {
+cudaError_t launch_tc(SelectParams& p, int S, cudaStream_t st) {
     const int smem = (int)sizeof(TcSmem<CAP>) + 1024;
     static bool attr = false;
     if (!attr) {
@@ -212,62 +220,14 @@ cudaError_t launch_tc(SelectParams& p, int S, cudaStream_t st, const CUtensorMap
         attr = true;
     }
     dim3 grid(S, p.B * p.Q);
-    return launch_ex(index_tc_kernel<MODE, CAP>, grid, dim3(kThreads), smem, st, 0, p, map);
+    return launch_ex(index_tc_kernel<MODE, CAP>, grid, dim3(kThreads), smem, st, 0, p);
 }
-
-namespace pipe {
-namespace {
-
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-    if (!encode) {
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-    }
-    return encode;
-}
-
-}  // namespace
-
-bool encode_ik_map(CUtensorMap* map, const uint8_t* ik, int64_t rows, int box_rows) {
-    PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
-    if (!encode) return false;
-    cuuint64_t dims[2] = {32, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {32};
-    cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, (void*)ik, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-bool encode_ik_map_perm(CUtensorMap* map, const uint8_t* ik, int64_t rows) {
-    PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
-    if (!encode) return false;
-    // x: the 32 bytes of a row; y: groups of 4 rows (stride 128 B); z: the row in the group (stride 32 B)
-    cuuint64_t dims[3] = {32, (cuuint64_t)(rows / 4), 4};
-    cuuint64_t strides[2] = {128, 32};
-    cuuint32_t box[3] = {32, 32, 4};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, (void*)ik, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-}  // namespace pipe
 
 cudaError_t launch_index_tc(int op, SelectParams& p, int S, cudaStream_t st) {
     const int mode = (op == CSA2_OP_POOL_TOPK) ? 1 : 0;
-    CUtensorMap map;
-    if (!pipe::encode_ik_map(&map, p.ik, (int64_t)p.B * p.cap, mode == 0 ? kTile : kBlk)) return cudaErrorInvalidValue;
     // the buffer must hold k survivors plus one stage of offers
-    if (p.k <= 2048 - kTPS * kTile) return mode == 0 ? launch_tc<0, 2048>(p, S, st, map) : launch_tc<1, 2048>(p, S, st, map);
-    return mode == 0 ? launch_tc<0, 4096>(p, S, st, map) : launch_tc<1, 4096>(p, S, st, map);
+    if (p.k <= 2048 - kTPS * kTile) return mode == 0 ? launch_tc<0, 2048>(p, S, st) : launch_tc<1, 2048>(p, S, st);
+    return mode == 0 ? launch_tc<0, 4096>(p, S, st) : launch_tc<1, 4096>(p, S, st);
 }
 
 }  // namespace csa2

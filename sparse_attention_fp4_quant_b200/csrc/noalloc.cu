@@ -51,7 +51,8 @@ csa2_status csa2_index_topk_noalloc(const uint8_t* q, const uint8_t* q_sc, const
     if (B < 1 || Q < 1 || (int64_t)B * Q > 65535 || k < 1 || k > CSA2_MAX_K) return CSA2_ERR_INVALID_ARG;
     if (!q || !q_sc || !w || !q_pos || !idx_out || !kv || !kv->ik || !kv->ik_sc || !kv->n_entries) return CSA2_ERR_INVALID_ARG;
     if (kv->cap < 1 || (kv->m != 1 && kv->m != 2) || kv->cap > (int64_t(1) << 31) / 8) return CSA2_ERR_INVALID_ARG;
-    if (((uintptr_t)q & 15u) || ((uintptr_t)kv->ik & 15u) || ((uintptr_t)kv->ik_sc & 15u)) return CSA2_ERR_INVALID_ARG;
+    if (((uintptr_t)q & 15u) || ((uintptr_t)kv->ik & 15u) || ((uintptr_t)kv->ik_sc & 15u) || kv->cap % 128 != 0)
+        return CSA2_ERR_INVALID_ARG;
     if (((uintptr_t)q_sc & 3u) || ((uintptr_t)w & 3u)) return CSA2_ERR_INVALID_ARG;
     const size_t need = select_ws_bytes(CSA2_OP_INDEX_TOPK, B, Q, kv->cap, k, 0);
     if (need > kScratchBytes) return CSA2_ERR_WORKSPACE;

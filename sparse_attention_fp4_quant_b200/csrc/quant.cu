@@ -139,8 +139,8 @@ __global__ void __launch_bounds__(256) index_k_proj_kernel(const uint16_t* __res
         quant16(v, sc, lo, hi);
         int64_t orow = dst_rows ? __ldg(dst_rows + row) : row;
         if (orow >= 0 && orow < out_rows) {
-            *reinterpret_cast<uint2*>(kc + orow * 32 + 8 * g) = make_uint2(lo, hi);
-            ks[orow * 4 + g] = (uint8_t)sc;
+            *reinterpret_cast<uint2*>(kc + ik_code_off(orow, g >> 1) + 8 * (g & 1)) = make_uint2(lo, hi);
+            ks[ik_scale_off(orow) + g] = (uint8_t)sc;
         }
     }
 }
@@ -191,8 +191,8 @@ __global__ void __launch_bounds__(256) index_k_proj_rows_kernel(const uint16_t* 
             quant16(v, sc, lo, hi);
             const int64_t orow = dst_rows ? __ldg(dst_rows + row2) : row2;
             if (orow >= 0 && orow < out_rows) {
-                *reinterpret_cast<uint2*>(kc + orow * 32 + 8 * g) = make_uint2(lo, hi);
-                ks[orow * 4 + g] = (uint8_t)sc;
+                *reinterpret_cast<uint2*>(kc + ik_code_off(orow, g >> 1) + 8 * (g & 1)) = make_uint2(lo, hi);
+                ks[ik_scale_off(orow) + g] = (uint8_t)sc;
             }
         }
     }
@@ -277,8 +277,8 @@ __global__ void __launch_bounds__(kAppThreads) append_kernel(const uint16_t* __r
         quant16(v, sc, lo, hi);
         const int64_t orow = dst_rows ? __ldg(dst_rows + r0 + tid) : r0 + tid;
         if (orow >= 0 && orow < out_rows) {
-            *reinterpret_cast<uint2*>(kc + orow * 32 + 8 * cb) = make_uint2(lo, hi);
-            ks[orow * 4 + cb] = (uint8_t)sc;
+            *reinterpret_cast<uint2*>(kc + ik_code_off(orow, cb >> 1) + 8 * (cb & 1)) = make_uint2(lo, hi);
+            ks[ik_scale_off(orow) + cb] = (uint8_t)sc;
         }
     }
 }

@@ -33,6 +33,33 @@ def attn_close(gpu_bf16, ref):
     return bool(ok.all()), stats
 
 
+def ik_untile(codes, scales):
+    """Row-major [n, 32] codes and [n, 4] scales from the indexer-K cache order (any
+    leading shape with a multiple of 128 entries).  In a 128-entry tile, half h of
+    entry e's codes sits at 256 (e // 8 % 16) + 128 h + 16 (e % 8); scales are row-major."""
+    c = np.asarray(codes).reshape(-1, 16, 2, 8, 16).transpose(0, 1, 3, 2, 4).reshape(-1, 32)
+    return c, np.asarray(scales).reshape(-1, 4)
+
+
+def ik_tile(codes, scales):
+    """Inverse of ik_untile: row-major indexer K -> the cache order (flat bytes)."""
+    c = np.ascontiguousarray(np.asarray(codes).reshape(-1, 16, 8, 2, 16).transpose(0, 1, 3, 2, 4)).reshape(-1)
+    return c, np.ascontiguousarray(np.asarray(scales)).reshape(-1)
+
+
+def kv_ik_rows(kv):
+    """The device cache's indexer K as row-major numpy [B, cap, 32] / [B, cap, 4]."""
+    c, s = ik_untile(np_(kv.ik), np_(kv.ik_sc))
+    return c.reshape(kv.B, kv.cap, 32), s.reshape(kv.B, kv.cap, 4)
+
+
+def set_kv_ik_rows(kv, codes, scales):
+    """Write row-major indexer K [B, cap, 32] / [B, cap, 4] into the device cache's tiled order."""
+    c, s = ik_tile(codes, scales)
+    kv.ik.copy_(torch.from_numpy(c).view(kv.B, kv.cap, 32))
+    kv.ik_sc.copy_(torch.from_numpy(s).view(kv.B, kv.cap, 4))
+
+
 class Group:
     """A CSA2 layer group: bf16 latent rows (generator), the oracle's quantised
     cache (numpy) and the CUDA path's own quantised cache (device)."""

@@ -61,10 +61,17 @@ def test_invalid_arguments_rejected_before_launch(L):
     # projection matrix not 16-byte aligned
     assert L.csa2_index_k_proj(fake, 4, P(0x1004), fake, fake, None, 4, None) == 1
     import sparse_attention_fp4_quant_b200 as csa
-    kv = csa.csa2_kv(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 100, 3)  # m = 3 is invalid
+    # indexer-K output rows that are not whole 128-entry tiles
+    assert L.csa2_index_k_proj(fake, 4, fake, fake, fake, None, 100, None) == 1
+    assert L.csa2_append_tokens(fake, 4, fake, fake, fake, fake, fake, None, 100, None) == 1
+    kv = csa.csa2_kv(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 128, 3)  # m = 3 is invalid
     assert L.csa2_index_topk(fake, fake, fake, ctypes.byref(kv), fake, 1, 1, 512, fake, None, fake, 1 << 20,
                              None) == 1
     kv.m = 1
+    kv.cap = 1000   # not whole tiles of the indexer-K order
+    assert L.csa2_index_topk(fake, fake, fake, ctypes.byref(kv), fake, 1, 1, 512, fake, None, fake, 1 << 20,
+                             None) == 1
+    kv.cap = 128
     assert L.csa2_index_topk(fake, fake, fake, ctypes.byref(kv), fake, 1, 1, 4096, fake, None, fake, 1 << 20,
                              None) == 1   # k > CSA2_MAX_K
     assert L.csa2_index_topk(fake, fake, fake, ctypes.byref(kv), fake, 1, 1, 512, fake, None, fake, 0,

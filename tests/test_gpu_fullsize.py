@@ -216,7 +216,7 @@ def test_c4_replay_and_decoder_step(csa):
     """B=4, 262,144 entries: SWA Bounded Replay of the last 128 tokens (s = ctx - 128) through a
     Full layer, then one decode step through the 20-layer decoder pattern with the append."""
     B, n = 4, 262144
-    grp = BigGroup(csa, 140, B, n + 8, [n] * B, keep=(2,))
+    grp = BigGroup(csa, 140, B, n + 128, [n] * B, keep=(2,))
     s = n - 128
     Q = 128
     # ---- replay: 128 queries per batch row at tokens s .. n-1, Full layer

@@ -9,7 +9,8 @@ import torch
 
 import oracle
 import synth
-from gpu_common import SM_SCALE, Group, attn_close, bits, index_query, np_, swa_for
+from gpu_common import (SM_SCALE, Group, attn_close, bits, ik_untile, index_query, kv_ik_rows, np_, set_kv_ik_rows,
+                        swa_for)
 
 pytestmark = pytest.mark.gpu
 
@@ -76,14 +77,19 @@ def test_quant_latents_and_dst_rows(csa, ch):
 def test_index_k_proj_bit_exact(csa):
     x = synth.latent(5, 1000, 0, "cuda")
     W = synth.proj_w(3).cuda()
-    kc, ks = csa.csa2_index_k_proj(x, W)
+    kc, ks = csa.csa2_index_k_proj(x, W)   # 1024 rows: whole tiles of the cache order
+    assert kc.shape == (1024, 32)
     oc, os_ = oracle.index_k_proj(bits(x), np_(W))
-    assert np.array_equal(np_(kc), oc) and np.array_equal(np_(ks), os_)
+    gc, gs = ik_untile(np_(kc), np_(ks))
+    assert np.array_equal(gc[:1000], oc) and np.array_equal(gs[:1000], os_)
     dst = (torch.arange(1000, device="cuda", dtype=torch.int64) * 3 + 1)
-    bc = torch.zeros((3001, 32), dtype=torch.uint8, device="cuda")
-    bs = torch.zeros((3001, 4), dtype=torch.uint8, device="cuda")
+    bc = torch.zeros((3072, 32), dtype=torch.uint8, device="cuda")
+    bs = torch.zeros((3072, 4), dtype=torch.uint8, device="cuda")
     csa.csa2_index_k_proj(x, W, bc, bs, dst)
-    assert np.array_equal(np_(bc)[1::3][:1000], oc) and np.array_equal(np_(bs)[1::3][:1000], os_)
+    gc, gs = ik_untile(np_(bc), np_(bs))
+    assert np.array_equal(gc[1::3][:1000], oc) and np.array_equal(gs[1::3][:1000], os_)
+    with pytest.raises(RuntimeError):   # output rows must be whole tiles
+        csa.csa2_index_k_proj(x, W, bc[:3001], bs[:3001], dst)
 
 
 @pytest.mark.parametrize("rows", [1, 32, 45, 2049])
@@ -94,7 +100,7 @@ def test_append_tokens_bit_exact(csa, rows):
     lb = bits(x)
     olc, ols = oracle.quant_nvfp4(lb)
     okc, oks = oracle.index_k_proj(lb, np_(W))
-    out_rows = 3 * rows + 1
+    out_rows = (3 * rows + 1 + 127) // 128 * 128   # whole tiles of the indexer-K order
     dst = torch.arange(rows, device="cuda", dtype=torch.int64) * 3 + 1
     lc = torch.zeros((out_rows, 256), dtype=torch.uint8, device="cuda")
     ls = torch.zeros((out_rows, 32), dtype=torch.uint8, device="cuda")
@@ -102,17 +108,19 @@ def test_append_tokens_bit_exact(csa, rows):
     ks = torch.zeros((out_rows, 4), dtype=torch.uint8, device="cuda")
     csa.csa2_append_tokens(x, W, (lc, ls, kc, ks), dst)
     assert np.array_equal(np_(lc)[1::3][:rows], olc) and np.array_equal(np_(ls)[1::3][:rows], ols)
-    assert np.array_equal(np_(kc)[1::3][:rows], okc) and np.array_equal(np_(ks)[1::3][:rows], oks)
+    gkc, gks = ik_untile(np_(kc), np_(ks))
+    assert np.array_equal(gkc[1::3][:rows], okc) and np.array_equal(gks[1::3][:rows], oks)
     untouched = np.ones(out_rows, bool)
     untouched[1::3][:rows] = False
-    assert not np_(lc)[untouched].any() and not np_(kc)[untouched].any()
+    assert not np_(lc)[untouched].any() and not gkc[untouched].any() and not gks[untouched].any()
 
 
 # ---------------------------------------------------------------- index / Top-K
 def _index_case(seed, B, Q, cap, n_entries, m, q_pos, k):
     grp = Group(seed, B, cap, n_entries, m)
     o = grp.oracle_cache()
-    assert np.array_equal(np_(grp.kv.ik), o["ik"]) and np.array_equal(np_(grp.kv.ik_sc), o["iks"])
+    gik, giks = kv_ik_rows(grp.kv)
+    assert np.array_equal(gik, o["ik"]) and np.array_equal(giks, o["iks"])
     iq, iqs, w, oiq, oiqs, ow = index_query(seed + 1, B, Q)
     assert np.array_equal(np_(iq), oiq) and np.array_equal(np_(iqs), oiqs)
     qp = torch.tensor(q_pos, dtype=torch.int32, device="cuda")
@@ -122,7 +130,7 @@ def _index_case(seed, B, Q, cap, n_entries, m, q_pos, k):
 @pytest.mark.parametrize("m", [1, 2])
 @pytest.mark.parametrize("k", [1, 37, 512, 2048])
 def test_index_topk_ragged(csa, m, k):
-    B, Q, cap = 3, 2, 9000
+    B, Q, cap = 3, 2, 9088
     n_entries = [9000, 4097, 1]
     q_pos = [[9000 * m - 1, 3000], [4096 * m + 50, 511], [0, 77]]
     grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(11 * m + k, B, Q, cap, n_entries, m, q_pos, k)
@@ -136,7 +144,7 @@ def test_index_topk_ragged(csa, m, k):
 def test_index_topk_many_queries(csa):
     # 160 queries: more than one cluster per query can hold at once, so the
     # streaming per-share kernel serves them (prefill-like causal positions)
-    B, Q, cap, m, k = 2, 80, 3000, 2, 512
+    B, Q, cap, m, k = 2, 80, 3072, 2, 512
     n_entries = [3000, 2100]
     rng = np.random.default_rng(5)
     q_pos = rng.integers(0, 6000, size=(B, Q)).astype(np.int32)
@@ -147,15 +155,16 @@ def test_index_topk_many_queries(csa):
     assert np.array_equal(np_(idx), ridx)
 
 
-@pytest.mark.parametrize("cap", [1001, 1002, 1004])
-def test_index_topk_capacity_not_multiple_of_4(csa, cap):
-    # rows of the cache that are not a whole number of 4-row groups take the
-    # per-share kernel; multiples of 4 take the cluster kernel
+@pytest.mark.parametrize("n", [128, 129, 255, 1001])
+def test_index_topk_small_ragged_caches(csa, n):
+    # visible ranges of a tile, just over one, one short of two, and ragged: the
+    # cluster kernel's last tile and the per-share kernel's last stage
     B, Q, m = 2, 1, 1
-    n_entries = [cap, cap - 3]
-    q_pos = [[cap - 1], [cap - 4]]
+    cap = (n + 127) // 128 * 128
+    n_entries = [n, max(1, n - 3)]
+    q_pos = [[n - 1], [n - 4]]
     for k in (64, 512):
-        grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(90 + cap % 7, B, Q, cap, n_entries, m, q_pos, k)
+        grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(90 + n % 7, B, Q, cap, n_entries, m, q_pos, k)
         idx, bm = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, k, blockmax=True)
         ridx, rbm = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, m, np.array(q_pos, np.int32),
                                       k, blockmax=True)
@@ -163,10 +172,15 @@ def test_index_topk_capacity_not_multiple_of_4(csa, cap):
         assert np.array_equal(np_(bm), rbm)
 
 
+def test_kv_capacity_must_be_whole_tiles(csa):
+    with pytest.raises(ValueError):
+        csa.KV(1, 1000, 1, "cuda")
+
+
 def test_index_blockmax_signed_zero_and_negative_weights(csa):
     # negative head weights make scores <= 0, with -0 and +0 in the same block;
     # a block maximum keeps the first of equal values in position order
-    B, Q, cap, m, k = 1, 2, 4000, 1, 512
+    B, Q, cap, m, k = 1, 2, 4096, 1, 512
     q_pos = [[3999, 2500]]
     grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(95, B, Q, cap, [4000], m, q_pos, k)
     w = torch.tensor([[[-0.25, 0.5, -0.75, 0.125], [-1.0, -0.5, -0.25, -0.125]]], dtype=torch.float32, device="cuda")
@@ -188,7 +202,7 @@ def test_index_scores_extreme_block_scales(csa):
     extremes = np.array([0x01, 0x02, 0x08, 0x30, 0x40, 0x77, 0x7E], np.uint8)
     iks = extremes[rng.integers(0, len(extremes), size=(B, cap, 4))].astype(np.uint8)
     o["iks"] = iks
-    grp.kv.ik_sc.copy_(torch.from_numpy(iks))
+    set_kv_ik_rows(grp.kv, o["ik"], iks)
     iq, iqs, w, oiq, oiqs, ow = index_query(19, B, Q)
     qsc = extremes[rng.integers(0, len(extremes), size=(B, Q, 16))].astype(np.uint8)
     oiqs = qsc
@@ -201,11 +215,13 @@ def test_index_scores_extreme_block_scales(csa):
 
 
 def test_index_topk_ties_and_zero_scores(csa):
-    B, Q, cap = 1, 3, 20000
+    B, Q, cap = 1, 3, 20096
     grp = Group(21, B, cap, [20000])
     # duplicate one key everywhere in a stripe: many exactly equal scores
-    grp.kv.ik[0, 1000:9000] = grp.kv.ik[0, 5]
-    grp.kv.ik_sc[0, 1000:9000] = grp.kv.ik_sc[0, 5]
+    gik, giks = kv_ik_rows(grp.kv)
+    gik[0, 1000:9000] = gik[0, 5]
+    giks[0, 1000:9000] = giks[0, 5]
+    set_kv_ik_rows(grp.kv, gik, giks)
     o = grp.oracle_cache()
     o = dict(o)
     o["ik"] = o["ik"].copy()
@@ -225,7 +241,7 @@ def test_index_topk_ties_and_zero_scores(csa):
 
 
 def test_device_error_flag_stays_clear(csa):
-    B, Q, cap, k = 2, 1, 3000, 64
+    B, Q, cap, k = 2, 1, 3072, 64
     grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(31, B, Q, cap, [3000, 2000], 1, [[2999], [1999]], k)
     ws = torch.zeros(csa.csa2_workspace_bytes(csa.OP_INDEX_TOPK, B, Q, cap, k), dtype=torch.uint8, device="cuda")
     idx = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, k, ws=ws)
@@ -237,7 +253,7 @@ def test_device_error_flag_stays_clear(csa):
 
 
 def test_binding_rejects_mismatched_shapes(csa):
-    kv = csa.KV(1, 64, 1, "cuda")
+    kv = csa.KV(1, 128, 1, "cuda")
     q = torch.zeros((2, 1, 128), dtype=torch.uint8, device="cuda")
     qs = torch.zeros((2, 1, 16), dtype=torch.uint8, device="cuda")
     w = torch.zeros((2, 1, 4), dtype=torch.float32, device="cuda")
@@ -250,7 +266,7 @@ def test_binding_rejects_mismatched_shapes(csa):
 
 # ---------------------------------------------------------------- pool
 def test_pool_build_and_pool_topk(csa):
-    B, Q, cap = 2, 2, 30000
+    B, Q, cap = 2, 2, 30080
     n_entries = [30000, 17001]
     q_pos = [[29999, 20000], [17000, 9]]
     grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(31, B, Q, cap, n_entries, 1, q_pos, 512)
@@ -295,7 +311,7 @@ def _attn_case(csa, seed, B, Q, cap, n_entries, k, T, window, q_pos, pos0, repla
 
 @pytest.mark.parametrize("B,Q", [(1, 1), (3, 2), (32, 1)])
 def test_sparse_attn_decode(csa, B, Q):
-    cap, k, T = 5000, 512, 128
+    cap, k, T = 5120, 512, 128
     rng = np.random.default_rng(B * 10 + Q)
     n_entries = [5000 - 7 * b for b in range(B)]
     idx = np.sort(rng.integers(0, 4990, (B, Q, k)), axis=-1).astype(np.int32)
@@ -308,7 +324,7 @@ def test_sparse_attn_decode(csa, B, Q):
 @pytest.mark.parametrize("window", [1, 2, 4, 77, 128])
 @pytest.mark.parametrize("Q", [8, 128])   # 16 queries: one cluster each; 256: split-K kernel
 def test_sparse_attn_replay_mask(csa, window, Q):
-    B, cap, k, T = 2, 3000, 64, 128
+    B, cap, k, T = 2, 3072, 64, 128
     rng = np.random.default_rng(window + Q)
     s = [3000 - 128, 2500]
     q_pos = [[s[b] + qi for qi in range(Q)] for b in range(B)]
@@ -318,7 +334,7 @@ def test_sparse_attn_replay_mask(csa, window, Q):
 
 
 def test_sparse_attn_edge_cases(csa):
-    B, Q, cap = 2, 3, 600
+    B, Q, cap = 2, 3, 640
     # k = 0 (SWA only); T = 0 (main only); query with nothing visible -> zeros
     rng = np.random.default_rng(7)
     idx = np.full((B, Q, 0), -1, np.int32)
@@ -333,7 +349,7 @@ def test_sparse_attn_edge_cases(csa):
 def test_layer_dispatch_decoder_pattern(csa):
     """The decoder pattern F R R R (X R R R) x 4 through csa2_layer_step equals the
     oracle's layer composition (bit-exact indices; attention within tolerance)."""
-    B, Q, cap, T = 2, 1, 6000, 128
+    B, Q, cap, T = 2, 1, 6016, 128
     n_before = [5000, 4321]
     grp = Group(70, B, cap, n_before)
     o = {kk: v.copy() for kk, v in grp.oracle_cache().items()}
@@ -373,7 +389,7 @@ def test_layer_dispatch_decoder_pattern(csa):
                      window=128, q_pos=q_pos_np)
         ref, _ = oracle.layer_step(mode, st, layer)
         if first:
-            assert np.array_equal(np_(grp.kv.lat), o["lat"]) and np.array_equal(np_(grp.kv.ik), o["ik"])
+            assert np.array_equal(np_(grp.kv.lat), o["lat"]) and np.array_equal(kv_ik_rows(grp.kv)[0], o["ik"])
             assert np.array_equal(np_(pool), st["pool"])
         assert np.array_equal(np_(idx), st["idx"]), (li, mode)
         ok, stats = attn_close(out, ref)

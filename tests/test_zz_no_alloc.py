@@ -28,7 +28,7 @@ def _case(seed, B, Q, cap):
 
 
 def test_noalloc_matches_workspace_call_twice():
-    csa, kv, iq, iqs, w, q_pos = _case(5, 4, 2, 40000)
+    csa, kv, iq, iqs, w, q_pos = _case(5, 4, 2, 40064)
     assert "csa2_index_topk_noalloc" in csa.EXPORTS
     for k in (512, 2048):
         ref, ref_bm = csa.csa2_index_topk(iq, iqs, w, kv, q_pos, k, blockmax=True)
