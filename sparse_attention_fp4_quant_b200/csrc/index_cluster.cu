@@ -4,16 +4,19 @@
 //
 // Each CTA scores a contiguous 1/C of the query's visible entries with the
 // tcgen05 pipeline of index_pipe.cuh (a stage is one bulk copy of four tiles'
-// codes and one of their scales; 8 stages in flight) and keeps every order key in TMEM
-// (lane m, one column per tile: up to 32,768 keys beside the pipeline's 256
-// columns), while the epilogue counts the keys' top 11 bits into a 2,048-bin
-// histogram.  The cluster then finds the K-th largest key T exactly in three
-// radix passes (bits 31..21, 20..10, 9..0): each pass sums the CTAs'
-// histograms through distributed shared memory and locates the bin holding
-// the K-th key from the top; passes 2 and 3 re-read the keys from TMEM.  The
-// selected set is every key above T plus the lowest-positioned keys equal to T
-// (ties go to the lower position).  A last read marks both kinds in position
-// bitmaps; CTA r covers positions below those of CTA r + 1, so its quota of
+// codes and one of their scales; 8 stages in flight) and keeps every order key
+// in TMEM (lane m, one column per tile: up to 32,768 keys beside the
+// pipeline's 256 columns), while the epilogue counts the keys' top 11 bits
+// into a 2,048-bin histogram.  The cluster sums the histograms through
+// distributed shared memory and finds the bin d1 holding the K-th largest key.
+// One read of the keys then marks every entry of a higher bin as selected
+// (position bitmaps) and lists the entries of bin d1, the candidates.  When the
+// cluster's candidates are few (the usual case) every CTA gathers all of them
+// and finds the K-th key T exactly with two local radix passes (bits 20..10,
+// 9..0); otherwise (many equal or close keys) two more passes over the keys in
+// TMEM find T with cluster-wide histograms.  The selected set is every key
+// above T plus the lowest-positioned keys equal to T (ties go to the lower
+// position).  CTA r covers positions below those of CTA r + 1, so its quota of
 // ties and its output offset follow from the lower-ranked CTAs' counts, and
 // two block-wide prefix sums over the bitmap words give every selected
 // position its place in the ascending output.
@@ -40,9 +43,13 @@ constexpr uint32_t kTmemCols = kPipeCols + kMaxTiles;
 constexpr int kWords = kMaxTiles * kTile / 32;          // bitmap words over the CTA's entries
 constexpr int kNB1 = 2048, kNB2 = 2048, kNB3 = 1024;   // radix digits: bits 31..21, 20..10, 9..0
 constexpr int kSel = 256;                  // threads of the scans (warps 0-7)
+constexpr int kCandCap = 4096;             // candidates (keys of the threshold's top bin) a CTA lists
+constexpr int kGatherCap = 8192;           // candidates of a cluster gathered for the local select
+constexpr uint32_t kSlowPath = 0xFFFFFFFFu;
 constexpr int kSelWarps = kSel / 32;
 using ClPipe = Pipe<kRing>;
-static_assert((kNB2 + kNB3 + 2 * kWords) * 4 <= (int)sizeof(ClPipe::A), "select scratch fits the ring");
+static_assert((kNB2 + kNB3 + 2 * kWords) * 4 + (kCandCap + kGatherCap) * 8 <= (int)sizeof(ClPipe::A),
+              "select scratch fits the ring");
 static_assert(kTmemCols == 512, "TMEM");
 
 struct ClSmem {
@@ -51,8 +58,13 @@ struct ClSmem {
     uint32_t wsum[kSelWarps];               // scan: per-warp totals
     uint32_t res[2];                        // find_bin: (bin, keys above the bin)
     uint32_t wcnt[8][2];                    // per sweeping warp: keys > T, keys == T
-    alignas(8) uint32_t pub[2];             // this CTA's (> T, == T) counts, read by the cluster
+    alignas(8) uint32_t pub[2];             // this CTA's (entries above bin d1, candidates), read by the cluster
+    alignas(8) uint32_t pub2[2];            // (> T, == T) counts of the multi-pass path, read by the cluster
     uint32_t cbase[2];                      // this CTA's tie quota and output offset
+    uint32_t ncand;                         // candidates appended (may exceed the list)
+    uint32_t fast;                          // candidates of the cluster, or kSlowPath
+    uint32_t peer[16][2];                   // per CTA: entries above bin d1, candidates of lower ranks
+    uint32_t rcnt[16][2];                   // per CTA: candidates above T, equal to T
 };
 
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
@@ -62,6 +74,21 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
         if (lane >= o) v += y;
     }
     return v;
+}
+
+// 32 x 32 bit transpose across the warp: in, bit j of lane l is element
+// (l, j); out, bit l of lane j is element (l, j).  Five block swaps of halving
+// size through shuffles.
+__device__ __forceinline__ uint32_t warp_transpose_bits(uint32_t x, int lane) {
+    constexpr uint32_t kMask[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+        const int sh = 16 >> i;
+        const uint32_t m = kMask[i];
+        const uint32_t y = __shfl_xor_sync(0xFFFFFFFFu, x, sh);
+        x = (lane & sh) ? ((x & ~m) | ((y >> sh) & m)) : ((x & m) | ((y << sh) & ~m));
+    }
+    return x;
 }
 
 // Exclusive prefix of v over threads 0..255 in thread order (threads 256+ pass
@@ -82,11 +109,13 @@ __device__ __forceinline__ uint32_t block_scan_excl(ClSmem& s, uint32_t v, int t
     return pre;
 }
 
-// Sum the NB-bin histogram `hist` over the cluster's CTAs and find the bin b
-// holding the R-th largest key (R >= 1): keys above b < R <= keys above b +
-// count of b.  Leaves (b, keys above b) in s.res.  All threads of the CTA call it.
+// Sum the NB-bin histogram `hist` over the CTAs r0 .. r0 + n - 1 of the
+// cluster (n = 1, r0 = own rank: this CTA's alone) and find the bin b holding
+// the R-th largest key (R >= 1): keys above b < R <= keys above b + count of b.
+// Leaves (b, keys above b) in s.res.  All threads of the CTA call it.
 template <int NB>
-__device__ __forceinline__ void find_bin(ClSmem& s, const uint32_t* hist, uint32_t C, uint32_t R, int tid) {
+__device__ __forceinline__ void find_bin(ClSmem& s, const uint32_t* hist, uint32_t r_first, uint32_t n, uint32_t R,
+                                         int tid) {
     constexpr int PER = NB / kSel;   // bins per thread, highest bins on thread 0
     constexpr int NV = PER / 4;      // 16-byte loads per CTA
     constexpr int RG = 4;            // CTAs whose loads are in flight together
@@ -98,18 +127,18 @@ __device__ __forceinline__ void find_bin(ClSmem& s, const uint32_t* hist, uint32
     const int b0 = NB - PER * (tid + 1);   // this thread's lowest bin
     if (tid < kSel) {
         const uint32_t la = tc::smem_u32(hist + b0);
-        for (uint32_t r0 = 0; r0 < C; r0 += RG) {
+        for (uint32_t r0 = 0; r0 < n; r0 += RG) {
             uint4 x[RG][NV];
 #pragma unroll
             for (int g = 0; g < RG; ++g)
-                if (r0 + g < C) {
-                    const uint32_t ra = cl::map_rank(la, r0 + g);
+                if (r0 + g < n) {
+                    const uint32_t ra = cl::map_rank(la, r_first + r0 + g);
 #pragma unroll
                     for (int v = 0; v < NV; ++v) x[g][v] = cl::ld_v4(ra + 16u * v);
                 }
 #pragma unroll
             for (int g = 0; g < RG; ++g)
-                if (r0 + g < C) {
+                if (r0 + g < n) {
 #pragma unroll
                     for (int v = 0; v < NV; ++v) {
                         h[4 * v + 0] += x[g][v].x;
@@ -276,105 +305,247 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* hist3 = hist2 + kNB2;
     uint32_t* selbm = hist3 + kNB3;   // entries above T (then also the ties taken)
     uint32_t* tiebm = selbm + kWords; // entries equal to T
+    uint2* cand = reinterpret_cast<uint2*>(tiebm + kWords);   // this CTA's keys of bin d1: (key, entry)
+    uint2* gath = cand + kCandCap;                             // the cluster's, gathered: (key, entry | rank << 16)
     for (int i = tid; i < kNB2 + kNB3 + 2 * kWords; i += kThreads) hist2[i] = 0;
+    if (tid < 32) s.rcnt[tid >> 1][tid & 1] = 0;
+    if (tid == 0) s.ncand = 0;
 
     cl::sync();                                   // every CTA's hist1 is complete
-    find_bin<kNB1>(s, s.hist1, C, K1, tid);
+    find_bin<kNB1>(s, s.hist1, 0, C, K1, tid);
     const uint32_t d1 = s.res[0];
-    uint32_t R = K1 - s.res[1];
-    sweep_cols(tbase, warp, ntiles, [&](const uint32_t(&v)[32], int c0, int) {
-        uint32_t m = 0;   // bit j: column c0 + j matches (independent compares, then a short loop)
-#pragma unroll
-        for (int j = 0; j < 32; ++j) m |= (uint32_t)(c0 + j < ntiles && (v[j] >> 21) == d1) << j;
-        while (m != 0u) {
-            const int j = __ffs(m) - 1;
-            m &= m - 1u;
-            atomicAdd(&hist2[(v[j] >> 10) & (kNB2 - 1)], 1u);
-        }
-    });
-    cl::sync();
-    find_bin<kNB2>(s, hist2, C, R, tid);
-    const uint32_t p2 = (d1 << 11) | s.res[0];
-    R -= s.res[1];
-    sweep_cols(tbase, warp, ntiles, [&](const uint32_t(&v)[32], int c0, int) {
-        uint32_t m = 0;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) m |= (uint32_t)(c0 + j < ntiles && (v[j] >> 10) == p2) << j;
-        while (m != 0u) {
-            const int j = __ffs(m) - 1;
-            m &= m - 1u;
-            atomicAdd(&hist3[v[j] & (kNB3 - 1)], 1u);
-        }
-    });
-    cl::sync();
-    find_bin<kNB3>(s, hist3, C, R, tid);
-    const uint32_t T = (p2 << 10) | s.res[0];
-    R -= s.res[1];   // ties at T still to take, lowest positions first (1 <= R)
+    const uint32_t R = K1 - s.res[1];             // keys still to take from bin d1 (1 <= R)
 
-    // ---------------------------------------------------------------- output
-    // keys > T and == T: counted, and marked in position bitmaps (column c of lane l
-    // is entry 128 c + 32 q + l: bitmap word 4 c + q, bit l)
-    uint32_t gt = 0, eq = 0;
+    // One read of the keys: an entry of a bin above d1 is selected whatever T
+    // is (marked in the bitmaps: one word per column and lane quarter, built by
+    // a bit transpose of the lanes' column masks); an entry of bin d1 is a
+    // candidate, appended to this CTA's list.
+    uint32_t above = 0;
     sweep_cols(tbase, warp, ntiles, [&](const uint32_t(&v)[32], int c0, int q) {
-        uint32_t mg = 0, me = 0;
+        uint32_t ma = 0, mc = 0;   // bit j: the key of column c0 + j is above bin d1 / in bin d1
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-            const bool valid = c0 + j < ntiles;
-            mg |= (uint32_t)(valid && v[j] > T) << j;
-            me |= (uint32_t)(valid && v[j] == T) << j;
+            const uint32_t bin = v[j] >> 21;
+            ma |= (uint32_t)(bin > d1) << j;
+            mc |= (uint32_t)(bin == d1) << j;
         }
-        gt += __popc(mg);
-        eq += __popc(me);
-        const uint32_t bit = 1u << lane;
-        const int w0 = 4 * c0 + q;
-        while (mg != 0u) {
-            const int j = __ffs(mg) - 1;
-            mg &= mg - 1u;
-            atomicOr(&selbm[w0 + 4 * j], bit);
+        if (ntiles - c0 < 32) {   // columns past the last tile hold no keys
+            const uint32_t cm = (1u << (ntiles - c0)) - 1u;
+            ma &= cm;
+            mc &= cm;
         }
-        while (me != 0u) {
-            const int j = __ffs(me) - 1;
-            me &= me - 1u;
-            atomicOr(&tiebm[w0 + 4 * j], bit);
+        const uint32_t word = warp_transpose_bits(ma, lane);   // column c0 + lane; bit l: lane l
+        if (c0 + lane < ntiles) selbm[4 * (c0 + lane) + q] = word;
+        above += __popc(word);
+        if (__any_sync(0xFFFFFFFFu, mc != 0u)) {
+            const uint32_t n = __popc(mc);
+            const uint32_t incl = warp_incl_scan(n, lane);
+            uint32_t base = 0;
+            if (lane == 31) base = atomicAdd(&s.ncand, incl);
+            uint32_t slot = __shfl_sync(0xFFFFFFFFu, base, 31) + incl - n;
+            const uint32_t e0 = 128u * (uint32_t)c0 + 32u * (uint32_t)q + (uint32_t)lane;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                if ((mc >> j) & 1u) {
+                    if (slot < (uint32_t)kCandCap) cand[slot] = make_uint2(v[j], e0 + 128u * (uint32_t)j);
+                    ++slot;
+                }
+            }
         }
     });
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        gt += __shfl_xor_sync(0xFFFFFFFFu, gt, o);
-        eq += __shfl_xor_sync(0xFFFFFFFFu, eq, o);
-    }
-    if (warp >= 2 && lane == 0) {
-        s.wcnt[warp - 2][0] = gt;
-        s.wcnt[warp - 2][1] = eq;
-    }
+    for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xFFFFFFFFu, above, o);
+    if (warp >= 2 && lane == 0) s.wcnt[warp - 2][0] = above;
     tc::tc_fence_before();
     __syncthreads();
-    if (warp == 1) tc::tmem_dealloc(tbase, kTmemCols);   // no TMEM reads past this point
     if (tid == 0) {
-        uint32_t g = 0, e = 0;
-        for (int w = 0; w < 8; ++w) {
-            g += s.wcnt[w][0];
-            e += s.wcnt[w][1];
-        }
-        s.pub[0] = g;
-        s.pub[1] = e;
+        uint32_t a = 0;
+        for (int w = 0; w < 8; ++w) a += s.wcnt[w][0];
+        s.pub[0] = a;
+        s.pub[1] = s.ncand;   // may exceed the list's capacity
     }
-    cl::sync();                                   // every CTA's counts are published
+    cl::sync();                                   // every CTA's counts and candidates are published
     if (warp == 0) {
-        uint32_t g = 0, e = 0;
+        uint2 x = make_uint2(0u, 0u);
+        if ((uint32_t)lane < C) x = cl::ld_v2(cl::map_rank(tc::smem_u32(s.pub), (uint32_t)lane));
+        const uint32_t cincl = warp_incl_scan(x.y, lane);
+        const bool over = __any_sync(0xFFFFFFFFu, x.y > (uint32_t)kCandCap);
+        const uint32_t total = __shfl_sync(0xFFFFFFFFu, cincl, 31);
         if ((uint32_t)lane < C) {
-            const uint2 x = cl::ld_v2(cl::map_rank(tc::smem_u32(s.pub), (uint32_t)lane));
-            g = x.x;
-            e = x.y;
+            s.peer[lane][0] = x.x;            // entries above bin d1
+            s.peer[lane][1] = cincl - x.y;    // candidates of lower-ranked CTAs
         }
-        const uint32_t tb = warp_incl_scan(e, lane) - e;             // ties in lower-ranked CTAs
-        const uint32_t take = tb < R ? min(e, R - tb) : 0u;
-        const uint32_t ob = warp_incl_scan(g + take, lane) - (g + take);
-        const uint32_t my_take = __shfl_sync(0xFFFFFFFFu, take, (int)rank);
-        const uint32_t my_ob = __shfl_sync(0xFFFFFFFFu, ob, (int)rank);
-        if (lane == 0) {
-            s.cbase[0] = my_take;
-            s.cbase[1] = my_ob;
+        if (lane == 0) s.fast = (!over && total <= (uint32_t)kGatherCap) ? total : kSlowPath;
+    }
+    __syncthreads();
+
+    const uint32_t ncg = s.fast;
+    if (ncg != kSlowPath) {
+        // ---- the threshold bin is small: gather it and finish the select locally
+        if (warp == 1) tc::tmem_dealloc(tbase, kTmemCols);   // no TMEM reads past this point
+        constexpr int kU = 8;   // distributed loads in flight per thread
+        for (uint32_t i0 = 0; i0 < ncg; i0 += kU * kThreads) {
+            uint2 x[kU];
+            uint32_t rr[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const uint32_t i = i0 + (uint32_t)(u * kThreads + tid);
+                rr[u] = 0;
+                x[u] = make_uint2(0u, 0u);
+                if (i < ncg) {
+                    uint32_t r = 0;
+                    while (r + 1 < C && s.peer[r + 1][1] <= i) ++r;
+                    rr[u] = r;
+                    x[u] = cl::ld_v2(cl::map_rank(tc::smem_u32(&cand[i - s.peer[r][1]]), r));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const uint32_t i = i0 + (uint32_t)(u * kThreads + tid);
+                if (i < ncg) gath[i] = make_uint2(x[u].x, x[u].y | (rr[u] << 16));
+            }
+        }
+        __syncthreads();
+        for (uint32_t i = tid; i < ncg; i += kThreads) atomicAdd(&hist2[(gath[i].x >> 10) & (kNB2 - 1)], 1u);
+        __syncthreads();
+        find_bin<kNB2>(s, hist2, rank, 1, R, tid);
+        const uint32_t p2 = (d1 << 11) | s.res[0];
+        const uint32_t R3 = R - s.res[1];
+        for (uint32_t i = tid; i < ncg; i += kThreads) {
+            const uint32_t key = gath[i].x;
+            if ((key >> 10) == p2) atomicAdd(&hist3[key & (kNB3 - 1)], 1u);
+        }
+        __syncthreads();
+        find_bin<kNB3>(s, hist3, rank, 1, R3, tid);
+        const uint32_t T = (p2 << 10) | s.res[0];
+        const uint32_t Rt = R3 - s.res[1];   // keys equal to T to take, lowest positions first (1 <= Rt)
+        // every CTA's counts above and at T; this CTA's own candidates into the bitmaps
+        for (uint32_t i = (uint32_t)(warp * 32 + lane); i - (uint32_t)lane < ncg; i += kThreads) {
+            const bool ok = i < ncg;
+            const uint2 x = ok ? gath[i] : make_uint2(0u, 0u);
+            const uint32_t r = ok ? (x.y >> 16) : 0xFFFFu;
+            const bool gt = ok && x.x > T, eq = ok && x.x == T;
+            const uint32_t peers = __match_any_sync(0xFFFFFFFFu, r);
+            const uint32_t bg = __ballot_sync(0xFFFFFFFFu, gt) & peers, be = __ballot_sync(0xFFFFFFFFu, eq) & peers;
+            if (ok && lane == __ffs(peers) - 1) {
+                if (bg != 0u) atomicAdd(&s.rcnt[r][0], (uint32_t)__popc(bg));
+                if (be != 0u) atomicAdd(&s.rcnt[r][1], (uint32_t)__popc(be));
+            }
+            if (r == rank && (gt || eq)) {
+                const uint32_t e = x.y & 0xFFFFu;
+                atomicOr(&(gt ? selbm : tiebm)[e >> 5], 1u << (e & 31));
+            }
+        }
+        __syncthreads();
+        if (tid == 0) {   // CTA r covers positions below CTA r + 1: ties go to the lower ranks first
+            uint32_t tb = 0, ob = 0;
+            for (uint32_t r = 0; r < C; ++r) {
+                const uint32_t e = s.rcnt[r][1];
+                const uint32_t take = tb < Rt ? min(e, Rt - tb) : 0u;
+                if (r == rank) {
+                    s.cbase[0] = take;
+                    s.cbase[1] = ob;
+                }
+                tb += e;
+                ob += s.peer[r][0] + s.rcnt[r][0] + take;
+            }
+        }
+    } else {
+        // ---- a threshold bin too large to gather (many equal or close keys):
+        // two more radix passes over the keys in TMEM, each with a cluster-wide find
+        uint32_t Rs = R;
+        sweep_cols(tbase, warp, ntiles, [&](const uint32_t(&v)[32], int c0, int) {
+            uint32_t m = 0;   // bit j: column c0 + j matches (independent compares, then a short loop)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) m |= (uint32_t)(c0 + j < ntiles && (v[j] >> 21) == d1) << j;
+            while (m != 0u) {
+                const int j = __ffs(m) - 1;
+                m &= m - 1u;
+                atomicAdd(&hist2[(v[j] >> 10) & (kNB2 - 1)], 1u);
+            }
+        });
+        cl::sync();
+        find_bin<kNB2>(s, hist2, 0, C, Rs, tid);
+        const uint32_t p2 = (d1 << 11) | s.res[0];
+        Rs -= s.res[1];
+        sweep_cols(tbase, warp, ntiles, [&](const uint32_t(&v)[32], int c0, int) {
+            uint32_t m = 0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) m |= (uint32_t)(c0 + j < ntiles && (v[j] >> 10) == p2) << j;
+            while (m != 0u) {
+                const int j = __ffs(m) - 1;
+                m &= m - 1u;
+                atomicAdd(&hist3[v[j] & (kNB3 - 1)], 1u);
+            }
+        });
+        cl::sync();
+        find_bin<kNB3>(s, hist3, 0, C, Rs, tid);
+        const uint32_t T = (p2 << 10) | s.res[0];
+        Rs -= s.res[1];   // ties at T still to take, lowest positions first (1 <= Rs)
+        // keys > T and == T: counted, and marked in position bitmaps (column c of lane l
+        // is entry 128 c + 32 q + l: bitmap word 4 c + q, bit l)
+        uint32_t gt = 0, eq = 0;
+        sweep_cols(tbase, warp, ntiles, [&](const uint32_t(&v)[32], int c0, int q) {
+            uint32_t mg = 0, me = 0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const bool valid = c0 + j < ntiles;
+                mg |= (uint32_t)(valid && v[j] > T) << j;
+                me |= (uint32_t)(valid && v[j] == T) << j;
+            }
+            gt += __popc(mg);
+            eq += __popc(me);
+            const uint32_t bit = 1u << lane;
+            const int w0 = 4 * c0 + q;
+            while (mg != 0u) {
+                const int j = __ffs(mg) - 1;
+                mg &= mg - 1u;
+                atomicOr(&selbm[w0 + 4 * j], bit);
+            }
+            while (me != 0u) {
+                const int j = __ffs(me) - 1;
+                me &= me - 1u;
+                atomicOr(&tiebm[w0 + 4 * j], bit);
+            }
+        });
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            gt += __shfl_xor_sync(0xFFFFFFFFu, gt, o);
+            eq += __shfl_xor_sync(0xFFFFFFFFu, eq, o);
+        }
+        if (warp >= 2 && lane == 0) {
+            s.wcnt[warp - 2][0] = gt;
+            s.wcnt[warp - 2][1] = eq;
+        }
+        tc::tc_fence_before();
+        __syncthreads();
+        if (warp == 1) tc::tmem_dealloc(tbase, kTmemCols);   // no TMEM reads past this point
+        if (tid == 0) {
+            uint32_t g = 0, e = 0;
+            for (int w = 0; w < 8; ++w) {
+                g += s.wcnt[w][0];
+                e += s.wcnt[w][1];
+            }
+            s.pub2[0] = g;
+            s.pub2[1] = e;
+        }
+        cl::sync();                               // every CTA's counts are published
+        if (warp == 0) {
+            uint32_t g = 0, e = 0;
+            if ((uint32_t)lane < C) {
+                const uint2 x = cl::ld_v2(cl::map_rank(tc::smem_u32(s.pub2), (uint32_t)lane));
+                g = x.x;
+                e = x.y;
+            }
+            const uint32_t tb = warp_incl_scan(e, lane) - e;             // ties in lower-ranked CTAs
+            const uint32_t take = tb < Rs ? min(e, Rs - tb) : 0u;
+            const uint32_t ob = warp_incl_scan(g + take, lane) - (g + take);
+            const uint32_t my_take = __shfl_sync(0xFFFFFFFFu, take, (int)rank);
+            const uint32_t my_ob = __shfl_sync(0xFFFFFFFFu, ob, (int)rank);
+            if (lane == 0) {
+                s.cbase[0] = my_take;
+                s.cbase[1] = my_ob;
+            }
         }
     }
     __syncthreads();
