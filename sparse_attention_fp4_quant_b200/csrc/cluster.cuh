@@ -40,6 +40,12 @@ __device__ __forceinline__ uint4 ld_v4(uint32_t addr) {
     return v;
 }
 
+__device__ __forceinline__ uint32_t ld_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ uint2 ld_v2(uint32_t addr) {
     uint2 v;
     asm volatile("ld.shared::cluster.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");

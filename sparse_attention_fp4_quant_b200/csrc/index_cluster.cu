@@ -43,12 +43,13 @@ constexpr uint32_t kTmemCols = kPipeCols + kMaxTiles;
 constexpr int kWords = kMaxTiles * kTile / 32;          // bitmap words over the CTA's entries
 constexpr int kNB1 = 2048, kNB2 = 2048, kNB3 = 1024;   // radix digits: bits 31..21, 20..10, 9..0
 constexpr int kSel = 256;                  // threads of the scans (warps 0-7)
-constexpr int kCandCap = 4096;             // candidates (keys of the threshold's top bin) a CTA lists
+constexpr int kCandPerWarp = 256;          // candidates (keys of the threshold's top bin) a sweeping warp lists
+constexpr int kCandCap = 8 * kCandPerWarp; // and a CTA
 constexpr int kGatherCap = 8192;           // candidates of a cluster gathered for the local select
 constexpr uint32_t kSlowPath = 0xFFFFFFFFu;
 constexpr int kSelWarps = kSel / 32;
 using ClPipe = Pipe<kRing>;
-static_assert((kNB2 + kNB3 + 2 * kWords) * 4 + (kCandCap + kGatherCap) * 8 <= (int)sizeof(ClPipe::A),
+static_assert((kNB2 + kNB3 + 2 * kWords) * 4 + (2 * kCandCap + kGatherCap) * 8 <= (int)sizeof(ClPipe::A),
               "select scratch fits the ring");
 static_assert(kTmemCols == 512, "TMEM");
 
@@ -61,7 +62,8 @@ struct ClSmem {
     alignas(8) uint32_t pub[2];             // this CTA's (entries above bin d1, candidates), read by the cluster
     alignas(8) uint32_t pub2[2];            // (> T, == T) counts of the multi-pass path, read by the cluster
     uint32_t cbase[2];                      // this CTA's tie quota and output offset
-    uint32_t ncand;                         // candidates appended (may exceed the list)
+    uint32_t wcand[8];                      // candidates each sweeping warp found (may exceed its list)
+    alignas(8) uint32_t coarse[64];         // hist1 in 64 bins of 32
     uint32_t fast;                          // candidates of the cluster, or kSlowPath
     uint32_t peer[16][2];                   // per CTA: entries above bin d1, candidates of lower ranks
     uint32_t rcnt[16][2];                   // per CTA: candidates above T, equal to T
@@ -74,6 +76,21 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
         if (lane >= o) v += y;
     }
     return v;
+}
+
+// v[j] for a run-time j without indexing the array (which would move it to
+// local memory): a binary select tree on the bits of j.
+__device__ __forceinline__ uint32_t pick32(const uint32_t (&v)[32], uint32_t j) {
+    uint32_t a[16], b[8], c[4], d[2];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a[i] = (j & 16u) ? v[i + 16] : v[i];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) b[i] = (j & 8u) ? a[i + 8] : a[i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[i] = (j & 4u) ? b[i + 4] : b[i];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) d[i] = (j & 2u) ? c[i + 2] : c[i];
+    return (j & 1u) ? d[1] : d[0];
 }
 
 // 32 x 32 bit transpose across the warp: in, bit j of lane l is element
@@ -107,6 +124,63 @@ __device__ __forceinline__ uint32_t block_scan_excl(ClSmem& s, uint32_t v, int t
     *total = tot;
     __syncthreads();
     return pre;
+}
+
+// One warp: the bin d1 of hist1 (summed over the cluster's C CTAs) holding
+// the R-th largest key, in two levels: the 64 coarse sums (32 bins each) give
+// the coarse bin, its 32 bins the fine one.  Leaves (d1, keys above d1) in
+// s.res for the CTA.
+__device__ __forceinline__ void find_top_bin(ClSmem& s, uint32_t C, uint32_t R, int lane) {
+    constexpr int RG = 4;   // CTAs whose loads are in flight together
+    // lane l: coarse bins 2l and 2l + 1 (the highest bins on lane 31)
+    uint32_t lo = 0, hi = 0;
+    const uint32_t ca = tc::smem_u32(&s.coarse[2 * lane]);
+    for (uint32_t r0 = 0; r0 < C; r0 += RG) {
+        uint2 x[RG];
+#pragma unroll
+        for (int g = 0; g < RG; ++g) x[g] = r0 + g < C ? cl::ld_v2(cl::map_rank(ca, r0 + g)) : make_uint2(0u, 0u);
+#pragma unroll
+        for (int g = 0; g < RG; ++g) {
+            lo += x[g].x;
+            hi += x[g].y;
+        }
+    }
+    uint32_t suf = lo + hi;   // keys in this lane's coarse bins and every higher lane's
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xFFFFFFFFu, suf, o);
+        if (lane + o < 32) suf += y;
+    }
+    const uint32_t abv = suf - lo - hi;
+    const int L = __ffs(__ballot_sync(0xFFFFFFFFu, abv < R && R <= suf)) - 1;
+    uint32_t cb = 0, cab = 0;
+    if (lane == L) {
+        cb = abv + hi >= R ? 2u * lane + 1u : 2u * lane;
+        cab = abv + hi >= R ? abv : abv + hi;
+    }
+    cb = __shfl_sync(0xFFFFFFFFu, cb, L);
+    cab = __shfl_sync(0xFFFFFFFFu, cab, L);
+    // lane l: bin 32 cb + l
+    uint32_t f = 0;
+    const uint32_t fa = tc::smem_u32(&s.hist1[32 * cb + lane]);
+    for (uint32_t r0 = 0; r0 < C; r0 += RG) {
+        uint32_t x[RG];
+#pragma unroll
+        for (int g = 0; g < RG; ++g) x[g] = r0 + g < C ? cl::ld_u32(cl::map_rank(fa, r0 + g)) : 0u;
+#pragma unroll
+        for (int g = 0; g < RG; ++g) f += x[g];
+    }
+    uint32_t fs = f;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xFFFFFFFFu, fs, o);
+        if (lane + o < 32) fs += y;
+    }
+    const uint32_t R2 = R - cab, fab = fs - f;
+    if (fab < R2 && R2 <= fs) {
+        s.res[0] = 32u * cb + (uint32_t)lane;
+        s.res[1] = cab + fab;
+    }
 }
 
 // Sum the NB-bin histogram `hist` over the CTAs r0 .. r0 + n - 1 of the
@@ -306,13 +380,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* selbm = hist3 + kNB3;   // entries above T (then also the ties taken)
     uint32_t* tiebm = selbm + kWords; // entries equal to T
     uint2* cand = reinterpret_cast<uint2*>(tiebm + kWords);   // this CTA's keys of bin d1: (key, entry)
-    uint2* gath = cand + kCandCap;                             // the cluster's, gathered: (key, entry | rank << 16)
+    uint2* wlist = cand + kCandCap;                            // each sweeping warp's, before compaction
+    uint2* gath = wlist + kCandCap;                            // the cluster's, gathered: (key, entry | rank << 16)
     for (int i = tid; i < kNB2 + kNB3 + 2 * kWords; i += kThreads) hist2[i] = 0;
     if (tid < 32) s.rcnt[tid >> 1][tid & 1] = 0;
-    if (tid == 0) s.ncand = 0;
+    if (warp >= 2) {   // hist1 in coarse bins of 32, for the cluster's two-level search
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int cb = 8 * (warp - 2) + i;
+            const uint32_t x = __reduce_add_sync(0xFFFFFFFFu, s.hist1[32 * cb + lane]);
+            if (lane == 0) s.coarse[cb] = x;
+        }
+    }
 
     cl::sync();                                   // every CTA's hist1 is complete
-    find_bin<kNB1>(s, s.hist1, 0, C, K1, tid);
+    if (warp == 0) find_top_bin(s, C, K1, lane);
+    __syncthreads();
     const uint32_t d1 = s.res[0];
     const uint32_t R = K1 - s.res[1];             // keys still to take from bin d1 (1 <= R)
 
@@ -320,15 +403,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // is (marked in the bitmaps: one word per column and lane quarter, built by
     // a bit transpose of the lanes' column masks); an entry of bin d1 is a
     // candidate, appended to this CTA's list.
-    uint32_t above = 0;
+    uint32_t above = 0, nlist = 0;   // nlist: this warp's candidates (warp-uniform)
+    uint2* mylist = wlist + (warp >= 2 ? warp - 2 : 0) * kCandPerWarp;
+    const uint32_t top = ((d1 + 1u) << 21) - 1u;   // keys above bin d1 are > top (none when d1 = 2047)
+    const uint32_t bot = d1 << 21;                 // keys of bin d1: key - bot < 2^21
     sweep_cols(tbase, warp, ntiles, [&](const uint32_t(&v)[32], int c0, int q) {
-        uint32_t ma = 0, mc = 0;   // bit j: the key of column c0 + j is above bin d1 / in bin d1
+        uint32_t ma4[4] = {0u, 0u, 0u, 0u}, mc4[4] = {0u, 0u, 0u, 0u};   // four short chains
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-            const uint32_t bin = v[j] >> 21;
-            ma |= (uint32_t)(bin > d1) << j;
-            mc |= (uint32_t)(bin == d1) << j;
+            ma4[j & 3] |= (uint32_t)(v[j] > top) << j;
+            mc4[j & 3] |= (uint32_t)(v[j] - bot < (1u << 21)) << j;
         }
+        // bit j: the key of column c0 + j is above bin d1 / in bin d1
+        uint32_t ma = (ma4[0] | ma4[1]) | (ma4[2] | ma4[3]), mc = (mc4[0] | mc4[1]) | (mc4[2] | mc4[3]);
         if (ntiles - c0 < 32) {   // columns past the last tile hold no keys
             const uint32_t cm = (1u << (ntiles - c0)) - 1u;
             ma &= cm;
@@ -340,14 +427,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (__any_sync(0xFFFFFFFFu, mc != 0u)) {
             const uint32_t n = __popc(mc);
             const uint32_t incl = warp_incl_scan(n, lane);
-            uint32_t base = 0;
-            if (lane == 31) base = atomicAdd(&s.ncand, incl);
-            uint32_t slot = __shfl_sync(0xFFFFFFFFu, base, 31) + incl - n;
+            const uint32_t base = nlist + incl - n;
+            nlist += __shfl_sync(0xFFFFFFFFu, incl, 31);
             const uint32_t e0 = 128u * (uint32_t)c0 + 32u * (uint32_t)q + (uint32_t)lane;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                if ((mc >> j) & 1u) {
-                    if (slot < (uint32_t)kCandCap) cand[slot] = make_uint2(v[j], e0 + 128u * (uint32_t)j);
+            // a lane has few candidates: visit its set bits, picking the key by a
+            // five-level select on the column's bits (the keys stay in registers)
+            uint32_t m = mc, slot = base;
+            while (__any_sync(0xFFFFFFFFu, m != 0u)) {
+                if (m != 0u) {
+                    const uint32_t j = (uint32_t)__ffs(m) - 1u;
+                    m &= m - 1u;
+                    if (slot < (uint32_t)kCandPerWarp) mylist[slot] = make_uint2(pick32(v, j), e0 + 128u * j);
                     ++slot;
                 }
             }
@@ -355,14 +445,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     });
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xFFFFFFFFu, above, o);
-    if (warp >= 2 && lane == 0) s.wcnt[warp - 2][0] = above;
+    if (warp >= 2 && lane == 0) {
+        s.wcnt[warp - 2][0] = above;
+        s.wcand[warp - 2] = nlist;
+    }
     tc::tc_fence_before();
     __syncthreads();
+    if (warp >= 2) {   // compact the warps' lists into this CTA's list, in warp order
+        uint32_t base = 0;
+        for (int w = 0; w < warp - 2; ++w) base += min(s.wcand[w], (uint32_t)kCandPerWarp);
+        const uint32_t n = min(nlist, (uint32_t)kCandPerWarp);
+        for (uint32_t i = lane; i < n; i += 32) cand[base + i] = mylist[i];
+    }
     if (tid == 0) {
-        uint32_t a = 0;
-        for (int w = 0; w < 8; ++w) a += s.wcnt[w][0];
+        uint32_t a = 0, n = 0;
+        bool over = false;
+        for (int w = 0; w < 8; ++w) {
+            a += s.wcnt[w][0];
+            n += s.wcand[w];
+            over = over || s.wcand[w] > (uint32_t)kCandPerWarp;
+        }
         s.pub[0] = a;
-        s.pub[1] = s.ncand;   // may exceed the list's capacity
+        s.pub[1] = over ? (uint32_t)kCandCap + 1u : n;   // above the capacity: too many to gather
     }
     cl::sync();                                   // every CTA's counts and candidates are published
     if (warp == 0) {
@@ -461,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             while (m != 0u) {
                 const int j = __ffs(m) - 1;
                 m &= m - 1u;
-                atomicAdd(&hist2[(v[j] >> 10) & (kNB2 - 1)], 1u);
+                atomicAdd(&hist2[(pick32(v, (uint32_t)j) >> 10) & (kNB2 - 1)], 1u);
             }
         });
         cl::sync();
@@ -475,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             while (m != 0u) {
                 const int j = __ffs(m) - 1;
                 m &= m - 1u;
-                atomicAdd(&hist3[v[j] & (kNB3 - 1)], 1u);
+                atomicAdd(&hist3[pick32(v, (uint32_t)j) & (kNB3 - 1)], 1u);
             }
         });
         cl::sync();
