@@ -72,7 +72,7 @@ def job_value(world, ms_max):
 
 def _kernel_hash():
     h = hashlib.sha256()
-    for f in ("index_cluster.cu", "index_pipe.cuh", "index_tc.cu", "tc.cuh", "common.cuh", "kernels.h"):
+    for f in ("index_cluster.cu", "index_pipe.cuh", "index_tc.cu", "tc.cuh", "common.cuh", "cluster.cuh", "kernels.h"):
         with open(os.path.join(ROOT, "sparse_attention_fp4_quant_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
