@@ -203,6 +203,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int i = et; i < k; i += kEpiN) p.out[(int64_t)bq * k + i] = i < cnt ? tk.pos_at(i) : -1;
 }
 
+// two CTAs per SM for the usual k (the k > 1536 variant runs one)
+static_assert(sizeof(TcSmem<2048>) + 1024 <= 113 * 1024, "shared memory of two CTAs per SM");
+
 }  // namespace
 
 bool index_tc_supported(const SelectParams& p) {

@@ -240,6 +240,36 @@ def test_index_topk_ties_and_zero_scores(csa):
         assert list(np_(idx)[0, 2]) == list(range(k))
 
 
+def test_index_topk_ties_at_threshold_across_ctas(csa):
+    # 400 copies of a high-scoring key and 600 of a slightly lower one, spread over
+    # the whole range: the threshold is the lower key, its ties are split over the
+    # cluster's CTAs and the lowest positions must win.  The threshold bin stays
+    # small, so the gathered-candidate select decides it.
+    B, Q, cap, k = 1, 1, 65536, 512
+    grp = Group(23, B, cap, [cap])
+    o = grp.oracle_cache()
+    iq, iqs, w, oiq, oiqs, ow = index_query(24, B, Q)
+    sc = np.array([oracle.index_score(oiq[0, 0], oiqs[0, 0], ow[0, 0], o["ik"][0, e], o["iks"][0, e])
+                   for e in range(0, cap, 61)], np.float64)
+    top = np.argsort(-sc)[:2] * 61                  # two of the best entries of a sample
+    hi, lo = (int(top[0]), int(top[1])) if sc[top[0] // 61] > sc[top[1] // 61] else (int(top[1]), int(top[0]))
+    assert sc[hi // 61] > sc[lo // 61]
+    rng = np.random.default_rng(25)
+    pos = rng.permutation(cap)
+    pos = pos[(pos != hi) & (pos != lo)]
+    gik, giks = kv_ik_rows(grp.kv)
+    oik, oiks = o["ik"].copy(), o["iks"].copy()
+    for dst, src in ((pos[:400], hi), (pos[400:1000], lo)):
+        gik[0, dst], giks[0, dst] = gik[0, src], giks[0, src]
+        oik[0, dst], oiks[0, dst] = oik[0, src], oiks[0, src]
+    set_kv_ik_rows(grp.kv, gik, giks)
+    q_pos = np.array([[cap - 1]], np.int32)
+    idx = csa.csa2_index_topk(iq, iqs, w, grp.kv, torch.from_numpy(q_pos).cuda(), k)
+    ridx = oracle.index_topk(oiq, oiqs, ow, oik, oiks, grp.n_entries, 1, q_pos, k)
+    assert np.array_equal(np_(idx), ridx)
+    assert np.isin(np.concatenate([pos[:400], [hi]]), ridx).all()   # every copy of the higher key
+
+
 def test_device_error_flag_stays_clear(csa):
     B, Q, cap, k = 2, 1, 3072, 64
     grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(31, B, Q, cap, [3000, 2000], 1, [[2999], [1999]], k)
