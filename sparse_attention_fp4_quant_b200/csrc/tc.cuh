@@ -1,5 +1,5 @@
 // tc.cuh -- thin wrappers over the sm_100a PTX used by the tensor-core kernels:
-// mbarriers with bounded waits, TMA tensor loads, cp.async, and tcgen05
+// mbarriers with bounded waits, bulk (TMA-engine) copies, and tcgen05
 // (TMEM allocation, smem->TMEM copies, block-scaled MMA, commits, TMEM loads).
 #pragma once
 #include <stdint.h>
@@ -72,16 +72,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                      smem_u32(dst)),
                  "l"(src), "r"(bytes), "r"(smem_u32(bar))
                  : "memory");
-}
-
-__device__ __forceinline__ void cp_async_4(void* dst, const void* src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-
-// Arrive on `bar` once all prior cp.async of this thread have landed (counts as one of the
-// barrier's expected arrivals).
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
