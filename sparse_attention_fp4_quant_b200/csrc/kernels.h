@@ -63,11 +63,17 @@ struct SelectParams {
     int32_t* cand_cnt;     // [B*Q][S]
     uint32_t* cand_key;    // [B*Q][S][k]
     int32_t* cand_pos;     // [B*Q][S][k]
+    void* mq_ws;           // index Top-K for many queries: key prefixes and histograms (else null)
 };
 
 int select_splits(int op, int B, int Q, int64_t cap, int k, int P);
-size_t select_ws_bytes(int op, int B, int Q, int64_t cap, int k, int P);
-void select_carve_ws(SelectParams& p, int S, void* ws, int B, int Q, int k);
+// mq = false leaves out the many-query index path's part (a fixed scratch that may not hold it)
+size_t select_ws_bytes(int op, int B, int Q, int64_t cap, int k, int P, bool mq = true);
+void select_carve_ws(SelectParams& p, int S, void* ws, int B, int Q, int k, bool mq = true);
+// Index Top-K for many queries per batch row (index_mq.cu).
+bool index_mq_eligible(int B, int Q, int64_t cap);
+size_t index_mq_ws_bytes(int B, int Q, int64_t cap);
+cudaError_t launch_index_mq(SelectParams& p, void* mq_ws, cudaStream_t st);
 cudaError_t launch_select(int op, SelectParams& p, int S, cudaStream_t st);
 bool index_tc_supported(const SelectParams& p);
 cudaError_t launch_index_tc(int op, SelectParams& p, int S, cudaStream_t st);

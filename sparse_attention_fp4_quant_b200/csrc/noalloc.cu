@@ -54,7 +54,8 @@ csa2_status csa2_index_topk_noalloc(const uint8_t* q, const uint8_t* q_sc, const
     if (((uintptr_t)q & 15u) || ((uintptr_t)kv->ik & 15u) || ((uintptr_t)kv->ik_sc & 15u) || kv->cap % 128 != 0)
         return CSA2_ERR_INVALID_ARG;
     if (((uintptr_t)q_sc & 3u) || ((uintptr_t)w & 3u)) return CSA2_ERR_INVALID_ARG;
-    const size_t need = select_ws_bytes(CSA2_OP_INDEX_TOPK, B, Q, kv->cap, k, 0);
+    // the fixed scratch serves the per-share and cluster paths (not the many-query one)
+    const size_t need = select_ws_bytes(CSA2_OP_INDEX_TOPK, B, Q, kv->cap, k, 0, false);
     if (need > kScratchBytes) return CSA2_ERR_WORKSPACE;
     void* ws = nullptr;
     cudaError_t e = scratch_on_current_device(&ws);
@@ -80,7 +81,7 @@ csa2_status csa2_index_topk_noalloc(const uint8_t* q, const uint8_t* q_sc, const
         p.blockmax = blockmax_out;
         p.nb_cap = (kv->cap + CSA2_BLOCK - 1) / CSA2_BLOCK;
         const int S = select_splits(CSA2_OP_INDEX_TOPK, B, Q, kv->cap, k, 0);
-        select_carve_ws(p, S, ws, B, Q, k);
+        select_carve_ws(p, S, ws, B, Q, k, false);
         e = launch_select(CSA2_OP_INDEX_TOPK, p, S, (cudaStream_t)stream);
     }
     if (e != cudaSuccess) {
