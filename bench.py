@@ -450,6 +450,74 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_prefill(args):
+    """The prefill chunk (one GPU): 65,536-token prompt compressed 2:1 into 32,768 entries,
+    4,096 queries at its end; index + Top-512 and one attention layer (main + SWA-128),
+    each timed with CUDA events over K steps, L2 flushed between steps."""
+    import sparse_attention_fp4_quant_b200 as csa
+    torch.cuda.set_device(0)
+    csa.lib()
+    device = "cuda"
+    Bp, n, Q, tokens, T = 1, 32768, 4096, 65536, 4096 + T_SWA - 1
+    kv = csa.KV(Bp, n, 2, device)
+    W = synth.proj_w(130).to(device)
+    lat = synth.latent(synth.seed_of("prefill-ctx", 0), n, 0, device)
+    csa.csa2_quant_nvfp4(lat, kv.lat.view(-1, 256), kv.lat_sc.view(-1, 32))
+    csa.csa2_index_k_proj(lat, W, kv.ik.view(-1, 32), kv.ik_sc.view(-1, 4))
+    del lat
+    kv.n_entries.fill_(n)
+    iq, iqs = csa.csa2_quant_nvfp4(synth.index_q(synth.seed_of("prefill-iq"), Bp, Q, device).view(-1, 64))
+    iq, iqs = iq.view(Bp, Q, 128), iqs.view(Bp, Q, 16)
+    w = synth.index_w(Bp, Q, device)
+    q_pos = (torch.arange(Q, device=device, dtype=torch.int32) + (tokens - Q)).view(Bp, Q)
+    q = synth.attn_q(synth.seed_of("prefill-q"), Bp, Q, device)
+    pos0 = tokens - T
+    swa, swa_sc = synth.swa_kv(synth.seed_of("prefill-swa"), T, pos0, device)
+    swa, swa_sc = swa.unsqueeze(0), swa_sc.unsqueeze(0)
+    pos0_t = torch.tensor([pos0], dtype=torch.int32, device=device)
+    idx = torch.empty((Bp, Q, TOPK), dtype=torch.int32, device=device)
+    out = torch.empty((Bp, Q, 16, 512), dtype=torch.bfloat16, device=device)
+    ws = torch.zeros(max(csa.csa2_workspace_bytes(csa.OP_INDEX_TOPK, Bp, Q, n, TOPK),
+                         csa.csa2_workspace_bytes(csa.OP_SPARSE_ATTN, Bp, Q, n, TOPK)), dtype=torch.uint8, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    st = torch.cuda.current_stream()
+    t_idx, t_att = [], []
+    for it in range(args.warmup + args.steps):
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record(st)
+        csa.csa2_index_topk(iq, iqs, w, kv, q_pos, TOPK, idx, ws=ws)
+        ev[1].record(st)
+        csa.csa2_sparse_attn(q, kv, idx, swa, swa_sc, pos0_t, q_pos, out=out, ws=ws)
+        ev[2].record(st)
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            t_idx.append(ev[0].elapsed_time(ev[1]))
+            t_att.append(ev[1].elapsed_time(ev[2]))
+    idx_ms, att_ms = float(np.mean(t_idx)), float(np.mean(t_att))
+    nvis = np.minimum((q_pos.cpu().numpy().astype(np.int64) + 1) // 2, n)
+    idx_flop = float(nvis.sum()) * 4 * 64 * 2           # dense-equivalent indexer Q.K^T
+    att_flop = float(Q) * 16 * (TOPK + T_SWA) * 512 * 4  # S and P V over every slot
+    with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+        bf16 = float(json.load(f)["bf16_tflops"])
+    fp4_peak = bf16 * 4.0   # nominal dense FP4 / BF16 ratio (9 / 2.25 PFLOP/s)
+    achieved = idx_flop / (idx_ms * 1e-3) / 1e12
+    print(json.dumps({
+        "metric": "CSA2 prefill chunk queries/s (index + Top-512 + one attention layer)",
+        "value": Q / ((idx_ms + att_ms) * 1e-3), "unit": "queries/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": idx_ms + att_ms, "higher_is_better": True, "dtype": "e2m1+bf16",
+        "data": "synthetic",
+        "config": {"workload": "c3: prefill chunk, 65,536-token prompt, m=2 (32,768 entries), 4,096 queries, "
+                               "Top-512, SWA-128", "l2": "flushed between timed steps"},
+        "index_ms": idx_ms, "attention_ms": att_ms,
+        "roofline": {"kernel": "csa2_index_topk (mq_score_kernel + mq_select_kernel)", "bound": "tensor",
+                     "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s", "frac": achieved / fp4_peak,
+                     "peak_source": "measured bf16 GEMM burst (MEASURED_PEAKS.json) x 4, the nominal FP4/BF16 ratio",
+                     "flop_per_launch": idx_flop},
+        "attention_tflops": att_flop / (att_ms * 1e-3) / 1e12,
+    }))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -457,8 +525,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["decode", "prefill"], default="decode",
+                    help="decode: the headline B=32 step (default); prefill: the 4,096-query chunk, one GPU")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.workload == "prefill":
+        run_prefill(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
