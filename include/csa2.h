@@ -183,7 +183,11 @@ CSA2_API csa2_status csa2_append_tokens(const void* x, int64_t rows, const float
  *   blockmax_out  device fp32 [B][Q][ceil(cap/8)] or NULL: the maximum score of
  *                 each block of 8 positions (visible positions only), -inf for
  *                 blocks with no visible position ([Blog] Fig. 5)
- *   ws, ws_bytes  device workspace of at least csa2_workspace_bytes(CSA2_OP_INDEX_TOPK, ...)
+ *   ws, ws_bytes  device workspace of at least csa2_workspace_bytes(CSA2_OP_INDEX_TOPK, ...);
+ *                 for more than 148 queries with at least 8 per batch row and
+ *                 cap <= 65,536 (a prefill chunk) it also holds every query's
+ *                 16-bit key prefixes and 2,048-bin histogram (2 B per query
+ *                 and entry + 8 KB per query)
  *                 bytes, zero-filled before its first use; every call leaves its
  *                 counters at zero again.  Calls that share a workspace must not
  *                 overlap on the GPU.  The int32 at byte offset
@@ -332,12 +336,14 @@ CSA2_API csa2_status csa2_layer_step(const csa2_layer_args* a, void* stream);
  * ws_bytes.  The scratch the call needs (the merge counters and the candidate
  * lists of the per-query shares) lives in one static device array of
  * CSA2_NOALLOC_SCRATCH_BYTES inside this library; every GPU that loads the
- * library holds that array until the process exits.  A call whose scratch would
- * exceed the array (csa2_workspace_bytes(CSA2_OP_INDEX_TOPK, B, Q, cap, k, 0) >
- * CSA2_NOALLOC_SCRATCH_BYTES) returns CSA2_ERR_WORKSPACE and launches nothing.
- * The call allocates nothing: no cudaMalloc, cudaFree or allocating library
- * routine; it clears the counters with cudaMemsetAsync on `stream` and then
- * launches the same kernel as csa2_index_topk.
+ * library holds that array until the process exits.  The call never takes the
+ * many-query path (whose key prefixes would not fit): a prefill-sized request
+ * runs the per-share kernels, with the same results.  A call whose scratch
+ * would exceed the array (csa2_workspace_bytes(CSA2_OP_INDEX_TOPK, B, Q, cap,
+ * k, 0) without the many-query part > CSA2_NOALLOC_SCRATCH_BYTES) returns
+ * CSA2_ERR_WORKSPACE and launches nothing.  The call allocates nothing: no
+ * cudaMalloc, cudaFree or allocating library routine; it clears the counters
+ * with cudaMemsetAsync on `stream` and then launches the index kernels.
  *
  * The first call on each device looks up the array's device address with that
  * device current (cudaGetSymbolAddress); make that first call before any stream

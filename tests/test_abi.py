@@ -45,6 +45,12 @@ def test_workspace_sizes_are_host_only(L):
     assert L.csa2_workspace_bytes(0, 0, 1, 10, 512, 0) == 0
     # one share per query needs only the counters
     assert L.csa2_workspace_bytes(csa.OP_INDEX_TOPK, 4096, 1, 1000, 512, 0) == 4096 * 4 + 256  # counters + status word
+    # many queries per batch row (a prefill chunk): the workspace also holds every query's
+    # 16-bit key prefixes and its 2,048-bin histogram for the many-query path
+    many = L.csa2_workspace_bytes(csa.OP_INDEX_TOPK, 1, 4096, 32768, 512, 0)
+    assert many >= 4096 * 32768 * 2 + 4096 * 2048 * 4
+    # beyond 65,536 entries that path is not taken, and nothing is reserved for it
+    assert L.csa2_workspace_bytes(csa.OP_INDEX_TOPK, 1, 4096, 131072, 512, 0) < 4096 * 131072 * 2
 
 
 def test_invalid_arguments_rejected_before_launch(L):
