@@ -3,7 +3,8 @@
 // CTA per query selects its Top-K.
 //
 // Scoring (mq_score_kernel, one CTA per 8 consecutive queries of a batch
-// row).  The block-scaled FP4 MMA of index_pipe.cuh with B = 8 block-diagonal
+// row; 16 epilogue warps, two queries each, so that four warps share each SM
+// sub-partition and hide each other's latency).  The block-scaled FP4 MMA of index_pipe.cuh with B = 8 block-diagonal
 // query operands side by side (N = 128: column 16 g + 4 h + b holds query g's
 // head h codes of block b only), so every key tile crosses shared memory once
 // for 8 queries and each accumulator column is still one exact block product
@@ -37,8 +38,11 @@ constexpr uint32_t kColSA = kAccT * kN;       // unit scales of A
 constexpr uint32_t kColSB = kColSA + 4;       // the queries' scales
 static_assert(kColSB + 4 <= kMqCols, "TMEM columns");
 constexpr uint32_t kIdescN = tc::idesc_mxf4nvf4(128, kN);
-constexpr int kMqThreads = 320;               // warp 0 copies, warp 1 MMA, warps 2-9 epilogue
-constexpr int kMqEpi = 256;
+constexpr int kEpiW = 16;                     // epilogue warps: four per TMEM lane quarter
+constexpr int kQPW = kG * 4 / kEpiW;          // queries per epilogue warp
+constexpr int kMqEpi = 32 * kEpiW;
+constexpr int kMqThreads = 64 + kMqEpi;       // warp 0 copies, warp 1 MMA, the rest epilogue
+static_assert(kQPW * kEpiW == 4 * kG, "every (lane quarter, query) pair has one warp");
 constexpr int kNB1 = 2048;                    // top-11-bit histogram bins
 
 struct MqSmem {
@@ -73,7 +77,7 @@ __global__ void __launch_bounds__(kMqThreads, 1) mq_score_kernel(SelectParams p,
     if (tid == 0) {
         for (int i = 0; i < kMqRing; ++i) {
             tc::mbar_init(&s.full[i], 1);
-            tc::mbar_init(&s.empty[i], 1 + kEpiWarps);   // MMA commit + each epilogue warp (scales read)
+            tc::mbar_init(&s.empty[i], 1 + kEpiW);   // MMA commit + each epilogue warp (scales read)
         }
         for (int i = 0; i < kAccT; ++i) {
             tc::mbar_init(&s.accfull[i], 1);
@@ -150,13 +154,13 @@ __global__ void __launch_bounds__(kMqThreads, 1) mq_score_kernel(SelectParams p,
     } else {
         // ---------------------------------------------------------------- epilogue
         const int quarter = warp & 3;                 // TMEM lanes this warp may read
-        const int gb = 4 * ((warp - 2) >> 2);         // queries gb .. gb + 3
+        const int gb = kQPW * ((warp - 2) >> 2);      // queries gb .. gb + kQPW - 1
         const int row = 32 * quarter + lane;
         const uint32_t lanes = (uint32_t)(32 * quarter) << 16;
-        float wq[4][4];
-        int nv[4];
+        float wq[kQPW][4];
+        int nv[kQPW];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < kQPW; ++j) {
             const int g = gb + j;
             nv[j] = g < ng ? n_visible(p.q_pos[bq0 + g], p.n_entries[b], p.m, p.cap) : 0;
 #pragma unroll
@@ -175,9 +179,9 @@ __global__ void __launch_bounds__(kMqThreads, 1) mq_score_kernel(SelectParams p,
                 }
                 if (dead) continue;
                 tc::tc_fence_after();
-                uint32_t v[4][16];
+                uint32_t v[kQPW][16];
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
+                for (int j = 0; j < kQPW; ++j)
                     tc::tmem_ld_32x32b_x16(tbase + lanes + (uint32_t)(a * kN + 16 * (gb + j)), v[j]);
                 tc::tmem_ld_wait();
                 tc::tc_fence_before();
@@ -191,7 +195,7 @@ __global__ void __launch_bounds__(kMqThreads, 1) mq_score_kernel(SelectParams p,
                 if (i == ntl - 1) release_stage(s, t, lane);
                 const int e = u * kTile + row;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < kQPW; ++j) {
                     const int g = gb + j;
                     if (g >= ng) break;   // warp-uniform
                     const bool valid = e < nv[j];
