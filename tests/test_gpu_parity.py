@@ -141,18 +141,20 @@ def test_index_topk_ragged(csa, m, k):
     assert np.array_equal(np_(bm), rbm)
 
 
-def test_index_topk_many_queries(csa):
-    # 160 queries: more than one cluster per query can hold at once, so the
-    # streaming per-share kernel serves them (prefill-like causal positions)
-    B, Q, cap, m, k = 2, 80, 3072, 2, 512
-    n_entries = [3000, 2100]
-    rng = np.random.default_rng(5)
+@pytest.mark.parametrize("B,Q", [(2, 80), (1, 150)])
+def test_index_topk_many_queries(csa, B, Q):
+    # more queries than one wave of clusters holds: the many-query kernels serve
+    # them (prefill-like causal positions; 150 = 18 groups of 8 and one of 6)
+    cap, m, k = 3072, 2, 512
+    n_entries = [3000, 2100][:B]
+    rng = np.random.default_rng(5 + Q)
     q_pos = rng.integers(0, 6000, size=(B, Q)).astype(np.int32)
     q_pos[0, :4] = [0, 1, 1023, 5999]
-    grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(77, B, Q, cap, n_entries, m, q_pos.tolist(), k)
-    idx = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, k)
-    ridx = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, m, q_pos, k)
+    grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(77 + Q, B, Q, cap, n_entries, m, q_pos.tolist(), k)
+    idx, bm = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, k, blockmax=True)
+    ridx, rbm = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, m, q_pos, k, blockmax=True)
     assert np.array_equal(np_(idx), ridx)
+    assert np.array_equal(np_(bm), rbm)
 
 
 @pytest.mark.parametrize("n", [128, 129, 255, 1001])
