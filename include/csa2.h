@@ -332,18 +332,25 @@ CSA2_API csa2_status csa2_layer_step(const csa2_layer_args* a, void* stream);
  * that hand out no scratch buffers, or latency-critical paths where a
  * cudaMalloc (which can synchronise the device) is not allowed.
  *
- * Arguments, results and errors are those of csa2_index_topk, minus ws and
- * ws_bytes.  The scratch the call needs (the merge counters and the candidate
- * lists of the per-query shares) lives in one static device array of
+ * Arguments and results are those of csa2_index_topk, minus ws and ws_bytes.
+ * The scratch the call needs (the merge counters and the candidate lists of
+ * the per-query shares) lives in one static device array of
  * CSA2_NOALLOC_SCRATCH_BYTES inside this library; every GPU that loads the
  * library holds that array until the process exits.  The call never takes the
  * many-query path (whose key prefixes would not fit): a prefill-sized request
  * runs the per-share kernels, with the same results.  A call whose scratch
  * would exceed the array (csa2_workspace_bytes(CSA2_OP_INDEX_TOPK, B, Q, cap,
- * k, 0) without the many-query part > CSA2_NOALLOC_SCRATCH_BYTES) returns
- * CSA2_ERR_WORKSPACE and launches nothing.  The call allocates nothing: no
- * cudaMalloc, cudaFree or allocating library routine; it clears the counters
- * with cudaMemsetAsync on `stream` and then launches the index kernels.
+ * k, 0) without the many-query part, plus 256 bytes, > CSA2_NOALLOC_SCRATCH_BYTES)
+ * returns CSA2_ERR_WORKSPACE and launches nothing.  The call allocates nothing:
+ * no cudaMalloc, cudaFree or allocating library routine; it clears its error
+ * flag and counters with cudaMemsetAsync on `stream` and then launches the
+ * index kernels.
+ *
+ * Errors: argument and launch errors are returned at once, as by
+ * csa2_index_topk.  A device-side wait that runs out of time (2 s) sets the
+ * array's own sticky error flag (there is no workspace for csa2_device_status
+ * to read); csa2_index_topk_noalloc_status reads it.  Each call clears the flag
+ * before it launches, so the flag reports the last call.
  *
  * The first call on each device looks up the array's device address with that
  * device current (cudaGetSymbolAddress); make that first call before any stream
@@ -356,6 +363,15 @@ CSA2_API csa2_status csa2_layer_step(const csa2_layer_args* a, void* stream);
 CSA2_API csa2_status csa2_index_topk_noalloc(const uint8_t* q, const uint8_t* q_sc, const float* w,
                                              const csa2_kv* kv, const int32_t* q_pos, int32_t B, int32_t Q,
                                              int32_t k, int32_t* idx_out, float* blockmax_out, void* stream);
+
+/*
+ * The error flag of the last csa2_index_topk_noalloc call on the current
+ * device: waits for `stream` (this call synchronises), returns CSA2_ERR_TIMEOUT
+ * if a device-side wait of that call ran out of time (its results are not
+ * valid), else CSA2_OK; CSA2_ERR_CUDA if the copy fails.  With clear != 0 a set
+ * flag is reset on `stream`.  Allocates nothing.
+ */
+CSA2_API csa2_status csa2_index_topk_noalloc_status(int32_t clear, void* stream);
 
 #ifdef __cplusplus
 }

@@ -48,7 +48,7 @@ _lib = None
 EXPORTS = ["csa2_status_str", "csa2_last_cuda_error", "csa2_quant_nvfp4", "csa2_index_k_proj", "csa2_append_tokens",
            "csa2_index_topk",
            "csa2_pool_build", "csa2_pool_topk", "csa2_sparse_attn", "csa2_workspace_bytes", "csa2_layer_step",
-           "csa2_index_topk_noalloc", "csa2_device_status"]
+           "csa2_index_topk_noalloc", "csa2_index_topk_noalloc_status", "csa2_device_status"]
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -77,6 +77,7 @@ def lib():
         "csa2_workspace_bytes": (sz, [ctypes.c_int, i32, i32, i64, i32, i32]),
         "csa2_layer_step": (ctypes.c_int, [ctypes.POINTER(csa2_layer_args), P]),
         "csa2_index_topk_noalloc": (ctypes.c_int, [P, P, P, KVP, P, i32, i32, i32, P, P, P]),
+        "csa2_index_topk_noalloc_status": (ctypes.c_int, [i32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -287,6 +288,12 @@ def csa2_index_topk_noalloc(q, q_sc, w, kv, q_pos, k, idx_out=None, blockmax=Fal
     _check(lib().csa2_index_topk_noalloc(_ptr(q), _ptr(q_sc), _ptr(w), kv.c(), _ptr(q_pos), B, Q, k, _ptr(idx_out),
                                          _ptr(bm), _stream()))
     return (idx_out, bm) if bm is not None else idx_out
+
+
+def csa2_index_topk_noalloc_status(clear=False):
+    """Waits for the current stream; raises CSA2Error (CSA2_ERR_TIMEOUT) if the last
+    csa2_index_topk_noalloc call on this device had a device-side wait run out of time."""
+    _check(lib().csa2_index_topk_noalloc_status(1 if clear else 0, _stream()))
 
 
 def csa2_pool_build(blockmax, kv, q_pos, max_blocks=POOL_BLOCKS, pool_out=None, ws=None):

@@ -304,7 +304,7 @@ int attn_splits(int B, int Q, int k, int window, int* tiles_per_split) {
     int ntiles = (k + window + kKT - 1) / kKT;
     if (ntiles < 1) ntiles = 1;
     int64_t bq = (int64_t)B * Q;
-    int64_t want = (2 * kNumSMs) / (bq > 0 ? bq : 1);
+    int64_t want = (2 * kSplitSMs) / (bq > 0 ? bq : 1);
     if (want < 1) want = 1;
     if (want > ntiles) want = ntiles;
     int tps = (int)((ntiles + want - 1) / want);
@@ -317,7 +317,7 @@ size_t attn_ws_bytes(int B, int Q, int k, int window) {
     // bound the split count over every window <= CSA2_MAX_WINDOW: S <= min(tiles, CTA budget)
     (void)window;
     int64_t bq = (int64_t)B * Q;
-    int64_t want = (2 * kNumSMs) / (bq > 0 ? bq : 1);
+    int64_t want = (2 * kSplitSMs) / (bq > 0 ? bq : 1);
     if (want < 1) want = 1;
     int64_t ntiles_max = (k + CSA2_MAX_WINDOW + kKT - 1) / kKT;
     int64_t S = want < ntiles_max ? want : ntiles_max;
@@ -329,7 +329,7 @@ size_t attn_ws_bytes(int B, int Q, int k, int window) {
 
 void attn_carve_ws(AttnParams& p, int S, void* ws) {
     int64_t bq = (int64_t)p.B * p.Q;
-    int64_t want = (2 * kNumSMs) / (bq > 0 ? bq : 1);
+    int64_t want = (2 * kSplitSMs) / (bq > 0 ? bq : 1);
     if (want < 1) want = 1;
     int64_t ntiles_max = (p.k + CSA2_MAX_WINDOW + kKT - 1) / kKT;
     int64_t Sb = want < ntiles_max ? want : ntiles_max;
@@ -344,13 +344,10 @@ void attn_carve_ws(AttnParams& p, int S, void* ws) {
 }
 
 cudaError_t launch_attn(AttnParams& p, int S, cudaStream_t st) {
-    static bool attr_set = false;
+    static DeviceOnce attr;
     const int smem = (int)sizeof(AttnSmem);
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    cudaError_t e = attr.run([&] { return cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); });
+    if (e != cudaSuccess) return e;
     dim3 grid(S, p.B * p.Q);
     return launch_ex(attn_kernel, grid, dim3(kAT), smem, st, 0, p);
 }

@@ -311,25 +311,31 @@ __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
     }
 }
 
-int g_max_active[17];
-bool g_max_active_known[17];
-bool g_attr_done = false, g_attr_ok = false, g_nonportable = false;
+DeviceOnce g_attr;
+bool g_nonportable[kMaxDevices];
 
 int smem_bytes() { return (int)sizeof(ClAttnSmem); }
 
+// Shared-memory size and (where allowed) 16-CTA clusters, once per device.
 bool set_attributes() {
-    if (g_attr_done) return g_attr_ok;
-    g_attr_done = true;
-    if (cudaFuncSetAttribute(attn_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes()) !=
-        cudaSuccess) {
-        (void)cudaGetLastError();
-        return false;
-    }
-    g_nonportable = cudaFuncSetAttribute(attn_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-                    cudaSuccess;
-    if (!g_nonportable) (void)cudaGetLastError();
-    g_attr_ok = true;
-    return true;
+    return g_attr.run([] {
+        cudaError_t e =
+            cudaFuncSetAttribute(attn_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
+        if (e != cudaSuccess) {
+            (void)cudaGetLastError();
+            return e;
+        }
+        const int d = current_device();
+        g_nonportable[d] =
+            cudaFuncSetAttribute(attn_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+        if (!g_nonportable[d]) (void)cudaGetLastError();
+        return cudaSuccess;
+    }) == cudaSuccess;
+}
+
+bool nonportable() {
+    const int d = current_device();
+    return d >= 0 && d < kMaxDevices && g_nonportable[d];
 }
 
 cudaLaunchConfig_t make_config(int C, int bq, cudaStream_t st, cudaLaunchAttribute* attr) {
@@ -347,18 +353,28 @@ cudaLaunchConfig_t make_config(int C, int bq, cudaStream_t st, cudaLaunchAttribu
     return cfg;
 }
 
-int max_active_clusters(int C, int bq) {
-    if (g_max_active_known[C]) return g_max_active[C];
-    cudaLaunchAttribute attr[1];
-    const cudaLaunchConfig_t cfg = make_config(C, bq, 0, attr);
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, attn_cluster_kernel, &cfg) != cudaSuccess) {
-        (void)cudaGetLastError();
-        n = 0;
-    }
-    g_max_active[C] = n;
-    g_max_active_known[C] = true;
-    return n;
+struct ClusterOcc {
+    int n[17];
+};
+DeviceValue<ClusterOcc> g_occ;
+
+// Clusters of C CTAs that can be resident at once on the current device (0 if refused).
+int max_active_clusters(int C) {
+    const ClusterOcc occ = g_occ.get(
+        [] {
+            ClusterOcc o{};
+            for (int c = 1; c <= (nonportable() ? 16 : 8); c <<= 1) {
+                cudaLaunchAttribute attr[1];
+                const cudaLaunchConfig_t cfg = make_config(c, 1, 0, attr);
+                if (cudaOccupancyMaxActiveClusters(&o.n[c], attn_cluster_kernel, &cfg) != cudaSuccess) {
+                    (void)cudaGetLastError();
+                    o.n[c] = 0;
+                }
+            }
+            return o;
+        },
+        ClusterOcc{});
+    return occ.n[C];
 }
 
 }  // namespace
@@ -366,11 +382,12 @@ int max_active_clusters(int C, int bq) {
 int attn_cluster_size(int B, int Q, int slots_total, int* keys_per_cta) {
     const int bq = B * Q;
     if (bq <= 0 || slots_total <= 0 || !set_attributes()) return 0;
-    for (int C = g_nonportable ? 16 : 8; C >= 1; C >>= 1) {
-        if ((int64_t)bq * C > kNumSMs) continue;
+    const int sms = device_sm_count();
+    for (int C = nonportable() ? 16 : 8; C >= 1; C >>= 1) {
+        if ((int64_t)bq * C > sms) continue;
         const int n = ((slots_total + C - 1) / C + 15) / 16 * 16;
         if (n > kMaxKeys) return 0;   // a smaller cluster only lengthens the chunk
-        if (max_active_clusters(C, bq) >= bq) {
+        if (max_active_clusters(C) >= bq) {
             if (keys_per_cta) *keys_per_cta = n;
             return C;
         }

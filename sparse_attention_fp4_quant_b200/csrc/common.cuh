@@ -13,7 +13,11 @@ constexpr int kH = CSA2_H;
 constexpr int kIH = CSA2_IH;
 constexpr int kID = CSA2_ID;
 constexpr int kBlk = CSA2_BLOCK;
-constexpr int kNumSMs = 148;
+// The CTA budget that split counts are derived from (B200's 148 SMs).  Split
+// counts fix workspace sizes, which callers compute on the host without a
+// device, so this stays a constant; the choice of kernel and cluster size uses
+// the device's own SM count (device_sm_count).
+constexpr int kSplitSMs = 148;
 
 // ---- formats -------------------------------------------------------------
 

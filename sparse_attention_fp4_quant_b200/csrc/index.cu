@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(kNT, 2) select_kernel(SelectParams p) {
 
 // ---- host side -------------------------------------------------------------
 
-static int slots() { return 2 * kNumSMs; }
+static int slots() { return 2 * kSplitSMs; }
 
 int select_splits(int op, int B, int Q, int64_t cap, int k, int P) {
     int64_t bq = (int64_t)B * Q;
@@ -203,15 +203,14 @@ cudaError_t launch_select(int op, SelectParams& p, int S, cudaStream_t st) {
     }
     dim3 grid(S, p.B * p.Q);
     const int smem = (int)sizeof(TK::Smem);
-    static bool attr[3] = {false, false, false};
+    static DeviceOnce attr[3];
     const int mode = op == CSA2_OP_INDEX_TOPK ? 0 : (op == CSA2_OP_POOL_TOPK ? 1 : 2);
-    if (!attr[mode]) {
-        cudaError_t e = mode == 0   ? cudaFuncSetAttribute(select_kernel<MODE_DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
-                        : mode == 1 ? cudaFuncSetAttribute(select_kernel<MODE_POOL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
-                                    : cudaFuncSetAttribute(select_kernel<MODE_BUILD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        attr[mode] = true;
-    }
+    cudaError_t e = attr[mode].run([&] {
+        return mode == 0   ? cudaFuncSetAttribute(select_kernel<MODE_DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+               : mode == 1 ? cudaFuncSetAttribute(select_kernel<MODE_POOL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+                           : cudaFuncSetAttribute(select_kernel<MODE_BUILD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    });
+    if (e != cudaSuccess) return e;
     if (mode == 0) return launch_ex(select_kernel<MODE_DENSE>, grid, dim3(kNT), smem, st, 0, p);
     if (mode == 1) return launch_ex(select_kernel<MODE_POOL>, grid, dim3(kNT), smem, st, 0, p);
     return launch_ex(select_kernel<MODE_BUILD>, grid, dim3(kNT), smem, st, 0, p);

@@ -698,50 +698,64 @@ __global__ void __launch_bounds__(kThreads, 1)
     cl::sync();                                   // no CTA leaves while the cluster may read it
 }
 
-int g_max_active[17];
-bool g_max_active_known[17];
-
-// Clusters of C CTAs that can be resident at once (0 if the size is refused).
-int max_active_clusters(int C, int bq, int smem) {
-    if (g_max_active_known[C]) return g_max_active[C];
-    int n = 0;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(C, bq);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, index_cluster_kernel, &cfg) != cudaSuccess) {
-        (void)cudaGetLastError();
-        n = 0;
-    }
-    g_max_active[C] = n;
-    g_max_active_known[C] = true;
-    return n;
-}
-
 int smem_bytes() { return (int)sizeof(ClSmem) + 1024; }
 
-bool g_attr_done = false;
-bool g_nonportable = false;
+DeviceOnce g_attr;
+bool g_nonportable[kMaxDevices];
 
+// Shared-memory size and (where allowed) 16-CTA clusters, once per device.
 bool set_attributes() {
-    if (g_attr_done) return true;
-    if (cudaFuncSetAttribute(index_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes()) !=
-        cudaSuccess) {
-        (void)cudaGetLastError();
-        return false;
-    }
-    g_nonportable = cudaFuncSetAttribute(index_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-                    cudaSuccess;
-    if (!g_nonportable) (void)cudaGetLastError();
-    g_attr_done = true;
-    return true;
+    return g_attr.run([] {
+        cudaError_t e =
+            cudaFuncSetAttribute(index_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
+        if (e != cudaSuccess) {
+            (void)cudaGetLastError();
+            return e;
+        }
+        const int d = current_device();
+        g_nonportable[d] =
+            cudaFuncSetAttribute(index_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+        if (!g_nonportable[d]) (void)cudaGetLastError();
+        return cudaSuccess;
+    }) == cudaSuccess;
+}
+
+bool nonportable() {
+    const int d = current_device();
+    return d >= 0 && d < kMaxDevices && g_nonportable[d];
+}
+
+struct ClusterOcc {
+    int n[17];
+};
+DeviceValue<ClusterOcc> g_occ;
+
+// Clusters of C CTAs that can be resident at once on the current device (0 if refused).
+int max_active_clusters(int C) {
+    const ClusterOcc occ = g_occ.get(
+        [] {
+            ClusterOcc o{};
+            for (int c = 1; c <= (nonportable() ? 16 : 8); c <<= 1) {
+                cudaLaunchConfig_t cfg = {};
+                cfg.gridDim = dim3(c, 1);
+                cfg.blockDim = dim3(kThreads);
+                cfg.dynamicSmemBytes = smem_bytes();
+                cudaLaunchAttribute attr[1];
+                attr[0].id = cudaLaunchAttributeClusterDimension;
+                attr[0].val.clusterDim.x = c;
+                attr[0].val.clusterDim.y = 1;
+                attr[0].val.clusterDim.z = 1;
+                cfg.attrs = attr;
+                cfg.numAttrs = 1;
+                if (cudaOccupancyMaxActiveClusters(&o.n[c], index_cluster_kernel, &cfg) != cudaSuccess) {
+                    (void)cudaGetLastError();
+                    o.n[c] = 0;
+                }
+            }
+            return o;
+        },
+        ClusterOcc{});
+    return occ.n[C];
 }
 
 }  // namespace
@@ -749,11 +763,12 @@ bool set_attributes() {
 int index_cluster_size(const SelectParams& p) {
     const int bq = p.B * p.Q;
     if (bq <= 0 || !set_attributes()) return 0;
-    for (int C = g_nonportable ? 16 : 8; C >= 1; C >>= 1) {
-        if ((int64_t)bq * C > kNumSMs) continue;
+    const int sms = device_sm_count();
+    for (int C = nonportable() ? 16 : 8; C >= 1; C >>= 1) {
+        if ((int64_t)bq * C > sms) continue;
         const int64_t chunk = ((p.cap + C - 1) / C + kTile - 1) / kTile * kTile;
         if (chunk > (int64_t)kMaxTiles * kTile) return 0;   // a smaller cluster only lengthens the chunk
-        if (max_active_clusters(C, bq, smem_bytes()) >= bq) return C;
+        if (max_active_clusters(C) >= bq) return C;
     }
     return 0;
 }

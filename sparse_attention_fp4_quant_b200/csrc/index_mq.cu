@@ -450,12 +450,12 @@ __global__ void __launch_bounds__(kST) mq_select_kernel(SelectParams p, const ui
     for (int i = (int)K1 + tid; i < k; i += kST) out[i] = -1;
 }
 
-bool g_mq_attr = false;
+DeviceOnce g_mq_attr;
 
 }  // namespace
 
 bool index_mq_eligible(int B, int Q, int64_t cap) {
-    return (int64_t)B * Q > kNumSMs && Q >= kG && cap <= kMaxVis;
+    return (int64_t)B * Q > kSplitSMs && Q >= kG && cap <= kMaxVis;
 }
 
 size_t index_mq_ws_bytes(int B, int Q, int64_t cap) {
@@ -469,14 +469,13 @@ cudaError_t launch_index_mq(SelectParams& p, void* mq_ws, cudaStream_t st) {
     uint32_t* hist = (uint32_t*)((char*)mq_ws + align256(bq * (size_t)p.cap * 2));
     const int smem1 = (int)sizeof(MqSmem) + 1024;
     const int smem2 = (int)sizeof(SelSmem);
-    if (!g_mq_attr) {
-        cudaError_t e = cudaFuncSetAttribute(mq_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(mq_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2);
-        if (e != cudaSuccess) return e;
-        g_mq_attr = true;
-    }
-    cudaError_t e = launch_ex(mq_score_kernel, dim3((p.Q + kG - 1) / kG, p.B), dim3(kMqThreads), smem1, st, 0, p,
+    cudaError_t e = g_mq_attr.run([&] {
+        cudaError_t r = cudaFuncSetAttribute(mq_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
+        if (r == cudaSuccess) r = cudaFuncSetAttribute(mq_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2);
+        return r;
+    });
+    if (e != cudaSuccess) return e;
+    e = launch_ex(mq_score_kernel, dim3((p.Q + kG - 1) / kG, p.B), dim3(kMqThreads), smem1, st, 0, p,
                               prefix, hist);
     if (e != cudaSuccess) return e;
     return launch_ex(mq_select_kernel, dim3((unsigned)bq), dim3(kST), smem2, st, 0, p, (const uint16_t*)prefix,

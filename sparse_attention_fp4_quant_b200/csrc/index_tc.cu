@@ -216,12 +216,10 @@ bool index_tc_supported(const SelectParams& p) {
 template <int MODE, int CAP>
 cudaError_t launch_tc(SelectParams& p, int S, cudaStream_t st) {
     const int smem = (int)sizeof(TcSmem<CAP>) + 1024;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(index_tc_kernel<MODE, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    static DeviceOnce attr;
+    cudaError_t e = attr.run(
+        [&] { return cudaFuncSetAttribute(index_tc_kernel<MODE, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); });
+    if (e != cudaSuccess) return e;
     dim3 grid(S, p.B * p.Q);
     return launch_ex(index_tc_kernel<MODE, CAP>, grid, dim3(kThreads), smem, st, 0, p);
 }

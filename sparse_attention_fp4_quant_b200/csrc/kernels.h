@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include "../../include/csa2.h"
+#include "host_util.h"
 
 namespace csa2 {
 

@@ -2,7 +2,9 @@
 // that cannot allocate device memory.  Its scratch (merge counters and the
 // per-share candidate lists) lives in one file-scope __device__ array of
 // CSA2_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds until
-// the process exits.
+// the process exits.  The array's first 256 bytes hold the call's sticky error
+// flag (read by csa2_index_topk_noalloc_status); the index kernels' scratch
+// follows it.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -15,6 +17,7 @@ using namespace csa2;
 namespace {
 
 constexpr size_t kScratchBytes = CSA2_NOALLOC_SCRATCH_BYTES;
+constexpr size_t kFlagBytes = 256;   // the sticky error flag, then the kernels' scratch
 constexpr int kMaxDevices = 128;
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
@@ -56,12 +59,14 @@ csa2_status csa2_index_topk_noalloc(const uint8_t* q, const uint8_t* q_sc, const
     if (((uintptr_t)q_sc & 3u) || ((uintptr_t)w & 3u)) return CSA2_ERR_INVALID_ARG;
     // the fixed scratch serves the per-share and cluster paths (not the many-query one)
     const size_t need = select_ws_bytes(CSA2_OP_INDEX_TOPK, B, Q, kv->cap, k, 0, false);
-    if (need > kScratchBytes) return CSA2_ERR_WORKSPACE;
-    void* ws = nullptr;
-    cudaError_t e = scratch_on_current_device(&ws);
+    if (need > kScratchBytes - kFlagBytes) return CSA2_ERR_WORKSPACE;
+    void* base = nullptr;
+    cudaError_t e = scratch_on_current_device(&base);
+    void* ws = static_cast<char*>(base) + kFlagBytes;
     if (e == cudaSuccess) {
-        // the merge counters must start at zero; the array keeps the last call's contents
-        e = cudaMemsetAsync(ws, 0, (size_t)B * Q * sizeof(int32_t), (cudaStream_t)stream);
+        // the flag and the merge counters must start at zero, and the array keeps
+        // the last call's contents: clear both (they are adjacent) in one memset
+        e = cudaMemsetAsync(base, 0, kFlagBytes + (size_t)B * Q * sizeof(int32_t), (cudaStream_t)stream);
     }
     if (e == cudaSuccess) {
         SelectParams p{};
@@ -82,6 +87,7 @@ csa2_status csa2_index_topk_noalloc(const uint8_t* q, const uint8_t* q_sc, const
         p.nb_cap = (kv->cap + CSA2_BLOCK - 1) / CSA2_BLOCK;
         const int S = select_splits(CSA2_OP_INDEX_TOPK, B, Q, kv->cap, k, 0);
         select_carve_ws(p, S, ws, B, Q, k, false);
+        p.status = static_cast<int32_t*>(base);   // the fixed flag, not the carved one
         e = launch_select(CSA2_OP_INDEX_TOPK, p, S, (cudaStream_t)stream);
     }
     if (e != cudaSuccess) {
@@ -89,6 +95,20 @@ csa2_status csa2_index_topk_noalloc(const uint8_t* q, const uint8_t* q_sc, const
         return CSA2_ERR_CUDA;
     }
     return CSA2_OK;
+}
+
+csa2_status csa2_index_topk_noalloc_status(int32_t clear, void* stream) {
+    void* base = nullptr;
+    cudaError_t e = scratch_on_current_device(&base);
+    int32_t flag = 0;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&flag, base, sizeof(flag), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e == cudaSuccess && flag && clear) e = cudaMemsetAsync(base, 0, sizeof(flag), (cudaStream_t)stream);
+    if (e != cudaSuccess) {
+        record_cuda_error((int)e);
+        return CSA2_ERR_CUDA;
+    }
+    return flag ? CSA2_ERR_TIMEOUT : CSA2_OK;
 }
 
 }  // extern "C"

@@ -292,12 +292,10 @@ cudaError_t launch_append(const void* x, int64_t rows, const float* W, uint8_t* 
         if (e != cudaSuccess) return e;
         return launch_index_k_proj(x, rows, W, k_codes, k_scales, dst_rows, out_rows, st);
     }
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAppSmem);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    static DeviceOnce attr;
+    cudaError_t e = attr.run(
+        [] { return cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAppSmem); });
+    if (e != cudaSuccess) return e;
     const int nproj = (int)((rows + kAppRows - 1) / kAppRows) * 4;
     const int nquant = (int)((rows * (kD / 16) + kAppThreads - 1) / kAppThreads);
     return launch_ex(append_kernel, dim3(nproj + nquant), dim3(kAppThreads), kAppSmem, st, 0,
@@ -309,13 +307,11 @@ cudaError_t launch_index_k_proj(const void* x, int64_t rows, const float* W, uin
                                 const int64_t* dst_rows, int64_t out_rows, cudaStream_t st) {
     if (rows == 0) return cudaSuccess;
     if (rows <= 2048) {
-        static bool attr = false;
-        if (!attr) {
-            cudaError_t e = cudaFuncSetAttribute(index_k_proj_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 kProjSmem);
-            if (e != cudaSuccess) return e;
-            attr = true;
-        }
+        static DeviceOnce attr;
+        cudaError_t e = attr.run([] {
+            return cudaFuncSetAttribute(index_k_proj_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kProjSmem);
+        });
+        if (e != cudaSuccess) return e;
         return launch_ex(index_k_proj_rows_kernel, dim3((unsigned)((rows + kProjRowsPerCTA - 1) / kProjRowsPerCTA)),
                          dim3(256), kProjSmem, st, 0, static_cast<const uint16_t*>(x), rows, W, k_codes, k_scales,
                          dst_rows, out_rows);

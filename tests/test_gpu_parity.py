@@ -157,6 +157,33 @@ def test_index_topk_many_queries(csa, B, Q):
     assert np.array_equal(np_(bm), rbm)
 
 
+def test_index_topk_many_queries_threshold_bin_overflow(csa):
+    # all-tie queries on the many-query path: with zero query codes or zero head
+    # weights every visible score is +0, so the threshold bin holds every visible
+    # entry (up to 8,000 > the selector's 4,096-entry candidate list) and the
+    # selector resolves it with its re-scoring passes; the other queries are normal
+    B, Q, cap, m = 1, 160, 8192, 1
+    rng = np.random.default_rng(31)
+    q_pos = rng.integers(3000, 8000, size=(B, Q)).astype(np.int32)
+    q_pos[0, :6] = [7999, 4096, 4095, 5000, 100, 0]
+    grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(131, B, Q, cap, [8000], m, q_pos.tolist(), 512)
+    zero_q = [0, 1, 2, 3, 17, 90, 159]
+    zero_w = [4, 5, 40, 41, 150]
+    iq[0, zero_q] = 0
+    oiq = oiq.copy()
+    oiq[0, zero_q] = 0
+    w[0, zero_w] = 0.0
+    ow = np_(w)
+    for k in (512, 2048):
+        idx, bm = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, k, blockmax=True)
+        ridx, rbm = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, m, q_pos, k, blockmax=True)
+        assert np.array_equal(np_(idx), ridx)
+        assert np.array_equal(np_(bm).view(np.uint32), rbm.view(np.uint32))
+        for qi in zero_q + zero_w:
+            nv = min(int(q_pos[0, qi]) + 1, 8000)
+            assert list(np_(idx)[0, qi, :min(k, nv)]) == list(range(min(k, nv)))
+
+
 @pytest.mark.parametrize("n", [128, 129, 255, 1001])
 def test_index_topk_small_ragged_caches(csa, n):
     # visible ranges of a tile, just over one, one short of two, and ragged: the
