@@ -50,6 +50,8 @@ def lib():
         L.orc_pool_topk.argtypes = [P, P, P, P, P, P, i64, i32, P, i32, P, i32, i32, i32, P]
         L.orc_sparse_attn.argtypes = [P, P, P, P, i64, P, i32, P, P, P, i32, i32, P, P,
                                       i32, i32, dbl, P, P]
+        L.orc_front_end_f32.argtypes = [P, i64, P, P, P, ctypes.c_float, P]
+        L.orc_front_end.argtypes = [P, i64, P, P, P, ctypes.c_float, P]
         _lib = L
     return _lib
 
@@ -99,6 +101,25 @@ def dequant_nvfp4(packed, scales):
     ch = packed.shape[-1] * 2
     out = np.zeros((rows, ch), np.float64)
     lib().orc_dequant_nvfp4(_p(packed), _p(scales), rows, ch, _p(out))
+    return out
+
+
+# ---------------------------------------------------------------- front end
+def front_end(x_bf16, cos, sin, w=None, eps=1e-6, f32=False):
+    """RMSNorm (eps, optional per-channel weight) then RoPE on channels 448..511 (pairs
+    (448 + 2k, 449 + 2k) with the caller's cos/sin [rows, 32]) of bf16 latents [rows, 512]:
+    bf16 bits [rows, 512] (or the fp32 values before the bf16 rounding with f32=True)."""
+    x = _c(x_bf16, np.uint16).reshape(-1, D)
+    rows = x.shape[0]
+    cos = _c(cos, np.float32).reshape(rows, 32)
+    sin = _c(sin, np.float32).reshape(rows, 32)
+    wv = None if w is None else _c(w, np.float32).reshape(D)
+    if f32:
+        out = np.zeros((rows, D), np.float32)
+        lib().orc_front_end_f32(_p(x), rows, _p(cos), _p(sin), _p(wv), float(eps), _p(out))
+    else:
+        out = np.zeros((rows, D), np.uint16)
+        lib().orc_front_end(_p(x), rows, _p(cos), _p(sin), _p(wv), float(eps), _p(out))
     return out
 
 

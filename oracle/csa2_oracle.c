@@ -149,6 +149,67 @@ void orc_dequant_nvfp4(const uint8_t* packed, const uint8_t* scales, int64_t row
 }
 
 /* ------------------------------------------------------------------------ */
+/* Front end of a new main-KV latent.  [Jdon] "缓存压缩真的是越大越好吗": the   */
+/* latent is RMSNorm'd (weight at most about 1, so its L2 norm is at most      */
+/* about sqrt(512)) and RoPE preserves that norm; [Blog] "FP4 与 SWA Bounded     */
+/* Replay" and [Lsln] 4.3: it is quantised after RoPE.  The fp32 order below is */
+/* this implementation's reading (the pages give none):                         */
+/*   ss   = fused multiply-add chain of x_c * x_c over c = 0..511 from +0       */
+/*   r    = 1 / sqrt(ss / 512 + eps)   (each step one IEEE fp32 rounding)       */
+/*   n_c  = (x_c * r) * w_c            (two rounded products)                   */
+/*   RoPE on the pairs (448 + 2k, 449 + 2k), k = 0..31, with the caller's       */
+/*   cos_k, sin_k:  a' = a cos - b sin,  b' = a sin + b cos  (products rounded, */
+/*   then one rounded add / subtract)                                           */
+/*   y_c  = n_c rounded to bf16 (nearest, ties to even)                         */
+/* ------------------------------------------------------------------------ */
+
+static uint16_t f32_to_bf16_rne(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7F800000u) == 0x7F800000u) return (uint16_t)((u >> 16) | ((u & 0xFFFFu) ? 0x40u : 0u));  /* inf / nan */
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7FFFu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+void orc_front_end_f32(const uint16_t* x, int64_t rows, const float* cos_t, const float* sin_t, const float* w,
+                       float eps, float* out) {
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t* xr = x + r * ORC_D;
+        float ss = 0.0f;
+        for (int c = 0; c < ORC_D; ++c) {
+            float v = bf16_to_f32(xr[c]);
+            ss = fmaf(v, v, ss);
+        }
+        float mean = ss / 512.0f;
+        float t = mean + eps;
+        float s = sqrtf(t);
+        float inv = 1.0f / s;
+        float* o = out + r * ORC_D;
+        for (int c = 0; c < ORC_D; ++c) {
+            float n = bf16_to_f32(xr[c]) * inv;
+            o[c] = n * (w ? w[c] : 1.0f);
+        }
+        for (int k = 0; k < 32; ++k) {
+            float a = o[448 + 2 * k], b = o[449 + 2 * k];
+            float cs = cos_t[r * 32 + k], sn = sin_t[r * 32 + k];
+            float ac = a * cs, bs = b * sn, as = a * sn, bc = b * cs;   /* separate roundings: no contraction */
+            o[448 + 2 * k] = ac - bs;
+            o[449 + 2 * k] = as + bc;
+        }
+    }
+}
+
+void orc_front_end(const uint16_t* x, int64_t rows, const float* cos_t, const float* sin_t, const float* w,
+                   float eps, uint16_t* y) {
+    float buf[ORC_D];
+    for (int64_t r = 0; r < rows; ++r) {
+        orc_front_end_f32(x + r * ORC_D, 1, cos_t + r * 32, sin_t + r * 32, w, eps, buf);
+        for (int c = 0; c < ORC_D; ++c) y[r * ORC_D + c] = f32_to_bf16_rne(buf[c]);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Indexer.  [Blog] "CSA2" section: a lightweight indexer scores the main KV  */
 /* with indexer Q/K and keeps the Top-K (512); the indexer K is projected     */
 /* from the main KV.  [Blog] "FP4 与 SWA Bounded Replay": indexer Q/K in FP4.  */

@@ -55,6 +55,12 @@ void orc_pool_topk(const uint8_t* q, const uint8_t* qs, const float* w,
                    const uint8_t* ik, const uint8_t* iks, const int32_t* n_entries, int64_t cap, int m,
                    const int32_t* pool, int P, const int32_t* q_pos, int B, int Q, int k, int32_t* idx_out);
 
+/* front end: RMSNorm + RoPE of a new latent (fp32 values, then bf16) */
+void orc_front_end_f32(const uint16_t* x, int64_t rows, const float* cos_t, const float* sin_t, const float* w,
+                       float eps, float* out);
+void orc_front_end(const uint16_t* x, int64_t rows, const float* cos_t, const float* sin_t, const float* w,
+                   float eps, uint16_t* y);
+
 /* attention */
 void orc_sparse_attn(const uint16_t* q, const uint8_t* lat, const uint8_t* lat_sc,
                      const int32_t* n_entries, int64_t cap, const int32_t* idx, int k,
