@@ -89,6 +89,19 @@ CSA2_API const char* csa2_status_str(csa2_status s);
 CSA2_API int csa2_last_cuda_error(void);
 
 /*
+ * Test hook for the device-side timeout path (the pages have no counterpart).
+ * While enabled (enable != 0; process-wide, off by default), index calls that
+ * run the per-share scoring kernel (csa2_index_topk and
+ * csa2_index_topk_noalloc for more queries than one wave of clusters holds,
+ * with fewer than 8 per batch row) announce their first copy stage on its
+ * barrier but issue no copy, so the CTAs' bounded waits (2 s) run out: the call
+ * sets its sticky error flag (read by csa2_device_status or
+ * csa2_index_topk_noalloc_status) and its results are not valid.  Nothing
+ * faults or hangs; the context stays usable.
+ */
+CSA2_API void csa2_test_starve_copies(int32_t enable);
+
+/*
  * The shared global KV of one CSA2 layer group: the FP4 main latent and the FP4
  * indexer K, both written by the group's Full layer and borrowed by its
  * Reindex and Reuse layers ([Blog] "CSA2" section, Fig. 4).
@@ -161,6 +174,33 @@ CSA2_API csa2_status csa2_index_k_proj(const void* x, int64_t rows, const float*
 CSA2_API csa2_status csa2_append_tokens(const void* x, int64_t rows, const float* W, uint8_t* lat_codes,
                                         uint8_t* lat_scales, uint8_t* k_codes, uint8_t* k_scales,
                                         const int64_t* dst_rows, int64_t out_rows, void* stream);
+
+/*
+ * Front end of new main-KV entries: RMSNorm and RoPE, then the append's
+ * quantisation, in one launch ([Jdon] "缓存压缩真的是越大越好吗": the latent is
+ * RMSNorm'd, so its L2 norm is at most about sqrt(512), and RoPE keeps that
+ * norm; [Blog] FP4 section: the latent is quantised after RoPE; [Blog] "CSA2"
+ * section: the indexer K is projected from the main KV).  For each row, in fp32
+ * with one IEEE rounding per step:
+ *   ss  = fused multiply-add chain of x_c * x_c over c = 0..511, from +0
+ *   r   = 1 / sqrt(ss / 512 + eps);   n_c = (x_c * r) * w_c
+ *   for k = 0..31, (a, b) = (n_{448+2k}, n_{449+2k}):
+ *         a' = a cos_k - b sin_k;   b' = a sin_k + b cos_k   (products rounded first)
+ *   y   = n rounded to bf16 (nearest, ties to even)
+ * then the bytes csa2_append_tokens(y, ...) writes (NVFP4 latent; projected,
+ * quantised indexer K).
+ *   x         device bf16 [rows][512] pre-norm latent rows, 16-byte aligned
+ *   rope_cos, rope_sin  device fp32 [rows][32]: cos and sin of each row's 32 angles
+ *   norm_w    device fp32 [512] RMSNorm weight, or NULL for weight 1
+ *   eps       RMSNorm epsilon (1e-6 in the synthetic workloads)
+ *   W, lat_codes, lat_scales, k_codes, k_scales, dst_rows, out_rows: as for
+ *             csa2_append_tokens (out_rows a multiple of 128)
+ *   y_out     device bf16 [rows][512] (16-byte aligned) receiving y, or NULL
+ */
+CSA2_API csa2_status csa2_front_end(const void* x, int64_t rows, const float* rope_cos, const float* rope_sin,
+                                   const float* norm_w, float eps, const float* W, uint8_t* lat_codes,
+                                   uint8_t* lat_scales, uint8_t* k_codes, uint8_t* k_scales, const int64_t* dst_rows,
+                                   int64_t out_rows, void* y_out, void* stream);
 
 /*
  * Step 2 -- FP4 index scoring + Top-K ([Blog] "CSA2" section: a lightweight

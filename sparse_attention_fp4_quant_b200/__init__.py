@@ -48,7 +48,8 @@ _lib = None
 EXPORTS = ["csa2_status_str", "csa2_last_cuda_error", "csa2_quant_nvfp4", "csa2_index_k_proj", "csa2_append_tokens",
            "csa2_index_topk",
            "csa2_pool_build", "csa2_pool_topk", "csa2_sparse_attn", "csa2_workspace_bytes", "csa2_layer_step",
-           "csa2_index_topk_noalloc", "csa2_index_topk_noalloc_status", "csa2_device_status"]
+           "csa2_index_topk_noalloc", "csa2_index_topk_noalloc_status", "csa2_device_status", "csa2_front_end",
+           "csa2_test_starve_copies"]
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -78,6 +79,8 @@ def lib():
         "csa2_layer_step": (ctypes.c_int, [ctypes.POINTER(csa2_layer_args), P]),
         "csa2_index_topk_noalloc": (ctypes.c_int, [P, P, P, KVP, P, i32, i32, i32, P, P, P]),
         "csa2_index_topk_noalloc_status": (ctypes.c_int, [i32, P]),
+        "csa2_test_starve_copies": (None, [i32]),
+        "csa2_front_end": (ctypes.c_int, [P, i64, P, P, P, ctypes.c_float, P, P, P, P, P, P, i64, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -242,6 +245,35 @@ def csa2_append_tokens(x, W, kv_or_outs, dst_rows=None):
         _size(_dev(t, torch.uint8, n), out_rows * per, n)
     _check(lib().csa2_append_tokens(_ptr(x), rows, _ptr(W), _ptr(lc), _ptr(ls), _ptr(kc), _ptr(ks), _ptr(dst_rows),
                                     out_rows, _stream()))
+
+
+def csa2_front_end(x, rope_cos, rope_sin, W, kv_or_outs, dst_rows=None, norm_w=None, eps=1e-6, y_out=None):
+    """Pre-norm bf16 rows x [rows, 512] -> RMSNorm, RoPE (fp32 cos/sin [rows, 32]), bf16, then the
+    append's bytes into a KV (or a tuple (lat_codes, lat_scales, k_codes, k_scales)); y_out, if given,
+    receives the post-RoPE bf16 rows."""
+    _dev(x, torch.bfloat16, "x")
+    rows = x.numel() // D
+    _size(x, rows * D, "x")
+    _size(_dev(rope_cos, torch.float32, "rope_cos"), rows * 32, "rope_cos")
+    _size(_dev(rope_sin, torch.float32, "rope_sin"), rows * 32, "rope_sin")
+    _size(_dev(W, torch.float32, "W"), D * ID, "W")
+    if norm_w is not None:
+        _size(_dev(norm_w, torch.float32, "norm_w"), D, "norm_w")
+    if isinstance(kv_or_outs, KV):
+        lc, ls, kc, ks = kv_or_outs.lat, kv_or_outs.lat_sc, kv_or_outs.ik, kv_or_outs.ik_sc
+    else:
+        lc, ls, kc, ks = kv_or_outs
+    out_rows = lc.numel() // (D // 2)
+    for t, n, per in ((lc, "lat_codes", D // 2), (ls, "lat_scales", D // 16), (kc, "k_codes", ID // 2),
+                      (ks, "k_scales", ID // 16)):
+        _size(_dev(t, torch.uint8, n), out_rows * per, n)
+    if dst_rows is not None:
+        _size(_dev(dst_rows, torch.int64, "dst_rows"), rows, "dst_rows")
+    if y_out is not None:
+        _size(_dev(y_out, torch.bfloat16, "y_out"), rows * D, "y_out")
+    _check(lib().csa2_front_end(_ptr(x), rows, _ptr(rope_cos), _ptr(rope_sin), _ptr(norm_w), float(eps), _ptr(W),
+                                _ptr(lc), _ptr(ls), _ptr(kc), _ptr(ks), _ptr(dst_rows), out_rows, _ptr(y_out),
+                                _stream()))
 
 
 def csa2_index_topk(q, q_sc, w, kv, q_pos, k, idx_out=None, blockmax=False, ws=None):

@@ -2,6 +2,8 @@
 // workspace sizing, launch, and the per-layer mode dispatch.
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "../../include/csa2.h"
 #include "kernels.h"
 
@@ -10,6 +12,7 @@ using namespace csa2;
 namespace {
 
 thread_local int g_last_cuda_error = 0;
+std::atomic<int> g_test_starve{0};
 
 csa2_status cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return CSA2_OK;
@@ -50,6 +53,7 @@ SelectParams select_params(const csa2_kv* kv, const int32_t* q_pos, int B, int Q
 
 namespace csa2 {
 void record_cuda_error(int e) { g_last_cuda_error = e; }
+int test_starve_copies() { return g_test_starve.load(std::memory_order_relaxed); }
 }  // namespace csa2
 
 extern "C" {
@@ -67,6 +71,8 @@ const char* csa2_status_str(csa2_status s) {
 }
 
 int csa2_last_cuda_error(void) { return g_last_cuda_error; }
+
+void csa2_test_starve_copies(int32_t enable) { g_test_starve.store(enable ? 1 : 0, std::memory_order_relaxed); }
 
 csa2_status csa2_quant_nvfp4(const void* x, int64_t rows, int32_t ch, uint8_t* codes, uint8_t* scales,
                              const int64_t* dst_rows, int64_t out_rows, void* stream) {
@@ -133,6 +139,22 @@ size_t csa2_workspace_bytes(csa2_op op, int32_t B, int32_t Q, int64_t cap, int32
     return 0;
 }
 
+csa2_status csa2_front_end(const void* x, int64_t rows, const float* rope_cos, const float* rope_sin,
+                           const float* norm_w, float eps, const float* W, uint8_t* lat_codes, uint8_t* lat_scales,
+                           uint8_t* k_codes, uint8_t* k_scales, const int64_t* dst_rows, int64_t out_rows, void* y_out,
+                           void* stream) {
+    if (rows < 0) return CSA2_ERR_INVALID_ARG;
+    if (rows == 0) return CSA2_OK;
+    if (!x || !rope_cos || !rope_sin || !W || !lat_codes || !lat_scales || !k_codes || !k_scales || !aligned16(x) ||
+        !aligned16(W) || ((uintptr_t)lat_codes & 7u) || ((uintptr_t)k_codes & 7u) || ((uintptr_t)rope_cos & 3u) ||
+        ((uintptr_t)rope_sin & 3u) || ((uintptr_t)norm_w & 3u) || (y_out && !aligned16(y_out)))
+        return CSA2_ERR_INVALID_ARG;
+    if (!(eps == eps)) return CSA2_ERR_INVALID_ARG;
+    if (out_rows < 0 || out_rows % 128 != 0 || (!dst_rows && out_rows < rows)) return CSA2_ERR_INVALID_ARG;
+    return cuda_status(launch_front_end(x, rows, rope_cos, rope_sin, norm_w, eps, W, lat_codes, lat_scales, k_codes,
+                                        k_scales, dst_rows, out_rows, y_out, (cudaStream_t)stream));
+}
+
 csa2_status csa2_index_topk(const uint8_t* q, const uint8_t* q_sc, const float* w, const csa2_kv* kv,
                             const int32_t* q_pos, int32_t B, int32_t Q, int32_t k, int32_t* idx_out,
                             float* blockmax_out, void* ws, size_t ws_bytes, void* stream) {
@@ -146,6 +168,7 @@ csa2_status csa2_index_topk(const uint8_t* q, const uint8_t* q_sc, const float* 
     p.w = w;
     p.out = idx_out;
     p.blockmax = blockmax_out;
+    p.test_starve = test_starve_copies();
     int S = select_splits(CSA2_OP_INDEX_TOPK, B, Q, kv->cap, k, 0);
     select_carve_ws(p, S, ws, B, Q, k);
     return cuda_status(launch_select(CSA2_OP_INDEX_TOPK, p, S, (cudaStream_t)stream));
@@ -217,10 +240,12 @@ csa2_status csa2_sparse_attn(const void* q, const csa2_kv* kv, const int32_t* id
     p.out = static_cast<uint16_t*>(out);
     p.lse = lse;
     p.slots_total = k + window;
-    const int C = attn_cluster_size(B, Q, p.slots_total, &p.keys_per_cta);
-    if (C > 0) return cuda_status(launch_attn_cluster(p, C, (cudaStream_t)stream));
     int S = attn_splits(B, Q, k, window, &p.tiles_per_split);
     attn_carve_ws(p, S, ws);
+    const int Ct = attn_tc_cluster_size(B, Q, k, window, &p.main_per_cta, &p.swa_per_cta);
+    if (Ct > 0) return cuda_status(launch_attn_tc(p, Ct, (cudaStream_t)stream));
+    const int C = attn_cluster_size(B, Q, p.slots_total, &p.keys_per_cta);
+    if (C > 0) return cuda_status(launch_attn_cluster(p, C, (cudaStream_t)stream));
     return cuda_status(launch_attn(p, S, (cudaStream_t)stream));
 }
 

@@ -322,7 +322,7 @@ size_t attn_ws_bytes(int B, int Q, int k, int window) {
     int64_t ntiles_max = (k + CSA2_MAX_WINDOW + kKT - 1) / kKT;
     int64_t S = want < ntiles_max ? want : ntiles_max;
     size_t ubq = (size_t)bq;
-    size_t bytes = align256(ubq * 4);
+    size_t bytes = align256(ubq * 4) + 256;   // counters, status word
     if (S > 1) bytes += align256(ubq * S * kH * kD * 4) + align256(ubq * S * kH * 2 * 4);
     return bytes;
 }
@@ -336,6 +336,8 @@ void attn_carve_ws(AttnParams& p, int S, void* ws) {
     char* c = (char*)ws;
     p.counters = (int32_t*)c;
     c += align256((size_t)bq * 4);
+    p.status = (int32_t*)c;
+    c += 256;
     if (S > 1) {
         p.part_o = (float*)c;
         c += align256((size_t)bq * Sb * kH * kD * 4);

@@ -112,12 +112,21 @@ __device__ __forceinline__ void setup_query(P& s, const uint8_t* q, const uint8_
 // the cache stores each 128-entry tile as the MMA's operand image and the
 // scales row-major, so a stage is one contiguous bulk copy of its tiles' codes
 // and one of their scales.  Lane 0 issues.
+//
+// With `starve` (a test hook) the first stage's bytes are announced on its
+// barrier but no copy is issued, so nothing ever completes that barrier: every
+// wait on it runs out of time and the CTA winds down through its error path.
 template <class P>
 __device__ __forceinline__ void producer_dense(P& s, const uint8_t* ik, const uint8_t* iks, int64_t row_base, int lo,
-                                               int ntiles, int nstages, int32_t* status, int lane) {
+                                               int ntiles, int nstages, int32_t* status, int lane, bool starve = false) {
     constexpr int kStages = P::kStages;
     int issued = 0;
     if (lane == 0) {
+        if (starve && nstages > 0) {
+            tc::mbar_arrive_expect_tx(&s.full[0], (uint32_t)min(kTPS, ntiles) * (kTile * 32u + kTile * 4u));
+            issued = 1;
+            nstages = 0;
+        }
         for (int t = 0; t < nstages; ++t) {
             const int slot = t % kStages;
             const uint32_t ph = (uint32_t)(t / kStages) & 1u;

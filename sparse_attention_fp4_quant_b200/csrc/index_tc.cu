@@ -79,7 +79,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     int32_t* status = p.status;
 
     if (warp == 0) {
-        if (MODE == 0) producer_dense(s.pipe, p.ik, p.ik_sc, row_base, lo, ntiles, nstages, status, lane);
+        if (MODE == 0)
+            producer_dense(s.pipe, p.ik, p.ik_sc, row_base, lo, ntiles, nstages, status, lane, p.test_starve != 0);
         else producer_pool(s.pipe, p.ik, p.ik_sc, row_base, lo, hi, ntiles, nstages, pool, nvis, status, lane);
     } else if (warp == 1) {
         mma_issuer(s.pipe, ntiles, nstages, status, lane);

@@ -65,7 +65,11 @@ struct SelectParams {
     uint32_t* cand_key;    // [B*Q][S][k]
     int32_t* cand_pos;     // [B*Q][S][k]
     void* mq_ws;           // index Top-K for many queries: key prefixes and histograms (else null)
+    int test_starve;       // test hook (csa2_test_starve_copies): the per-share producer issues no copies
 };
+
+// The test hook's current setting (read by the index entry points).
+int test_starve_copies();
 
 int select_splits(int op, int B, int Q, int64_t cap, int k, int P);
 // mq = false leaves out the many-query index path's part (a fixed scratch that may not hold it)
@@ -90,6 +94,10 @@ cudaError_t launch_index_k_proj(const void* x, int64_t rows, const float* W, uin
 cudaError_t launch_append(const void* x, int64_t rows, const float* W, uint8_t* lat_codes, uint8_t* lat_scales,
                           uint8_t* k_codes, uint8_t* k_scales, const int64_t* dst_rows, int64_t out_rows,
                           cudaStream_t st);
+cudaError_t launch_front_end(const void* x, int64_t rows, const float* rcos, const float* rsin, const float* nw,
+                             float eps, const float* W, uint8_t* lat_codes, uint8_t* lat_scales, uint8_t* k_codes,
+                             uint8_t* k_scales, const int64_t* dst_rows, int64_t out_rows, void* y_out,
+                             cudaStream_t st);
 
 // Sparse attention.
 struct AttnParams {
@@ -113,8 +121,11 @@ struct AttnParams {
     int slots_total;          // k + window
     int tiles_per_split;      // split-K form: 64-key tiles per split
     int keys_per_cta;         // cluster form: key slots per CTA
+    int main_per_cta;         // tensor-core cluster form: main slots per CTA
+    int swa_per_cta;          // tensor-core cluster form: window slots per CTA
     // workspace
     int32_t* counters;        // [B*Q]
+    int32_t* status;          // sticky: set to 1 if a device-side wait timed out
     float* part_o;            // [B*Q][S][16][512]
     float* part_ml;           // [B*Q][S][16][2]
 };
@@ -126,5 +137,8 @@ cudaError_t launch_attn(AttnParams& p, int S, cudaStream_t st);
 // One cluster of C CTAs per query; 0 = the shape does not fit.
 int attn_cluster_size(int B, int Q, int slots_total, int* keys_per_cta);
 cudaError_t launch_attn_cluster(AttnParams& p, int C, cudaStream_t st);
+// The same on the 5th-generation tensor cores (attn_tc.cu); 0 = the shape does not fit.
+int attn_tc_cluster_size(int B, int Q, int k, int window, int* main_per_cta, int* swa_per_cta);
+cudaError_t launch_attn_tc(AttnParams& p, int C, cudaStream_t st);
 
 }  // namespace csa2

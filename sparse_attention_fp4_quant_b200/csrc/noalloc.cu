@@ -85,6 +85,7 @@ csa2_status csa2_index_topk_noalloc(const uint8_t* q, const uint8_t* q_sc, const
         p.out = idx_out;
         p.blockmax = blockmax_out;
         p.nb_cap = (kv->cap + CSA2_BLOCK - 1) / CSA2_BLOCK;
+        p.test_starve = test_starve_copies();
         const int S = select_splits(CSA2_OP_INDEX_TOPK, B, Q, kv->cap, k, 0);
         select_carve_ws(p, S, ws, B, Q, k, false);
         p.status = static_cast<int32_t*>(base);   // the fixed flag, not the carved one

@@ -322,3 +322,190 @@ cudaError_t launch_index_k_proj(const void* x, int64_t rows, const float* W, uin
 }
 
 }  // namespace csa2
+
+namespace csa2 {
+
+// ---- fused front end --------------------------------------------------------
+// RMSNorm + RoPE of new pre-norm latent rows, bf16 rounding, NVFP4 quantisation
+// of the result and its indexer-K projection + quantisation, in one launch
+// ([Jdon] "缓存压缩真的是越大越好吗": the latent is RMSNorm'd and RoPE keeps its
+// norm; [Blog] "FP4 与 SWA Bounded Replay": quantised after RoPE; [Blog] "CSA2"
+// section: the indexer K is projected from the main KV).  fp32 order, each step
+// one IEEE rounding: ss = fused multiply-add chain of x_c^2 over c ascending;
+// r = 1 / sqrt(ss / 512 + eps); n_c = (x_c r) w_c; pairs (448 + 2k, 449 + 2k):
+// a' = a cos - b sin, b' = a sin + b cos with rounded products; y = bf16(n).
+// Then the bytes of csa2_quant_nvfp4(y) and csa2_index_k_proj(y).
+//
+// A CTA takes 64 rows (256 threads): the bf16 rows are staged in shared memory
+// (row stride 1040 B), 64 threads run the rows' sum-of-squares chains, every
+// thread normalises and rotates 16-byte chunks in place, quantises 16-channel
+// groups, and the projection runs as 4 x 4 register tiles of chains over 32-
+// channel chunks of W, as index_k_proj_kernel does.
+constexpr int kFR = 64;                 // rows per CTA
+constexpr int kFXS = kD + 8;            // bf16 per staged row (16 B pad)
+constexpr int kFrontSmem = kFR * kFXS * 2 + kPC * (kID + 4) * 4 + kFR * (kID + 4) * 4 + kFR * 4;
+
+__global__ void __launch_bounds__(256) front_end_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                        const float* __restrict__ rcos, const float* __restrict__ rsin,
+                                                        const float* __restrict__ nw, float eps,
+                                                        const float* __restrict__ W, uint8_t* __restrict__ lc,
+                                                        uint8_t* __restrict__ ls, uint8_t* __restrict__ kc,
+                                                        uint8_t* __restrict__ ks, const int64_t* __restrict__ dst_rows,
+                                                        int64_t out_rows, uint16_t* __restrict__ y_out) {
+    pdl_enter();
+    extern __shared__ __align__(16) uint8_t fe_smem[];
+    uint16_t* xs = reinterpret_cast<uint16_t*>(fe_smem);                                  // [64][kFXS] bf16
+    float* wsm = reinterpret_cast<float*>(fe_smem + kFR * kFXS * 2);                      // [32][68]
+    float* outs = wsm + kPC * (kID + 4);                                                  // [64][68]
+    float* inv = outs + kFR * (kID + 4);                                                  // [64]
+    const int tid = threadIdx.x;
+    const int64_t r0 = (int64_t)blockIdx.x * kFR;
+    const int nr = (int)min((int64_t)kFR, rows - r0);
+
+    // stage the rows (16 B per thread and step; rows past the end are zero)
+    for (int i = tid; i < kFR * (kD / 8); i += 256) {
+        const int rr = i / (kD / 8), q = i % (kD / 8);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (rr < nr) v = __ldg(reinterpret_cast<const uint4*>(x + (r0 + rr) * kD) + q);
+        *reinterpret_cast<uint4*>(xs + rr * kFXS + 8 * q) = v;
+    }
+    __syncthreads();
+    // sum of squares: one chain per row, channels ascending
+    if (tid < kFR) {
+        const uint16_t* xr = xs + tid * kFXS;
+        float ss = 0.0f;
+#pragma unroll 8
+        for (int c = 0; c < kD; ++c) {
+            const float v = __uint_as_float((uint32_t)xr[c] << 16);
+            ss = __fmaf_rn(v, v, ss);
+        }
+        const float t = __fadd_rn(__fdiv_rn(ss, 512.0f), eps);
+        inv[tid] = __fdiv_rn(1.0f, __fsqrt_rn(t));
+    }
+    __syncthreads();
+    // normalise, rotate, round to bf16 in place: 16-byte chunk q (channels 8q .. 8q + 7) of row rr
+    for (int i = tid; i < kFR * (kD / 8); i += 256) {
+        const int rr = i / (kD / 8), q = i % (kD / 8);
+        uint4* p = reinterpret_cast<uint4*>(xs + rr * kFXS + 8 * q);
+        const uint4 v = *p;
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+        const float r = inv[rr];
+        float n[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            n[2 * j] = __fmul_rn(__uint_as_float(u[j] << 16), r);
+            n[2 * j + 1] = __fmul_rn(__uint_as_float(u[j] & 0xFFFF0000u), r);
+        }
+        if (nw) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) n[j] = __fmul_rn(n[j], __ldg(nw + 8 * q + j));
+        }
+        if (q >= 56 && rr < nr) {   // channels 448 .. 511: pairs k = 4 (q - 56) .. + 3
+            const float* cs = rcos + (r0 + rr) * 32 + 4 * (q - 56);
+            const float* sn = rsin + (r0 + rr) * 32 + 4 * (q - 56);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float a = n[2 * j], b = n[2 * j + 1], c = __ldg(cs + j), s = __ldg(sn + j);
+                n[2 * j] = __fsub_rn(__fmul_rn(a, c), __fmul_rn(b, s));
+                n[2 * j + 1] = __fadd_rn(__fmul_rn(a, s), __fmul_rn(b, c));
+            }
+        }
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t lo = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(n[2 * j]));
+            const uint32_t hi = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(n[2 * j + 1]));
+            o[j] = lo | (hi << 16);
+        }
+        const uint4 ov = make_uint4(o[0], o[1], o[2], o[3]);
+        *p = ov;
+        if (y_out && rr < nr) *reinterpret_cast<uint4*>(y_out + (r0 + rr) * kD + 8 * q) = ov;
+    }
+    __syncthreads();
+    // main latent -> NVFP4: one thread per (row, 16-channel group)
+    for (int i = tid; i < kFR * (kD / 16); i += 256) {
+        const int rr = i / (kD / 16), g = i % (kD / 16);
+        if (rr >= nr) continue;
+        const uint4* src = reinterpret_cast<const uint4*>(xs + rr * kFXS + 16 * g);
+        const uint4 a = src[0], b = src[1];
+        const uint32_t u[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            v[2 * j] = __uint_as_float(u[j] << 16);
+            v[2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
+        }
+        uint32_t sc, lo, hi;
+        quant16(v, sc, lo, hi);
+        const int64_t orow = dst_rows ? __ldg(dst_rows + r0 + rr) : r0 + rr;
+        if (orow < 0 || orow >= out_rows) continue;
+        *reinterpret_cast<uint2*>(lc + orow * (kD / 2) + 8 * g) = make_uint2(lo, hi);
+        ls[orow * (kD / 16) + g] = (uint8_t)sc;
+    }
+    // indexer-K projection of the bf16 rows: 4 x 4 chains per thread, channels ascending
+    const int ty = tid >> 4, tx = tid & 15;
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+    for (int c0 = 0; c0 < kD; c0 += kPC) {
+        __syncthreads();   // the previous chunk of W is consumed (and, first time, the bf16 rows are final)
+#pragma unroll
+        for (int it = 0; it < (kPC * kID) / 256; ++it) {
+            const int e = it * 256 + tid;
+            const int cc = e / kID, jj = e % kID;
+            wsm[cc * (kID + 4) + jj] = __ldg(W + (int64_t)(c0 + cc) * kID + jj);
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int cc = 0; cc < kPC; ++cc) {
+            float a[4], bw[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = __uint_as_float((uint32_t)xs[(ty * 4 + i) * kFXS + c0 + cc] << 16);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) bw[j] = wsm[cc * (kID + 4) + tx * 4 + j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = __fmaf_rn(a[i], bw[j], acc[i][j]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) outs[(ty * 4 + i) * (kID + 4) + tx * 4 + j] = acc[i][j];
+    __syncthreads();
+    {
+        const int rr = tid >> 2, g = tid & 3;
+        if (rr < nr) {
+            float v[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = outs[rr * (kID + 4) + 16 * g + j];
+            uint32_t sc, lo, hi;
+            quant16(v, sc, lo, hi);
+            const int64_t orow = dst_rows ? __ldg(dst_rows + r0 + rr) : r0 + rr;
+            if (orow >= 0 && orow < out_rows) {
+                *reinterpret_cast<uint2*>(kc + ik_code_off(orow, g >> 1) + 8 * (g & 1)) = make_uint2(lo, hi);
+                ks[ik_scale_off(orow) + g] = (uint8_t)sc;
+            }
+        }
+    }
+}
+
+cudaError_t launch_front_end(const void* x, int64_t rows, const float* rcos, const float* rsin, const float* nw,
+                             float eps, const float* W, uint8_t* lat_codes, uint8_t* lat_scales, uint8_t* k_codes,
+                             uint8_t* k_scales, const int64_t* dst_rows, int64_t out_rows, void* y_out,
+                             cudaStream_t st) {
+    if (rows == 0) return cudaSuccess;
+    static DeviceOnce attr;
+    cudaError_t e = attr.run(
+        [] { return cudaFuncSetAttribute(front_end_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFrontSmem); });
+    if (e != cudaSuccess) return e;
+    const int64_t blocks = (rows + kFR - 1) / kFR;
+    return launch_ex(front_end_kernel, dim3((unsigned)blocks), dim3(256), kFrontSmem, st, 0,
+                     static_cast<const uint16_t*>(x), rows, rcos, rsin, nw, eps, W, lat_codes, lat_scales, k_codes,
+                     k_scales, dst_rows, out_rows, static_cast<uint16_t*>(y_out));
+}
+
+}  // namespace csa2

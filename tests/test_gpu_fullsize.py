@@ -213,32 +213,47 @@ def test_c3_prefill_chunk_m2(csa):
 
 
 def test_c4_replay_and_decoder_step(csa):
-    """B=4, 262,144 entries: SWA Bounded Replay of the last 128 tokens (s = ctx - 128) through a
-    Full layer, then one decode step through the 20-layer decoder pattern with the append."""
+    """B=4, 262,144 entries: SWA Bounded Replay of the last 128 tokens (s = ctx - 128) through
+    the 20-layer decoder pattern (fresh FP8 SWA KV per layer; Reuse layers borrow the indices,
+    Reindex layers search the Full layer's pool), then one decode step through the same 20
+    layers with the append.  Sampled queries of batch row 2 are checked at every indexing
+    layer (indices, pool) and at several attention layers."""
     B, n = 4, 262144
     grp = BigGroup(csa, 140, B, n + 128, [n] * B, keep=(2,))
     s = n - 128
     Q = 128
-    # ---- replay: 128 queries per batch row at tokens s .. n-1, Full layer
-    iq, iqs, w, oiq, oiqs, ow = index_query(141, B, Q)
+    sample = [0, 64, 127]
     qp_np = np.tile(s + np.arange(Q, dtype=np.int32), (B, 1))
     qp = torch.from_numpy(qp_np).cuda()
-    idx = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, 512)
-    gi = np_(idx)
-    sample = [0, 64, 127]
-    ik, iks = grp.oracle_k(2)
-    ridx = oracle.index_topk(oiq[2:3, sample], oiqs[2:3, sample], ow[2:3, sample], ik, iks, grp.n_entries[2:3], 1,
-                             qp_np[2:3, sample], 512)
-    assert np.array_equal(gi[2:3, sample], ridx)
-    q = synth.attn_q(142, B, Q, "cuda")
-    swa, swa_sc = swa_for(143, B, 128, [s] * B)
     rs = torch.full((B,), s, dtype=torch.int32, device="cuda")
-    out = csa.csa2_sparse_attn(q, grp.kv, idx, swa, swa_sc, rs, qp, replay_start=rs)
-    for j, qi in enumerate(sample):
-        ref, _ = _attn_ref(grp, 2, bits(q[2:3, qi:qi + 1]), ridx[:, j:j + 1], np_(swa)[2:3], np_(swa_sc)[2:3], s,
-                           qp_np[2, qi], replay=s)
-        ok, st = attn_close(out[2:3, qi:qi + 1], ref)
-        assert ok, (qi, st)
+    ridx_q = torch.zeros((B, Q, 512), dtype=torch.int32, device="cuda")
+    rpool = torch.zeros((B, Q, 2048), dtype=torch.int32, device="cuda")
+    rbm = torch.zeros((B, Q, (grp.cap + 7) // 8), dtype=torch.float32, device="cuda")
+    rik, riks = grp.oracle_k(2)
+    pool_ref = cur = None
+    for li, mode in enumerate(oracle.DECODER_PATTERN):
+        lq = synth.attn_q(synth.seed_of("c4rq", li), B, Q, "cuda")
+        lswa, lswa_sc = swa_for(synth.seed_of("c4rswa", li), B, 128, [s] * B)
+        liq = liqs = lw = loiq = loiqs = low = None
+        if mode != "reuse":
+            liq, liqs, lw, loiq, loiqs, low = index_query(synth.seed_of("c4riq", li), B, Q)
+        out = csa.csa2_layer_step(mode, grp.kv, qp, lq, lswa, lswa_sc, rs, ridx_q, 512, liq, liqs, lw, pool=rpool,
+                                  blockmax=rbm, k_proj=grp.W, replay_start=rs)
+        if mode == "full":
+            cur, bm_ref = oracle.index_topk(loiq[2:3, sample], loiqs[2:3, sample], low[2:3, sample], rik, riks,
+                                            grp.n_entries[2:3], 1, qp_np[2:3, sample], 512, blockmax=True)
+            pool_ref = oracle.pool_build(bm_ref, grp.n_entries[2:3], 1, qp_np[2:3, sample], 2048)
+            assert np.array_equal(np_(rpool)[2:3, sample], pool_ref)
+        elif mode == "reindex":
+            cur = oracle.pool_topk(loiq[2:3, sample], loiqs[2:3, sample], low[2:3, sample], rik, riks,
+                                   grp.n_entries[2:3], 1, pool_ref, qp_np[2:3, sample], 512)
+        assert np.array_equal(np_(ridx_q)[2:3, sample], cur), (li, mode)
+        if li in (0, 1, 4, 7, 12, 19):
+            for j, qi in enumerate(sample):
+                ref, _ = _attn_ref(grp, 2, bits(lq[2:3, qi:qi + 1]), cur[:, j:j + 1], np_(lswa)[2:3],
+                                   np_(lswa_sc)[2:3], s, qp_np[2, qi], replay=s)
+                ok, st = attn_close(out[2:3, qi:qi + 1], ref)
+                assert ok, (li, mode, qi, st)
     # ---- decode step: the new token (position n) is appended by the Full layer
     new_lat = torch.stack([synth.latent(synth.seed_of("c4new", b), 1, n, "cuda")[0] for b in range(B)])
     new_rows = torch.tensor([b * grp.cap + n for b in range(B)], dtype=torch.int64, device="cuda")

@@ -380,6 +380,35 @@ def test_sparse_attn_decode(csa, B, Q):
     _attn_case(csa, 40 + B, B, Q, cap, n_entries, k, T, 128, q_pos, pos0, None, idx)
 
 
+@pytest.mark.parametrize("B,Q,k,T,cap", [(8, 2, 512, 128, 1536), (32, 1, 500, 128, 1152), (1, 1, 2048, 128, 3072),
+                                         (37, 1, 512, 100, 1152), (2, 1, 37, 128, 1024)],
+                         ids=["c8", "c4_ragged_main", "c16_2048", "c4_short_window", "c16_small_k"])
+def test_sparse_attn_tensor_core_decode_shapes(csa, B, Q, k, T, cap):
+    # the tensor-core decode kernel at cluster sizes 8, 4 and 16: ragged main shares
+    # (500 = 4 x 125 rows, so the last rows of a CTA's tile are padding), the most
+    # main rows a CTA holds (2048 / 16 = 128), fewer stored window rows than the
+    # window (dead window slots), and a few main rows per CTA (37 / 16)
+    rng = np.random.default_rng(B + k)
+    n_entries = [cap - 50 - 3 * b for b in range(B)]
+    idx = np.sort(rng.integers(0, cap - 60, (B, Q, k)), axis=-1).astype(np.int32)
+    idx[:, :, ::37] = -1
+    q_pos = [[n_entries[b] - 1 - 2 * qi for qi in range(Q)] for b in range(B)]
+    pos0 = [n_entries[b] - T for b in range(B)]
+    _attn_case(csa, 80 + B, B, Q, cap, n_entries, k, T, 128, q_pos, pos0, None, idx)
+
+
+def test_sparse_attn_warp_mma_cluster_shape(csa):
+    # 40 queries with 280 main rows each: two CTAs per query hold 148 slots each,
+    # more main rows than the tensor-core kernel stages, so the warp-MMA cluster kernel serves it
+    B, Q, k, T, cap = 40, 1, 280, 16, 640
+    rng = np.random.default_rng(9)
+    n_entries = [600 - b for b in range(B)]
+    idx = np.sort(rng.integers(0, 560, (B, Q, k)), axis=-1).astype(np.int32)
+    q_pos = [[n_entries[b] - 1] for b in range(B)]
+    pos0 = [n_entries[b] - T for b in range(B)]
+    _attn_case(csa, 90, B, Q, cap, n_entries, k, T, 16, q_pos, pos0, None, idx)
+
+
 @pytest.mark.parametrize("window", [1, 2, 4, 77, 128])
 @pytest.mark.parametrize("Q", [8, 128])   # 16 queries: one cluster each; 256: split-K kernel
 def test_sparse_attn_replay_mask(csa, window, Q):
@@ -453,3 +482,51 @@ def test_layer_dispatch_decoder_pattern(csa):
         assert np.array_equal(np_(idx), st["idx"]), (li, mode)
         ok, stats = attn_close(out, ref)
         assert ok, (li, mode, stats)
+
+
+# ---------------------------------------------------------------- fused front end
+def _rope_tables(pos):
+    k = np.arange(32, dtype=np.float64)
+    ang = np.asarray(pos, np.float64).reshape(-1, 1) * 10000.0 ** (-2.0 * k / 64.0)
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
+@pytest.mark.parametrize("rows,weighted", [(1, False), (37, True), (64, False), (1000, True), (5000, False)])
+def test_front_end_bit_exact(csa, rows, weighted):
+    """RMSNorm + RoPE + bf16 + NVFP4 + indexer-K in one launch: every byte equals the oracle's
+    front end followed by its quantiser and projection (rows past a multiple of 64: ragged CTA)."""
+    x = (synth.normal(synth.seed_of("front", rows), (rows, 512), "cuda") * 1.7).to(torch.bfloat16)
+    pos = np.arange(rows) * 131 + 7
+    cos, sin = _rope_tables(pos)
+    w = (0.25 + synth.uniform(synth.seed_of("front-w", rows), 512).to(torch.float32)).cuda() if weighted else None
+    W = synth.proj_w(rows).cuda()
+    out_rows = (2 * rows + 128) // 128 * 128
+    dst = torch.arange(rows, device="cuda", dtype=torch.int64) * 2 + 1
+    lc = torch.zeros((out_rows, 256), dtype=torch.uint8, device="cuda")
+    ls = torch.zeros((out_rows, 32), dtype=torch.uint8, device="cuda")
+    kc = torch.zeros((out_rows, 32), dtype=torch.uint8, device="cuda")
+    ks = torch.zeros((out_rows, 4), dtype=torch.uint8, device="cuda")
+    y = torch.zeros((rows, 512), dtype=torch.bfloat16, device="cuda")
+    csa.csa2_front_end(x, torch.from_numpy(cos).cuda(), torch.from_numpy(sin).cuda(), W, (lc, ls, kc, ks), dst,
+                       norm_w=w, y_out=y)
+    oy = oracle.front_end(bits(x), cos, sin, None if w is None else np_(w))
+    assert np.array_equal(bits(y), oy)
+    olc, ols = oracle.quant_nvfp4(oy)
+    okc, oks = oracle.index_k_proj(oy, np_(W))
+    assert np.array_equal(np_(lc)[1::2][:rows], olc) and np.array_equal(np_(ls)[1::2][:rows], ols)
+    gkc, gks = ik_untile(np_(kc), np_(ks))
+    assert np.array_equal(gkc[1::2][:rows], okc) and np.array_equal(gks[1::2][:rows], oks)
+    assert not np_(lc)[0::2].any() and not gkc[0::2].any()
+
+
+def test_front_end_hand_worked_cases(csa):
+    import test_oracle_front as tf
+    for case in tf.CASES:
+        x = torch.from_numpy(tf._bits(case["x"]).view(np.int16)).view(torch.bfloat16).reshape(1, 512).cuda()
+        cos = torch.from_numpy(case["cos"]).cuda()
+        sin = torch.from_numpy(case["sin"]).cuda()
+        w = None if case["w"] is None else torch.from_numpy(case["w"]).cuda()
+        outs = tuple(torch.zeros((128, n), dtype=torch.uint8, device="cuda") for n in (256, 32, 32, 4))
+        y = torch.zeros((1, 512), dtype=torch.bfloat16, device="cuda")
+        csa.csa2_front_end(x, cos, sin, synth.proj_w(0).cuda(), outs, norm_w=w, y_out=y)
+        assert np.array_equal(bits(y)[0], tf._bits(case["out"])), case["name"]
