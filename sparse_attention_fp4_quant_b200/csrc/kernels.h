@@ -121,8 +121,6 @@ struct AttnParams {
     int slots_total;          // k + window
     int tiles_per_split;      // split-K form: 64-key tiles per split
     int keys_per_cta;         // cluster form: key slots per CTA
-    int main_per_cta;         // tensor-core cluster form: main slots per CTA
-    int swa_per_cta;          // tensor-core cluster form: window slots per CTA
     // workspace
     int32_t* counters;        // [B*Q]
     int32_t* status;          // sticky: set to 1 if a device-side wait timed out
@@ -137,8 +135,5 @@ cudaError_t launch_attn(AttnParams& p, int S, cudaStream_t st);
 // One cluster of C CTAs per query; 0 = the shape does not fit.
 int attn_cluster_size(int B, int Q, int slots_total, int* keys_per_cta);
 cudaError_t launch_attn_cluster(AttnParams& p, int C, cudaStream_t st);
-// The same on the 5th-generation tensor cores (attn_tc.cu); 0 = the shape does not fit.
-int attn_tc_cluster_size(int B, int Q, int k, int window, int* main_per_cta, int* swa_per_cta);
-cudaError_t launch_attn_tc(AttnParams& p, int C, cudaStream_t st);
 
 }  // namespace csa2

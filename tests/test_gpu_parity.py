@@ -382,12 +382,12 @@ def test_sparse_attn_decode(csa, B, Q):
 
 @pytest.mark.parametrize("B,Q,k,T,cap", [(8, 2, 512, 128, 1536), (32, 1, 500, 128, 1152), (1, 1, 2048, 128, 3072),
                                          (37, 1, 512, 100, 1152), (2, 1, 37, 128, 1024)],
-                         ids=["c8", "c4_ragged_main", "c16_2048", "c4_short_window", "c16_small_k"])
-def test_sparse_attn_tensor_core_decode_shapes(csa, B, Q, k, T, cap):
-    # the tensor-core decode kernel at cluster sizes 8, 4 and 16: ragged main shares
-    # (500 = 4 x 125 rows, so the last rows of a CTA's tile are padding), the most
-    # main rows a CTA holds (2048 / 16 = 128), fewer stored window rows than the
-    # window (dead window slots), and a few main rows per CTA (37 / 16)
+                         ids=["c8", "c4_ragged", "c16_2048", "c4_short_window", "c16_small_k"])
+def test_sparse_attn_decode_cluster_shapes(csa, B, Q, k, T, cap):
+    # the decode cluster kernel at cluster sizes 8, 4 and 16: ragged key shares
+    # (500 main slots), the most main rows a query takes (2048 over 16 CTAs),
+    # fewer stored window rows than the window (dead window slots), and a few
+    # main rows per CTA (37 over 16)
     rng = np.random.default_rng(B + k)
     n_entries = [cap - 50 - 3 * b for b in range(B)]
     idx = np.sort(rng.integers(0, cap - 60, (B, Q, k)), axis=-1).astype(np.int32)
@@ -397,9 +397,8 @@ def test_sparse_attn_tensor_core_decode_shapes(csa, B, Q, k, T, cap):
     _attn_case(csa, 80 + B, B, Q, cap, n_entries, k, T, 128, q_pos, pos0, None, idx)
 
 
-def test_sparse_attn_warp_mma_cluster_shape(csa):
-    # 40 queries with 280 main rows each: two CTAs per query hold 148 slots each,
-    # more main rows than the tensor-core kernel stages, so the warp-MMA cluster kernel serves it
+def test_sparse_attn_two_cta_clusters(csa):
+    # 40 queries with 280 main rows each: two CTAs per query hold 148 slots each
     B, Q, k, T, cap = 40, 1, 280, 16, 640
     rng = np.random.default_rng(9)
     n_entries = [600 - b for b in range(B)]
