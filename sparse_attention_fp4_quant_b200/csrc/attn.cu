@@ -17,6 +17,7 @@ namespace csa2 {
 constexpr int kAT = 256;      // threads per CTA (8 warps)
 constexpr int kKT = 64;       // keys per tile
 constexpr int kMaxSplits = (CSA2_MAX_K + CSA2_MAX_WINDOW + kKT - 1) / kKT;
+constexpr int kMaxSplitMain = CSA2_MAX_K + kKT;   // main-row ids a split reads (its tiles' slots below k)
 
 struct AttnSmem {
     uint8_t K[kKT * kRowB];   // 64 KB, 16-byte chunks XOR-swizzled by row & 7
@@ -31,6 +32,7 @@ struct AttnSmem {
     float cw[kMaxSplits][kH];  // combine weights 2^(m_s - M) / L per split and head
     float qmax[kAT / 32];      // per-warp max |q|
     int last;
+    int32_t eidx[kMaxSplitMain];   // this split's main-row ids, read once up front
 };
 
 __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
@@ -59,11 +61,27 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
     const int t0 = split * p.tiles_per_split;
     const int t1 = min(ntiles, t0 + p.tiles_per_split);
     // gather: key row and quarter of this thread; consecutive lanes take
-    // consecutive rows so their swizzled 16-byte stores hit distinct banks
+    // consecutive rows so their swizzled 16-byte stores hit distinct banks.
+    // The split's main-row ids go to shared memory first (one round trip for all
+    // tiles), so a tile's row loads never wait on an id load.
     const int gr = tid & (kKT - 1), gq = tid >> 6;
+    const int sm0 = t0 * kKT, sm1 = min(p.k, t1 * kKT);   // this split's main slots [sm0, sm1)
+    {
+        constexpr int kPer = (kMaxSplitMain + kAT - 1) / kAT;
+        int32_t ev[kPer];   // every id load of the thread in flight before any is stored
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int s = sm0 + tid + kAT * j;
+            ev[j] = s < sm1 ? (int32_t)ld_nc_u32(p.idx + (int64_t)bq * p.k + s) : -1;
+        }
+#pragma unroll
+        for (int j = 0; j < kPer; ++j)
+            if (sm0 + tid + kAT * j < sm1) sm.eidx[tid + kAT * j] = ev[j];
+    }
+    __syncthreads();
 
     RowQuarter rq;
-    if (t0 < t1) fetch_quarter(p, bq, b, t0 * kKT + gr, gq, i_pos, lo, pos0, nmain, rq);
+    if (t0 < t1) fetch_quarter_id(p, b, t0 * kKT + gr, gq, sm.eidx, sm0, i_pos, lo, pos0, nmain, rq);
 
     // Q [16][512] bf16 -> f16 times a power-of-two prescale -> swizzled smem
     {
@@ -105,18 +123,24 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
     for (int tile = t0; tile < t1; ++tile) {
         store_quarter(sm.K, sm.kf, sm.kvalid, gr, gq, rq);
         __syncthreads();
-        if (tile + 1 < t1) fetch_quarter(p, bq, b, (tile + 1) * kKT + gr, gq, i_pos, lo, pos0, nmain, rq);   // in flight meanwhile
+        if (tile + 1 < t1)   // in flight meanwhile
+            fetch_quarter_id(p, b, (tile + 1) * kKT + gr, gq, sm.eidx, sm0, i_pos, lo, pos0, nmain, rq);
 
-        // ---- S = Q K^T for keys 8*warp .. +7 ----
-        float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        // ---- S = Q K^T for keys 8*warp .. +7 (two accumulator chains: even and odd k-steps) ----
+        float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f}, s4b[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll 8
-        for (int ks = 0; ks < kD / 16; ++ks) {
-            uint32_t a0, a1, a2, a3, b0, b1;
-            ldsm_x4(sQ + swz(lane & 15, 2 * ks + (lane >> 4)), a0, a1, a2, a3);
+        for (int ks = 0; ks < kD / 16; ks += 2) {
+            uint32_t a0, a1, a2, a3, b0, b1, c0, c1, c2, c3, d0, d1;
             const int key = 8 * warp + (lane & 7);
+            ldsm_x4(sQ + swz(lane & 15, 2 * ks + (lane >> 4)), a0, a1, a2, a3);
             ldsm_x2(sK + swz(key, 2 * ks + ((lane >> 3) & 1)), b0, b1);
+            ldsm_x4(sQ + swz(lane & 15, 2 * ks + 2 + (lane >> 4)), c0, c1, c2, c3);
+            ldsm_x2(sK + swz(key, 2 * ks + 2 + ((lane >> 3) & 1)), d0, d1);
             mma_f16(s4, a0, a1, a2, a3, b0, b1);
+            mma_f16(s4b, c0, c1, c2, c3, d0, d1);
         }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) s4[j] += s4b[j];
         // logits (log2 units); masked keys -> -inf
         const int key0 = 8 * warp + 2 * qd;
         const float f0 = sm.kf[key0], f1 = sm.kf[key0 + 1];

@@ -115,11 +115,14 @@ struct RowQuarter {
     int kind;       // 0 = dead slot, 1 = FP4 main row, 2 = FP8 window row
 };
 
-__device__ __forceinline__ void fetch_quarter(const AttnParams& p, int bq, int b, int slot, int qq, int64_t i_pos,
-                                              int64_t lo, int64_t pos0, int64_t nmain, RowQuarter& q) {
+// Issue the loads of quarter qq (128 dims) of key slot `slot`: a main row's id comes
+// from shared memory (ids[slot - id0]), so its row loads never wait on an id load.
+__device__ __forceinline__ void fetch_quarter_id(const AttnParams& p, int b, int slot, int qq, const int32_t* ids,
+                                                 int id0, int64_t i_pos, int64_t lo, int64_t pos0, int64_t nmain,
+                                                 RowQuarter& q) {
     q.kind = 0;
     if (slot < p.k) {
-        const int32_t e = __ldg(p.idx + (int64_t)bq * p.k + slot);
+        const int32_t e = ids[slot - id0];
         if (e >= 0 && e < nmain) {
             q.kind = 1;
             const int64_t row = (int64_t)b * p.cap + e;
