@@ -304,8 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int group = (warp - 2) >> 2;        // tiles 2*group, 2*group+1 of each stage
         const int eo = quarter * 32 + lane;       // this thread's TMEM row = its entry within a tile
         const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
-        const float w0 = __ldg(p.w + (int64_t)bq * 4 + 0), w1 = __ldg(p.w + (int64_t)bq * 4 + 1);
-        const float w2 = __ldg(p.w + (int64_t)bq * 4 + 2), w3 = __ldg(p.w + (int64_t)bq * 4 + 3);
+        const uint64_t w01 = f2pack(__ldg(p.w + (int64_t)bq * 4 + 0), __ldg(p.w + (int64_t)bq * 4 + 1));
+        const uint64_t w23 = f2pack(__ldg(p.w + (int64_t)bq * 4 + 2), __ldg(p.w + (int64_t)bq * 4 + 3));
         float* bm = p.blockmax ? p.blockmax + (int64_t)bq * p.nb_cap : nullptr;
         bool dead = false;   // this warp stopped after a failed wait (or another role's)
         for (int t = 0; t < nstages; ++t) {
@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int j = 0; j < kTPG; ++j) {
                     const int g = g0 + j;
                     const bool valid = g < ntiles && lo + g * kTile + eo < hi;
-                    const float score = valid ? score_of(v[j], skw[j], w0, w1, w2, w3) : -INFINITY;
+                    const float score = valid ? score_of(v[j], key_scales(skw[j]), w01, w23) : -INFINITY;
                     key[j] = valid ? score_key(score) : 0u;
                     if (valid) atomicAdd(&s.hist1[key[j] >> 21], 1u);
                     if (bm) {

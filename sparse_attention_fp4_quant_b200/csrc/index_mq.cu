@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(kMqThreads, 1) mq_score_kernel(SelectParams p,
         }
         __syncwarp();
         for (int n = lane; n < 16 * ng; n += 32) {
-            const int g = n >> 4, h = (n >> 2) & 3, blk = n & 3;
+            const int g = n >> 4, h = n & 3, blk = (n >> 2) & 3;   // column 16 g + 4 blk + h
             const uint8_t* q = p.q + (bq0 + g) * 128;
             const uint8_t* qs = p.q_sc + (bq0 + g) * 16;
             uint8_t* row = s.Bq + (n >> 3) * 256 + (blk >> 1) * 128 + (n & 7) * 16 + 8 * (blk & 1);
@@ -157,14 +157,17 @@ __global__ void __launch_bounds__(kMqThreads, 1) mq_score_kernel(SelectParams p,
         const int gb = kQPW * ((warp - 2) >> 2);      // queries gb .. gb + kQPW - 1
         const int row = 32 * quarter + lane;
         const uint32_t lanes = (uint32_t)(32 * quarter) << 16;
-        float wq[kQPW][4];
+        uint64_t w01[kQPW], w23[kQPW];
         int nv[kQPW];
 #pragma unroll
         for (int j = 0; j < kQPW; ++j) {
             const int g = gb + j;
             nv[j] = g < ng ? n_visible(p.q_pos[bq0 + g], p.n_entries[b], p.m, p.cap) : 0;
+            float wq[4];
 #pragma unroll
-            for (int h = 0; h < 4; ++h) wq[j][h] = g < ng ? __ldg(p.w + (bq0 + g) * 4 + h) : 0.0f;
+            for (int h = 0; h < 4; ++h) wq[h] = g < ng ? __ldg(p.w + (bq0 + g) * 4 + h) : 0.0f;
+            w01[j] = f2pack(wq[0], wq[1]);
+            w23[j] = f2pack(wq[2], wq[3]);
         }
         bool dead = false;
         int u = 0;
@@ -191,7 +194,7 @@ __global__ void __launch_bounds__(kMqThreads, 1) mq_score_kernel(SelectParams p,
                     dead = true;
                     continue;
                 }
-                const uint32_t skw = stage_scales(s, t % kMqRing, i, row);
+                const KeyScales ks = key_scales(stage_scales(s, t % kMqRing, i, row));   // shared by the queries
                 if (i == ntl - 1) release_stage(s, t, lane);
                 const int e = u * kTile + row;
 #pragma unroll
@@ -199,7 +202,7 @@ __global__ void __launch_bounds__(kMqThreads, 1) mq_score_kernel(SelectParams p,
                     const int g = gb + j;
                     if (g >= ng) break;   // warp-uniform
                     const bool valid = e < nv[j];
-                    const float score = valid ? score_of(v[j], skw, wq[j][0], wq[j][1], wq[j][2], wq[j][3]) : -INFINITY;
+                    const float score = valid ? score_of(v[j], ks, w01[j], w23[j]) : -INFINITY;
                     const uint32_t key = score_key(score);
                     if (valid) {
                         atomicAdd(&s.hist[g][key >> 21], 1u);

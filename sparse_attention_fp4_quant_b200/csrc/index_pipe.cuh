@@ -4,7 +4,7 @@
 //
 // Scoring as a block-scaled FP4 MMA.  A = 128 indexer-K rows (E2M1, K = 64
 // channels) with unit block scales; B = the query as a block-diagonal 16 x 64
-// operand with its own E4M3 block scales: column n = 4 h + b holds head h's
+// operand with its own E4M3 block scales: column n = 4 b + h holds head h's
 // codes in block b only, so accumulator column n of row t is exactly
 //   (sum over 16 channels of q k) * sq[h][b]
 // (at most 16 significant bits: exact in fp32 whatever the MMA's summation
@@ -86,8 +86,9 @@ __device__ __forceinline__ void init_barriers(P& s, uint32_t epi_arrivals) {
 }
 
 // Warp 1: allocate `cols` TMEM columns (the pipeline uses the first kPipeCols)
-// and lay out the block-diagonal query operand.  Row n = 4h + b keeps head h's
-// 8 code bytes of block b; all else zero.
+// and lay out the block-diagonal query operand.  Row n = 4b + h keeps head h's
+// 8 code bytes of block b; all else zero.  (Block-major columns put the four
+// heads of a block in adjacent accumulator registers, which score_of pairs.)
 template <class P>
 __device__ __forceinline__ void setup_query(P& s, const uint8_t* q, const uint8_t* qs, int lane, uint32_t cols) {
     tc::tmem_alloc(&s.tmem_base, cols);
@@ -96,7 +97,7 @@ __device__ __forceinline__ void setup_query(P& s, const uint8_t* q, const uint8_
     for (int i = lane; i < 512; i += 32) s.SFA[i] = 0x38;   // E4M3 1.0
     __syncwarp();
     if (lane < 16) {
-        const int n = lane, h = n >> 2, blk = n & 3;
+        const int n = lane, h = n & 3, blk = n >> 2;
         const int kc = blk >> 1, off = 8 * (blk & 1);
         uint8_t* row = s.Bq + (n >> 3) * 256 + kc * 128 + (n & 7) * 16 + off;
         const uint8_t* src = q + 32 * h + 8 * blk;
@@ -233,23 +234,65 @@ __device__ __forceinline__ void mma_issuer(P& s, int ntiles, int nstages, int32_
     __syncwarp();
 }
 
-// The defined score of one row from its 16 accumulator columns (column 4h + b =
-// head h, block b, without the key's scale) and the row's 4 key scale bytes.
-__device__ __forceinline__ float score_of(const uint32_t (&v)[16], uint32_t sk_bytes, float w0, float w1, float w2,
-                                          float w3) {
-    const float* U = reinterpret_cast<const float*>(v);
+// Packed fp32 pairs: one IEEE round-to-nearest product or sum per lane.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// The row's four key block scales as (sk_b, sk_b) pairs.
+struct KeyScales {
+    uint64_t s2[4];
+};
+__device__ __forceinline__ KeyScales key_scales(uint32_t sk_bytes) {
     float sk[4];
     e4m3x4_to_f32(sk_bytes, sk);
-    float r[4];
+    KeyScales k;
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-        const float T0 = __fmul_rn(U[4 * h], sk[0]), T1 = __fmul_rn(U[4 * h + 1], sk[1]);
-        const float T2 = __fmul_rn(U[4 * h + 2], sk[2]), T3 = __fmul_rn(U[4 * h + 3], sk[3]);
-        const float d = __fadd_rn(__fadd_rn(__fadd_rn(T0, T1), T2), T3);
-        r[h] = d > 0.0f ? d : 0.0f;
+    for (int b = 0; b < 4; ++b) k.s2[b] = f2pack(sk[b], sk[b]);
+    return k;
+}
+
+// The defined score of one row from its 16 accumulator columns (column 4b + h =
+// block b of head h, without the key's scale) and the row's key scales:
+//   T[h][b] = acc * sk[b];  d_h = ((T0 + T1) + T2) + T3;  r_h = max(d_h, +0);
+//   score = ((w0 r0 + w1 r1) + w2 r2) + w3 r3,
+// every product and sum one fp32 rounding.  Heads (0, 1) and (2, 3) run as
+// packed pairs (lane by lane the same IEEE operations).  w01 = (w0, w1), w23 = (w2, w3).
+__device__ __forceinline__ float score_of(const uint32_t (&v)[16], const KeyScales& ks, uint64_t w01, uint64_t w23) {
+    uint64_t d01 = 0, d23 = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        const uint64_t t01 = f2mul(f2pack(__uint_as_float(v[4 * b]), __uint_as_float(v[4 * b + 1])), ks.s2[b]);
+        const uint64_t t23 = f2mul(f2pack(__uint_as_float(v[4 * b + 2]), __uint_as_float(v[4 * b + 3])), ks.s2[b]);
+        d01 = b == 0 ? t01 : f2add(d01, t01);
+        d23 = b == 0 ? t23 : f2add(d23, t23);
     }
-    return __fadd_rn(__fadd_rn(__fadd_rn(__fmul_rn(w0, r[0]), __fmul_rn(w1, r[1])), __fmul_rn(w2, r[2])),
-                     __fmul_rn(w3, r[3]));
+    float r0, r1, r2, r3;
+    f2unpack(d01, r0, r1);
+    f2unpack(d23, r2, r3);
+    r0 = r0 > 0.0f ? r0 : 0.0f;
+    r1 = r1 > 0.0f ? r1 : 0.0f;
+    r2 = r2 > 0.0f ? r2 : 0.0f;
+    r3 = r3 > 0.0f ? r3 : 0.0f;
+    float p0, p1, p2, p3;
+    f2unpack(f2mul(w01, f2pack(r0, r1)), p0, p1);
+    f2unpack(f2mul(w23, f2pack(r2, r3)), p2, p3);
+    return __fadd_rn(__fadd_rn(__fadd_rn(p0, p1), p2), p3);
 }
 
 // Epilogue warp, stage t in ring slot `slot`: the 4 scale bytes of row `row` of

@@ -91,8 +91,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int quarter = warp & 3;             // TMEM lanes this warp may read
         const int group = (warp - 2) >> 2;        // tiles 2*group, 2*group+1 of each stage
         const int row = quarter * 32 + lane;
-        const float w0 = __ldg(p.w + (int64_t)bq * 4 + 0), w1 = __ldg(p.w + (int64_t)bq * 4 + 1);
-        const float w2 = __ldg(p.w + (int64_t)bq * 4 + 2), w3 = __ldg(p.w + (int64_t)bq * 4 + 3);
+        const uint64_t w01 = f2pack(__ldg(p.w + (int64_t)bq * 4 + 0), __ldg(p.w + (int64_t)bq * 4 + 1));
+        const uint64_t w23 = f2pack(__ldg(p.w + (int64_t)bq * 4 + 2), __ldg(p.w + (int64_t)bq * 4 + 3));
         float* bm = (MODE == 0 && p.blockmax) ? p.blockmax + (int64_t)bq * p.nb_cap : nullptr;
         bool stop = false;
         for (int t = 0; t < nstages && !stop; ++t) {
@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                 }
                 const bool valid = e >= 0;
-                const float score = valid ? score_of(v[j], skw[j], w0, w1, w2, w3) : -INFINITY;
+                const float score = valid ? score_of(v[j], key_scales(skw[j]), w01, w23) : -INFINITY;
                 if (MODE == 0 && bm && g < ntiles) {
                     const float m8 = block_max8(score, lane);
                     if ((lane & 7) == 0 && valid) bm[e >> 3] = m8;
