@@ -242,7 +242,7 @@ csa2_status csa2_sparse_attn(const void* q, const csa2_kv* kv, const int32_t* id
     p.slots_total = k + window;
     int S = attn_splits(B, Q, k, window, &p.tiles_per_split);
     attn_carve_ws(p, S, ws);
-    const int C = attn_cluster_size(B, Q, p.slots_total, &p.keys_per_cta);
+    const int C = attn_cluster_size(B, Q, k, window, &p.main_per_cta, &p.swa_per_cta);
     if (C > 0) return cuda_status(launch_attn_cluster(p, C, (cudaStream_t)stream));
     return cuda_status(launch_attn(p, S, (cudaStream_t)stream));
 }

@@ -1,17 +1,19 @@
 // attn_cluster.cu -- csa2_sparse_attn for decode-sized query counts: one
 // thread-block cluster of C CTAs per query.
 //
-// CTA r of the cluster takes the key slots [r * n, (r + 1) * n) of its query
-// (n <= 160, a multiple of 16; slots as in attn_common.cuh) and gathers them
-// all at once, so a CTA waits on global memory once instead of once per tile.
+// CTA r of the cluster takes the main slots [r nm, (r + 1) nm) of its query's
+// k selected entries and the window slots [r nw, (r + 1) nw) of its W window
+// positions (nm = ceil(k / C), nw = ceil(W / C), nm + nw <= 160), so every CTA
+// moves about the same bytes, and gathers them all at once: a CTA waits on
+// global memory once instead of once per tile, and each warp reads whole rows.
 // The rows are dequantised to f16 in swizzled shared memory (K = V); with the
 // 16 heads as the M dimension, S = Q K^T runs on warp-level tensor-core MMAs
 // (each warp a quarter of the channels of a fifth of the keys), then the CTA's
 // own softmax (one warp per head: max and sum over its keys), then O_r = P V
-// (32 dims per warp; P as a rounded f16 term plus its f16 remainder).  The partial results meet in distributed shared memory:
-// each CTA stores, into CTA c's (by then idle) key buffer, its slice
-// [c * 512 / C, (c + 1) * 512 / C) of O_r (fp32) and its per-head (max, sum);
-// CTA c then forms its slice of the output as
+// (32 dims per warp; P rounded to f16, fp32 accumulation).  The partial results
+// meet in distributed shared memory: each CTA stores, into CTA c's (by then
+// idle) key buffer, its slice [c * 512 / C, (c + 1) * 512 / C) of O_r (fp32)
+// and its per-head (max, sum); CTA c then forms its slice of the output as
 //   sum_r 2^(m_r - M) O_r / sum_r 2^(m_r - M) l_r,   M = max_r m_r,
 // from its own shared memory and writes it as bf16.  No partials go to global
 // memory and no CTA waits for a ticket.
@@ -27,20 +29,21 @@ constexpr int kPStride = kMaxKeys * 2 + 16;   // bytes per head row of P (confli
 constexpr int kQG = 4;                        // key-tile groups of the S warps (x 4 channel groups)
 constexpr int kQT = kMaxKeys / 8 / kQG;       // key tiles per S warp
 constexpr int kSStride = kMaxKeys + 4;        // floats per head row of a partial S
+constexpr int kMaxC = 16;                     // largest cluster
 static_assert(kMaxKeys % 32 == 0 && kMaxKeys % (8 * kQG) == 0, "keys per CTA");
 static_assert(kCT / 32 == kH, "one warp per head in the softmax");
-static_assert(2 * kH * kSStride * 4 <= kH * kRowB + 2 * kH * kPStride, "partial S fit the Q and P buffers");
-static_assert((16 * kH * (kD / 16 + 4) + 16 * kH * 2) * 4 <= kMaxKeys * kRowB, "received slices fit the key buffer");
+static_assert(2 * kH * kSStride * 4 <= kH * kRowB + kH * kPStride, "partial S fit the Q and P buffers");
+static_assert((kH * (kD + 4 * kMaxC) + kMaxC * kH * 2) * 4 <= kMaxKeys * kRowB, "received slices fit the key buffer");
 
+// 188 KB: the rest of the SM's 256 KB stays L1, which holds the gather's loads in flight
 struct ClAttnSmem {
     uint8_t K[kMaxKeys * kRowB];   // f16 keys (= values), swizzled; afterwards the received output slices
     uint8_t Qs[kH * kRowB];        // f16 query (prescaled), swizzled; then (with P) the two partial S arrays
-    uint8_t P[kH * kPStride];      // f16 P (rounded), [head][key]
-    uint8_t Pl[kH * kPStride];     // f16 remainder P - rounded(P)
+    uint8_t P[kH * kPStride];      // f16 P, [head][key]
     float kf[kMaxKeys];            // per-key factor (1 for FP4 rows, token scale for SWA)
     int kvalid[kMaxKeys];
     alignas(16) float ml[kH][2];   // this CTA's (max, sum) per head (log2 units), read by the cluster
-    float cw[16][kH];              // combine weight of rank c for head h (for this CTA's output slice)
+    float cw[kMaxC][kH];           // combine weight of rank c for head h (for this CTA's output slice)
     float qmax[kCT / 32];          // per-warp max |q|
 };
 
@@ -61,59 +64,96 @@ __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
     if (nmain > p.cap) nmain = p.cap;
     float scale_log2 = p.sm_scale * 1.4426950408889634f;
 
-    // this CTA's slots [s0, s0 + nk), padded to n16 (dead slots past nk)
-    const int s0 = min(p.slots_total, (int)rank * p.keys_per_cta);
-    const int nk = min(p.slots_total, s0 + p.keys_per_cta) - s0;
+    // this CTA's rows: main slots [m0, m0 + nm) then window slots [w0, w0 + nw) (an interleaved
+    // share, so every CTA of the cluster moves about the same bytes), padded to n16 dead rows
+    const int m0 = min(p.k, (int)rank * p.main_per_cta);
+    const int nm = min(p.k, m0 + p.main_per_cta) - m0;
+    const int w0 = min(p.window, (int)rank * p.swa_per_cta);
+    const int nw = min(p.window, w0 + p.swa_per_cta) - w0;
+    const int nk = nm + nw;
     const int n16 = (nk + 15) & ~15;
 
     const uint32_t sK = (uint32_t)__cvta_generic_to_shared(sm.K);
     const uint32_t sQ = (uint32_t)__cvta_generic_to_shared(sm.Qs);
     const uint32_t sP = (uint32_t)__cvta_generic_to_shared(sm.P);
-    const uint32_t sPl = (uint32_t)__cvta_generic_to_shared(sm.Pl);
 
-    // ---- gather: row quarter u = r + n16 * qq (consecutive lanes, consecutive rows).
-    // Every load of the thread is in flight before any is used: the main-row
-    // ids first, then the rows, then the query.
+    // ---- gather.  Item u = 32 r + x: 16 dims (16 x .. 16 x + 15) of row r, so a warp
+    // reads one row's 256 B of codes (or 512 B of a window row) in whole lines.  Every
+    // load of the thread is in flight before any is used: the query and the row ids
+    // first (one id per row, shared by the warp), then the rows.
     {
-        constexpr int kPer = (kMaxKeys * 4 + kCT - 1) / kCT;   // 2
-        RowQuarter rq[kPer];
-        int rr[kPer], qs[kPer], slot[kPer];
-        int32_t e[kPer];
-#pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-            const int u = tid + kCT * j;
-            rr[j] = -1;
-            e[j] = -1;
-            slot[j] = p.slots_total;
-            if (u < 4 * n16) {
-                rr[j] = u % n16;
-                qs[j] = u / n16;
-                if (rr[j] < nk) slot[j] = s0 + rr[j];   // past nk: dead
-                if (slot[j] < p.k) e[j] = (int32_t)ld_nc_u32(p.idx + (int64_t)bq * p.k + slot[j]);
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-            rq[j].kind = 0;
-            if (rr[j] >= 0) {
-                int64_t row = 0;
-                const int kind = slot_row(p, b, slot[j], e[j], i_pos, lo, pos0, nmain, row);
-                issue_quarter(p, kind, row, qs[j], rq[j]);
-            }
-        }
         const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q + (int64_t)bq * kH * kD);
         uint4 qv[(kH * kD / 8) / kCT];
 #pragma unroll
         for (int it = 0; it < (kH * kD / 8) / kCT; ++it) qv[it] = ld_nc_v4(qsrc + 16 * (it * kCT + tid));
+        constexpr int kPer = kMaxKeys * 32 / kCT;   // 10 items per thread
+        int32_t e[kPer];
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int r = (tid >> 5) + (kCT / 32) * j;
+            e[j] = r < nm ? (int32_t)ld_nc_u32(p.idx + (int64_t)bq * p.k + m0 + r) : -1;
+        }
+        uint4 raw[kPer];
+        uint32_t sc[kPer];
+        int kind[kPer];   // 0 dead or padding, 1 FP4 main row, 2 FP8 window row
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int r = (tid >> 5) + (kCT / 32) * j, x = lane;
+            kind[j] = 0;
+            raw[j] = make_uint4(0, 0, 0, 0);
+            sc[j] = 0;
+            if (r < nm) {
+                if (e[j] >= 0 && e[j] < nmain) {
+                    const int64_t row = (int64_t)b * p.cap + e[j];
+                    const uint2 c2 = ld_nc_v2(p.lat + row * (kD / 2) + 8 * x);
+                    raw[j].x = c2.x;
+                    raw[j].y = c2.y;
+                    sc[j] = (uint32_t)__ldg(p.lat_sc + row * (kD / 16) + x);
+                    kind[j] = 1;
+                }
+            } else if (r < nk) {
+                const int64_t tau = i_pos - p.window + 1 + (w0 + (r - nm));
+                const int64_t rr = tau - pos0;
+                if (tau >= lo && tau <= i_pos && rr >= 0 && rr < p.T) {
+                    const int64_t row = (int64_t)b * p.T + rr;
+                    raw[j] = ld_nc_v4(p.swa + row * kD + 16 * x);
+                    if (x == 0) sc[j] = ld_nc_u32(p.swa_sc + row);
+                    kind[j] = 2;
+                }
+            }
+        }
         float qm = 0.0f;   // max |q| of the query, for its power-of-two prescale into f16
 #pragma unroll
         for (int it = 0; it < (kH * kD / 8) / kCT; ++it) qm = fmaxf(qm, bf16x8_maxabs(qv[it]));
 #pragma unroll
         for (int o2 = 16; o2 > 0; o2 >>= 1) qm = fmaxf(qm, __shfl_xor_sync(0xFFFFFFFFu, qm, o2));
         if (lane == 0) sm.qmax[warp] = qm;
+        // rows -> f16 in the swizzled key buffer: chunks 2x and 2x + 1 of row r (exact: every
+        // E2M1 x E4M3 product and every E4M3 value is an f16); dead and padding rows are zero
 #pragma unroll
-        for (int j = 0; j < kPer; ++j)
-            if (rr[j] >= 0) store_quarter(sm.K, sm.kf, sm.kvalid, rr[j], qs[j], rq[j]);
+        for (int j = 0; j < kPer; ++j) {
+            const int r = (tid >> 5) + (kCT / 32) * j, x = lane;
+            if (r >= n16) continue;
+            uint4 lo4 = make_uint4(0, 0, 0, 0), hi4 = make_uint4(0, 0, 0, 0);
+            if (kind[j] == 1) {
+                uint32_t s16;
+                asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s16) : "h"((uint16_t)sc[j]));
+                const uint32_t s2 = __byte_perm(s16, 0u, 0x1010);
+                lo4 = fp4x8_to_f16(raw[j].x, s2);
+                hi4 = fp4x8_to_f16(raw[j].y, s2);
+            } else if (kind[j] == 2) {
+                const uint2 a = fp8x4_to_f16(raw[j].x), bb = fp8x4_to_f16(raw[j].y);
+                const uint2 c = fp8x4_to_f16(raw[j].z), d = fp8x4_to_f16(raw[j].w);
+                lo4 = make_uint4(a.x, a.y, bb.x, bb.y);
+                hi4 = make_uint4(c.x, c.y, d.x, d.y);
+            }
+            *reinterpret_cast<uint4*>(sm.K + swz(r, 2 * x)) = lo4;
+            *reinterpret_cast<uint4*>(sm.K + swz(r, 2 * x + 1)) = hi4;
+            if (x == 0) {
+                sm.kvalid[r] = kind[j] != 0;
+                sm.kf[r] = kind[j] == 2 ? __uint_as_float(sc[j]) : 1.0f;
+            }
+        }
         __syncthreads();
         qm = sm.qmax[0];
 #pragma unroll
@@ -209,12 +249,7 @@ __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
 #pragma unroll
         for (int j = 0; j < kMaxKeys / 32; ++j) {
             const int t = lane + 32 * j;
-            if (t < n16) {
-                const float u = z[j] * fk[j];
-                const __half hi = __float2half_rn(u);
-                *reinterpret_cast<__half*>(sm.P + h * kPStride + 2 * t) = hi;
-                *reinterpret_cast<__half*>(sm.Pl + h * kPStride + 2 * t) = __float2half_rn(u - __half2float(hi));
-            }
+            if (t < n16) *reinterpret_cast<__half*>(sm.P + h * kPStride + 2 * t) = __float2half_rn(z[j] * fk[j]);
         }
         if (lane == 0) {
             sm.ml[h][0] = m;
@@ -230,10 +265,8 @@ __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) o[n][j] = 0.0f;
     for (int kk = 0; kk < (n16 >> 4); ++kk) {
-        uint32_t a0, a1, a2, a3, l0, l1, l2, l3;
-        const uint32_t poff = (uint32_t)((lane & 15) * kPStride + (16 * kk + 8 * (lane >> 4)) * 2);
-        ldsm_x4(sP + poff, a0, a1, a2, a3);
-        ldsm_x4(sPl + poff, l0, l1, l2, l3);
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(sP + (uint32_t)((lane & 15) * kPStride + (16 * kk + 8 * (lane >> 4)) * 2), a0, a1, a2, a3);
         const int mi = lane >> 3;
         const int key = 16 * kk + (mi & 1) * 8 + (lane & 7);
 #pragma unroll
@@ -242,48 +275,52 @@ __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
             ldsm_x4_t(sK + swz(key, 4 * warp + 2 * np + (mi >> 1)), b0, b1, b2, b3);
             mma_f16(o[2 * np], a0, a1, a2, a3, b0, b1);
             mma_f16(o[2 * np + 1], a0, a1, a2, a3, b2, b3);
-            mma_f16(o[2 * np], l0, l1, l2, l3, b0, b1);
-            mma_f16(o[2 * np + 1], l0, l1, l2, l3, b2, b3);
         }
     }
 
-    // ---- combine: every CTA pushes the slice of O_r and its (max, sum) that CTA c
-    // owns (dims [c DS, (c + 1) DS)) into c's key buffer, which is free once every
-    // CTA has finished P V
-    const int DS = kD / (int)C;
+    // ---- combine: every CTA stores the slice of O_r and its (max, sum) that CTA c owns
+    // (dims [c DS, (c + 1) DS)) into c's key buffer, free once every CTA has finished
+    // P V; 16 bytes at a time (lane pairs swap halves so each holds four consecutive
+    // dims of one head)
+    const int DS = kD / (int)C;   // output dims owned by each rank
     const int rstride = DS + 4;   // floats per head row of a received slice
-    float* Rf = reinterpret_cast<float*>(sm.K);                 // [C][16][rstride]
-    float* MLf = Rf + (int)C * kH * rstride;                    // [C][16][2]
+    float* R = reinterpret_cast<float*>(sm.K);   // [C][16][rstride]
+    float* RML = R + (int)C * kH * rstride;      // [C][16][2]
     cl::sync();   // #1: every CTA is done with its key buffer
     {
-        const uint32_t sR = (uint32_t)__cvta_generic_to_shared(Rf);
+        const uint32_t sR = (uint32_t)__cvta_generic_to_shared(R);
+        const bool odd = (qd & 1) != 0;
+        const int head = odd ? g + 8 : g;
 #pragma unroll
         for (int n = 0; n < 4; ++n) {
-            const int d = 32 * warp + 8 * n + 2 * qd;
+            const float r0 = __shfl_xor_sync(0xFFFFFFFFu, odd ? o[n][0] : o[n][2], 1);
+            const float r1 = __shfl_xor_sync(0xFFFFFFFFu, odd ? o[n][1] : o[n][3], 1);
+            const int d = 32 * warp + 8 * n + 2 * (qd & 2);
             const uint32_t owner = (uint32_t)(d / DS);
-            const int dd = d - (int)owner * DS;
-            const uint32_t a0 = sR + (uint32_t)(((int)rank * kH + g) * rstride + dd) * 4u;
-            const uint32_t a1 = sR + (uint32_t)(((int)rank * kH + g + 8) * rstride + dd) * 4u;
-            cl::st_v2f(cl::map_rank(a0, owner), o[n][0], o[n][1]);
-            cl::st_v2f(cl::map_rank(a1, owner), o[n][2], o[n][3]);
+            const int off = ((int)rank * kH + head) * rstride + (d - (int)owner * DS);
+            const uint32_t a = cl::map_rank(sR + 4u * (uint32_t)off, owner);
+            if (odd)
+                cl::st_v4f(a, r0, r1, o[n][2], o[n][3]);
+            else
+                cl::st_v4f(a, o[n][0], o[n][1], r0, r1);
         }
         if (tid < kH * (int)C) {
             const uint32_t owner = (uint32_t)(tid / kH);
             const int h = tid % kH;
-            const uint32_t a = (uint32_t)__cvta_generic_to_shared(MLf + ((int)rank * kH + h) * 2);
+            const uint32_t a = (uint32_t)__cvta_generic_to_shared(RML + ((int)rank * kH + h) * 2);
             cl::st_v2f(cl::map_rank(a, owner), sm.ml[h][0], sm.ml[h][1]);
         }
     }
     cl::sync();   // #2: every slice has arrived; nothing reads another CTA's memory after this
     if (tid < kH) {
         float M = -INFINITY;
-        for (uint32_t c = 0; c < C; ++c) M = fmaxf(M, MLf[((int)c * kH + tid) * 2]);
+        for (uint32_t c = 0; c < C; ++c) M = fmaxf(M, RML[((int)c * kH + tid) * 2]);
         const float Mu = (M == -INFINITY) ? 0.0f : M;
         float L = 0.0f;
         for (uint32_t c = 0; c < C; ++c) {
-            const float wgt = exp2f(MLf[((int)c * kH + tid) * 2] - Mu);
+            const float wgt = exp2f(RML[((int)c * kH + tid) * 2] - Mu);
             sm.cw[c][tid] = wgt;
-            L += MLf[((int)c * kH + tid) * 2 + 1] * wgt;
+            L += RML[((int)c * kH + tid) * 2 + 1] * wgt;
         }
         const float inv = L > 0.0f ? 1.0f / L : 0.0f;
         for (uint32_t c = 0; c < C; ++c) sm.cw[c][tid] *= inv;
@@ -298,7 +335,7 @@ __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
             const int dd = 4 * (e4 - h * per_head);
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
             for (uint32_t c = 0; c < C; ++c) {
-                const float4 x = *reinterpret_cast<const float4*>(Rf + ((int)c * kH + h) * rstride + dd);
+                const float4 x = *reinterpret_cast<const float4*>(R + ((int)c * kH + h) * rstride + dd);
                 const float wgt = sm.cw[c][h];
                 acc.x += x.x * wgt;
                 acc.y += x.y * wgt;
@@ -379,16 +416,17 @@ int max_active_clusters(int C) {
 
 }  // namespace
 
-int attn_cluster_size(int B, int Q, int slots_total, int* keys_per_cta) {
+int attn_cluster_size(int B, int Q, int k, int window, int* main_per_cta, int* swa_per_cta) {
     const int bq = B * Q;
-    if (bq <= 0 || slots_total <= 0 || !set_attributes()) return 0;
+    if (bq <= 0 || k < 0 || window < 0 || k + window <= 0 || !set_attributes()) return 0;
     const int sms = device_sm_count();
     for (int C = nonportable() ? 16 : 8; C >= 1; C >>= 1) {
         if ((int64_t)bq * C > sms) continue;
-        const int n = ((slots_total + C - 1) / C + 15) / 16 * 16;
-        if (n > kMaxKeys) return 0;   // a smaller cluster only lengthens the chunk
+        const int nm = (k + C - 1) / C, nw = (window + C - 1) / C;
+        if (nm + nw > kMaxKeys) return 0;   // a smaller cluster only lengthens the share
         if (max_active_clusters(C) >= bq) {
-            if (keys_per_cta) *keys_per_cta = n;
+            if (main_per_cta) *main_per_cta = nm;
+            if (swa_per_cta) *swa_per_cta = nw;
             return C;
         }
     }

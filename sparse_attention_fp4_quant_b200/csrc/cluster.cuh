@@ -1,5 +1,5 @@
 // cluster.cuh -- thread-block cluster primitives (sm_100a): rank, barrier over
-// the cluster, and loads from another CTA's shared memory.
+// the cluster, and loads from and stores into another CTA's shared memory.
 #pragma once
 #include <stdint.h>
 
@@ -50,6 +50,10 @@ __device__ __forceinline__ uint2 ld_v2(uint32_t addr) {
     uint2 v;
     asm volatile("ld.shared::cluster.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
     return v;
+}
+
+__device__ __forceinline__ void st_v4f(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 
 __device__ __forceinline__ void st_v2f(uint32_t addr, float a, float b) {

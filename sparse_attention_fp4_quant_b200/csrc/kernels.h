@@ -120,7 +120,8 @@ struct AttnParams {
     float* lse;               // [B*Q][16] or null
     int slots_total;          // k + window
     int tiles_per_split;      // split-K form: 64-key tiles per split
-    int keys_per_cta;         // cluster form: key slots per CTA
+    int main_per_cta;         // cluster form: main slots per CTA (CTA r: [r n, (r + 1) n) of k)
+    int swa_per_cta;          // cluster form: window slots per CTA (likewise of the window)
     // workspace
     int32_t* counters;        // [B*Q]
     int32_t* status;          // sticky: set to 1 if a device-side wait timed out
@@ -133,7 +134,7 @@ size_t attn_ws_bytes(int B, int Q, int k, int window);
 void attn_carve_ws(AttnParams& p, int S, void* ws);
 cudaError_t launch_attn(AttnParams& p, int S, cudaStream_t st);
 // One cluster of C CTAs per query; 0 = the shape does not fit.
-int attn_cluster_size(int B, int Q, int slots_total, int* keys_per_cta);
+int attn_cluster_size(int B, int Q, int k, int window, int* main_per_cta, int* swa_per_cta);
 cudaError_t launch_attn_cluster(AttnParams& p, int C, cudaStream_t st);
 
 }  // namespace csa2
