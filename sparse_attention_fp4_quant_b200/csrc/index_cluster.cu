@@ -288,14 +288,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     int32_t* status = p.status;
     int32_t* out = p.out + (int64_t)bq * k;
 
-    if (tid == 0) init_barriers(s.pipe, kEpiN);
-    if (warp == 1) setup_query(s.pipe, p.q + (int64_t)bq * 128, p.q_sc + (int64_t)bq * 16, lane, kTmemCols);
-    for (int i = tid; i < kNB1; i += kThreads) s.hist1[i] = 0;
-    __syncthreads();
-    const uint32_t tbase = s.pipe.tmem_base;
+    // Warp 0 starts the copies as soon as the barriers exist; the other warps set up
+    // the query, TMEM and the histogram meanwhile and meet on named barrier 1 (warp 0
+    // only arrives there).
+    if (warp == 0) {
+        if (lane == 0) init_barriers(s.pipe, kEpiN);
+        __syncwarp();
+        asm volatile("bar.arrive 1, %0;" ::"n"(kThreads) : "memory");
+        producer_dense(s.pipe, p.ik, p.ik_sc, row_base, lo, ntiles, nstages, status, lane);
+    } else {
+        if (warp == 1) setup_query(s.pipe, p.q + (int64_t)bq * 128, p.q_sc + (int64_t)bq * 16, lane, kTmemCols);
+        for (int i = tid - 32; i < kNB1; i += kThreads - 32) s.hist1[i] = 0;
+        tc::tc_fence_before();
+        asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
+        tc::tc_fence_after();
+    }
+    uint32_t tbase = warp == 0 ? 0u : s.pipe.tmem_base;   // warp 0 reads it after scoring
 
     if (warp == 0) {
-        producer_dense(s.pipe, p.ik, p.ik_sc, row_base, lo, ntiles, nstages, status, lane);
     } else if (warp == 1) {
         mma_issuer(s.pipe, ntiles, nstages, status, lane);
     } else {
@@ -312,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int a = t % kAcc;
             const uint32_t aph = (uint32_t)(t / kAcc) & 1u;
             if (!dead && __any_sync(0xFFFFFFFFu, aborted(s.pipe))) dead = true;
-            if (!dead && !__all_sync(0xFFFFFFFFu, tc::mbar_wait(&s.pipe.accfull[a], aph))) {   // warp-uniform
+            if (!dead && !__all_sync(0xFFFFFFFFu, tc::mbar_wait_spin(&s.pipe.accfull[a], aph))) {   // warp-uniform
                 if (lane == 0) raise_abort(s.pipe, status);
                 dead = true;
             }
@@ -366,6 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
+    tbase = s.pipe.tmem_base;
 
     // ---------------------------------------------------------------- select
     const uint32_t K1 = (uint32_t)min(k, nvis);

@@ -131,7 +131,7 @@ __device__ __forceinline__ void producer_dense(P& s, const uint8_t* ik, const ui
         for (int t = 0; t < nstages; ++t) {
             const int slot = t % kStages;
             const uint32_t ph = (uint32_t)(t / kStages) & 1u;
-            if (!tc::mbar_wait(&s.empty[slot], ph ^ 1u)) {
+            if (!tc::mbar_wait_spin(&s.empty[slot], ph ^ 1u)) {
                 raise_abort(s, status);
                 break;
             }
@@ -213,7 +213,7 @@ __device__ __forceinline__ void mma_issuer(P& s, int ntiles, int nstages, int32_
             const uint32_t ph = (uint32_t)(t / kStages) & 1u;
             const int a = t % kAcc;
             const uint32_t aph = (uint32_t)(t / kAcc) & 1u;
-            if (!tc::mbar_wait(&s.full[slot], ph) || !tc::mbar_wait(&s.accempty[a], aph ^ 1u)) {
+            if (!tc::mbar_wait_spin(&s.full[slot], ph) || !tc::mbar_wait_spin(&s.accempty[a], aph ^ 1u)) {
                 raise_abort(s, status);
                 break;
             }
