@@ -8,8 +8,8 @@
 // in swizzled shared memory (K = V), and S = Q K^T (8 keys per warp) and
 // O += P V (64 dims per warp) run on warp-level tensor-core MMAs with the 16
 // heads as the M dimension; the softmax is online across tiles.  P enters P V
-// as two f16 terms (rounded value + remainder).  Splits
-// of one query are merged by the last CTA to finish (atomic ticket).
+// rounded to f16 (fp32 accumulation).  Splits of one query are merged by the
+// last CTA to finish (atomic ticket).
 #include "attn_common.cuh"
 
 namespace csa2 {
@@ -22,8 +22,7 @@ constexpr int kMaxSplitMain = CSA2_MAX_K + kKT;   // main-row ids a split reads 
 struct AttnSmem {
     uint8_t K[kKT * kRowB];   // 64 KB, 16-byte chunks XOR-swizzled by row & 7
     uint8_t Qs[kH * kRowB];   // 16 KB, same swizzle
-    uint8_t P[kH * kKT * 2];  // 2 KB, f16 P (rounded), 8 chunks per row, same swizzle
-    uint8_t Pl[kH * kKT * 2]; // 2 KB, f16 remainder P - rounded(P)
+    uint8_t P[kH * kKT * 2];  // 2 KB, f16 P, 8 chunks per row, same swizzle
     float kf[kKT];            // per-key factor (1 for FP4 rows, token scale for SWA)
     int kvalid[kKT];
     float red_max[8][kH];
@@ -55,7 +54,6 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
     const uint32_t sK = (uint32_t)__cvta_generic_to_shared(sm.K);
     const uint32_t sQ = (uint32_t)__cvta_generic_to_shared(sm.Qs);
     const uint32_t sP = (uint32_t)__cvta_generic_to_shared(sm.P);
-    const uint32_t sPl = (uint32_t)__cvta_generic_to_shared(sm.Pl);
 
     const int ntiles = (p.slots_total + kKT - 1) / kKT;
     const int t0 = split * p.tiles_per_split;
@@ -172,11 +170,8 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
             const uint32_t off0 = g * 128 + ((chunk ^ (g & 7)) << 4) + within;
             const uint32_t off1 = (g + 8) * 128 + ((chunk ^ ((g + 8) & 7)) << 4) + within;
             const float u00 = p00 * f0, u01 = p01 * f1, u10 = p10 * f0, u11 = p11 * f1;
-            const __half2 h0 = __floats2half2_rn(u00, u01), h1 = __floats2half2_rn(u10, u11);
-            *reinterpret_cast<__half2*>(sm.P + off0) = h0;
-            *reinterpret_cast<__half2*>(sm.P + off1) = h1;
-            *reinterpret_cast<uint32_t*>(sm.Pl + off0) = pack_f16(u00 - __low2float(h0), u01 - __high2float(h0));
-            *reinterpret_cast<uint32_t*>(sm.Pl + off1) = pack_f16(u10 - __low2float(h1), u11 - __high2float(h1));
+            *reinterpret_cast<__half2*>(sm.P + off0) = __floats2half2_rn(u00, u01);
+            *reinterpret_cast<__half2*>(sm.P + off1) = __floats2half2_rn(u10, u11);
         }
         float sum0 = p00 + p01, sum1 = p10 + p11;
 #pragma unroll
@@ -217,12 +212,10 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
             }
 #pragma unroll
             for (int kk = 0; kk < kKT / 16; ++kk) {
-                uint32_t a0, a1, a2, a3, l0, l1, l2, l3;
+                uint32_t a0, a1, a2, a3;
                 {
                     const int row = lane & 15, chunk = 2 * kk + (lane >> 4);
-                    const uint32_t off = (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
-                    ldsm_x4(sP + off, a0, a1, a2, a3);
-                    ldsm_x4(sPl + off, l0, l1, l2, l3);
+                    ldsm_x4(sP + (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4)), a0, a1, a2, a3);
                 }
                 const int mi = lane >> 3;
                 const int key = 16 * kk + (mi & 1) * 8 + (lane & 7);
@@ -232,8 +225,6 @@ __global__ void __launch_bounds__(kAT, 2) attn_kernel(AttnParams p) {
                     ldsm_x4_t(sK + swz(key, 8 * warp + 2 * np + (mi >> 1)), b0, b1, b2, b3);
                     mma_f16(o[2 * np], a0, a1, a2, a3, b0, b1);
                     mma_f16(o[2 * np + 1], a0, a1, a2, a3, b2, b3);
-                    mma_f16(o[2 * np], l0, l1, l2, l3, b0, b1);
-                    mma_f16(o[2 * np + 1], l0, l1, l2, l3, b2, b3);
                 }
             }
         }

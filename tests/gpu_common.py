@@ -29,7 +29,8 @@ def attn_close(gpu_bf16, ref):
     ok = err <= TOL_ABS + TOL_REL * np.abs(ref)
     big = np.abs(ref) > 1e-2
     stats = dict(max_abs=float(err.max()) if err.size else 0.0,
-                 max_rel=float((err[big] / np.abs(ref[big])).max()) if big.any() else 0.0)
+                 max_rel=float((err[big] / np.abs(ref[big])).max()) if big.any() else 0.0,
+                 worst=float((err / (TOL_ABS + TOL_REL * np.abs(ref))).max()) if err.size else 0.0)
     return bool(ok.all()), stats
 
 
