@@ -11,12 +11,14 @@
 // (each warp a quarter of the channels of a fifth of the keys), then the CTA's
 // own softmax (one warp per head: max and sum over its keys), then O_r = P V
 // (32 dims per warp; P rounded to f16, fp32 accumulation).  The partial results
-// meet in distributed shared memory: each CTA stores, into CTA c's (by then
-// idle) key buffer, its slice [c * 512 / C, (c + 1) * 512 / C) of O_r (fp32)
-// and its per-head (max, sum); CTA c then forms its slice of the output as
+// meet in distributed shared memory: each CTA keeps its O_r (fp32) and per-head
+// (max, sum) in its own shared memory, and after one cluster barrier CTA c
+// loads the slice [c * 512 / C, (c + 1) * 512 / C) of every rank's O_r and
+// forms its slice of the output as
 //   sum_r 2^(m_r - M) O_r / sum_r 2^(m_r - M) l_r,   M = max_r m_r,
-// from its own shared memory and writes it as bf16.  No partials go to global
-// memory and no CTA waits for a ticket.
+// written as bf16.  (Stores into the owners' memory drained at ~12 bytes per
+// clock and needed a second full barrier.)  No partials go to global memory and
+// no CTA waits for a ticket.
 #include "attn_common.cuh"
 #include "cluster.cuh"
 
@@ -29,21 +31,19 @@ constexpr int kPStride = kMaxKeys * 2 + 16;   // bytes per head row of P (confli
 constexpr int kQG = 4;                        // key-tile groups of the S warps (x 4 channel groups)
 constexpr int kQT = kMaxKeys / 8 / kQG;       // key tiles per S warp
 constexpr int kSStride = kMaxKeys + 4;        // floats per head row of a partial S
-constexpr int kMaxC = 16;                     // largest cluster
 static_assert(kMaxKeys % 32 == 0 && kMaxKeys % (8 * kQG) == 0, "keys per CTA");
 static_assert(kCT / 32 == kH, "one warp per head in the softmax");
 static_assert(2 * kH * kSStride * 4 <= kH * kRowB + kH * kPStride, "partial S fit the Q and P buffers");
-static_assert((kH * (kD + 4 * kMaxC) + kMaxC * kH * 2) * 4 <= kMaxKeys * kRowB, "received slices fit the key buffer");
+static_assert(kH * (kD + 4) * 4 <= kMaxKeys * kRowB, "O_r fits the key buffer");
 
 // 188 KB: the rest of the SM's 256 KB stays L1, which holds the gather's loads in flight
 struct ClAttnSmem {
-    uint8_t K[kMaxKeys * kRowB];   // f16 keys (= values), swizzled; afterwards the received output slices
+    uint8_t K[kMaxKeys * kRowB];   // f16 keys (= values), swizzled; afterwards this CTA's O_r
     uint8_t Qs[kH * kRowB];        // f16 query (prescaled), swizzled; then (with P) the two partial S arrays
     uint8_t P[kH * kPStride];      // f16 P, [head][key]
     float kf[kMaxKeys];            // per-key factor (1 for FP4 rows, token scale for SWA)
     int kvalid[kMaxKeys];
     alignas(16) float ml[kH][2];   // this CTA's (max, sum) per head (log2 units), read by the cluster
-    float cw[kMaxC][kH];           // combine weight of rank c for head h (for this CTA's output slice)
     float qmax[kCT / 32];          // per-warp max |q|
 };
 
@@ -278,74 +278,80 @@ __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
         }
     }
 
-    // ---- combine: every CTA stores the slice of O_r and its (max, sum) that CTA c owns
-    // (dims [c DS, (c + 1) DS)) into c's key buffer, free once every CTA has finished
-    // P V; 16 bytes at a time (lane pairs swap halves so each holds four consecutive
-    // dims of one head)
-    const int DS = kD / (int)C;   // output dims owned by each rank
-    const int rstride = DS + 4;   // floats per head row of a received slice
-    float* R = reinterpret_cast<float*>(sm.K);   // [C][16][rstride]
-    float* RML = R + (int)C * kH * rstride;      // [C][16][2]
-    cl::sync();   // #1: every CTA is done with its key buffer
-    {
-        const uint32_t sR = (uint32_t)__cvta_generic_to_shared(R);
-        const bool odd = (qd & 1) != 0;
-        const int head = odd ? g + 8 : g;
+    // ---- combine: every CTA keeps its O_r (fp32 [16][512]) in its own key buffer (free once
+    // its warps are done with P V) beside its (max, sum) per head; after one cluster barrier,
+    // CTA c loads dims [c DS, (c + 1) DS) of every rank's O_r and the ranks' (max, sum) of the
+    // same head, four ranks' loads in flight together, and forms its output slice
+    //   sum_r 2^(m_r - M) O_r / sum_r 2^(m_r - M) l_r,   M = max_r m_r
+    // (over the ranks in order, four at a time with a running maximum).  The loads are the last
+    // use of another CTA's memory: an arrive after them and a wait at the very end keep every
+    // CTA resident until all have read.
+    constexpr int kOS = kD + 4;   // floats per head row of O_r (conflict-free float2 stores)
+    float* Ow = reinterpret_cast<float*>(sm.K);
+    __syncthreads();   // every warp is done reading the key buffer
 #pragma unroll
-        for (int n = 0; n < 4; ++n) {
-            const float r0 = __shfl_xor_sync(0xFFFFFFFFu, odd ? o[n][0] : o[n][2], 1);
-            const float r1 = __shfl_xor_sync(0xFFFFFFFFu, odd ? o[n][1] : o[n][3], 1);
-            const int d = 32 * warp + 8 * n + 2 * (qd & 2);
-            const uint32_t owner = (uint32_t)(d / DS);
-            const int off = ((int)rank * kH + head) * rstride + (d - (int)owner * DS);
-            const uint32_t a = cl::map_rank(sR + 4u * (uint32_t)off, owner);
-            if (odd)
-                cl::st_v4f(a, r0, r1, o[n][2], o[n][3]);
-            else
-                cl::st_v4f(a, o[n][0], o[n][1], r0, r1);
-        }
-        if (tid < kH * (int)C) {
-            const uint32_t owner = (uint32_t)(tid / kH);
-            const int h = tid % kH;
-            const uint32_t a = (uint32_t)__cvta_generic_to_shared(RML + ((int)rank * kH + h) * 2);
-            cl::st_v2f(cl::map_rank(a, owner), sm.ml[h][0], sm.ml[h][1]);
-        }
+    for (int n = 0; n < 4; ++n) {
+        const int d = 32 * warp + 8 * n + 2 * qd;
+        *reinterpret_cast<float2*>(Ow + g * kOS + d) = make_float2(o[n][0], o[n][1]);
+        *reinterpret_cast<float2*>(Ow + (g + 8) * kOS + d) = make_float2(o[n][2], o[n][3]);
     }
-    cl::sync();   // #2: every slice has arrived; nothing reads another CTA's memory after this
-    if (tid < kH) {
-        float M = -INFINITY;
-        for (uint32_t c = 0; c < C; ++c) M = fmaxf(M, RML[((int)c * kH + tid) * 2]);
-        const float Mu = (M == -INFINITY) ? 0.0f : M;
-        float L = 0.0f;
-        for (uint32_t c = 0; c < C; ++c) {
-            const float wgt = exp2f(RML[((int)c * kH + tid) * 2] - Mu);
-            sm.cw[c][tid] = wgt;
-            L += RML[((int)c * kH + tid) * 2 + 1] * wgt;
-        }
-        const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-        for (uint32_t c = 0; c < C; ++c) sm.cw[c][tid] *= inv;
-        if (p.lse && rank == 0) p.lse[(int64_t)bq * kH + tid] = L > 0.0f ? (Mu + log2f(L)) * 0.6931471805599453f : -INFINITY;
-    }
-    __syncthreads();
+    cl::sync();   // every CTA's O_r and (max, sum) are in place
     {
-        const int per_head = DS / 4;   // float4 per head in the slice
+        const int DS = kD / (int)C;       // output dims owned by each rank
+        const int per_head = DS / 4;      // float4 of one head's slice
+        const uint32_t sO = (uint32_t)__cvta_generic_to_shared(Ow);
+        const uint32_t sML = (uint32_t)__cvta_generic_to_shared(&sm.ml[0][0]);
         uint16_t* out = p.out + (int64_t)bq * kH * kD;
         for (int e4 = tid; e4 < kH * per_head; e4 += kCT) {
             const int h = e4 / per_head;
-            const int dd = 4 * (e4 - h * per_head);
+            const int d = (int)rank * DS + 4 * (e4 - h * per_head);
+            const uint32_t oa = sO + 4u * (uint32_t)(h * kOS + d), ma = sML + 8u * (uint32_t)h;
+            float M = -INFINITY, L = 0.0f;
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (uint32_t c = 0; c < C; ++c) {
-                const float4 x = *reinterpret_cast<const float4*>(R + ((int)c * kH + h) * rstride + dd);
-                const float wgt = sm.cw[c][h];
-                acc.x += x.x * wgt;
-                acc.y += x.y * wgt;
-                acc.z += x.z * wgt;
-                acc.w += x.w * wgt;
+            for (uint32_t r0 = 0; r0 < C; r0 += 4) {
+                uint4 x[4];
+                uint2 ml[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (r0 + j < C) {
+                        x[j] = cl::ld_v4(cl::map_rank(oa, r0 + j));
+                        ml[j] = cl::ld_v2(cl::map_rank(ma, r0 + j));
+                    }
+                }
+                float Mn = M;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (r0 + j < C) Mn = fmaxf(Mn, __uint_as_float(ml[j].x));
+                const float Mu = (Mn == -INFINITY) ? 0.0f : Mn;
+                const float sc = (M == -INFINITY) ? 0.0f : exp2f(M - Mu);   // rescale what came before
+                L *= sc;
+                acc.x *= sc;
+                acc.y *= sc;
+                acc.z *= sc;
+                acc.w *= sc;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (r0 + j < C) {
+                        const float w = exp2f(__uint_as_float(ml[j].x) - Mu);
+                        L += __uint_as_float(ml[j].y) * w;
+                        acc.x += __uint_as_float(x[j].x) * w;
+                        acc.y += __uint_as_float(x[j].y) * w;
+                        acc.z += __uint_as_float(x[j].z) * w;
+                        acc.w += __uint_as_float(x[j].w) * w;
+                    }
+                }
+                M = Mn;
             }
-            *reinterpret_cast<uint2*>(out + h * kD + (int)rank * DS + dd) =
-                make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
+            const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+            *reinterpret_cast<uint2*>(out + h * kD + d) =
+                make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
+            if (p.lse && rank == 0 && d == 0)
+                p.lse[(int64_t)bq * kH + h] = L > 0.0f ? (((M == -INFINITY) ? 0.0f : M) + log2f(L)) * 0.6931471805599453f
+                                                       : -INFINITY;
         }
     }
+    cl::arrive_release();   // this CTA has read every rank's memory it needs
+    cl::wait_acquire();     // ... and so has every other: no CTA leaves while it could be read
 }
 
 DeviceOnce g_attr;

@@ -1,5 +1,6 @@
 // cluster.cuh -- thread-block cluster primitives (sm_100a): rank, barrier over
-// the cluster, and loads from and stores into another CTA's shared memory.
+// the cluster (whole or as arrive / wait), and loads from and stores into
+// another CTA's shared memory.
 #pragma once
 #include <stdint.h>
 
@@ -23,6 +24,10 @@ __device__ __forceinline__ uint32_t ctas() {
 __device__ __forceinline__ void sync() {
     asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
+
+// The two halves of sync(): arrive early, wait where the ordering is needed.
+__device__ __forceinline__ void arrive_release() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
+__device__ __forceinline__ void wait_acquire() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
 
 // Address of the same shared-memory variable in CTA `r` of the cluster.
 __device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t r) {
