@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(kCT, 1) attn_cluster_kernel(AttnParams p) {
                                                        : -INFINITY;
         }
     }
-    cl::arrive_release();   // this CTA has read every rank's memory it needs
+    cl::arrive_relaxed();   // this CTA has read every rank's memory it needs
     cl::wait_acquire();     // ... and so has every other: no CTA leaves while it could be read
 }
 

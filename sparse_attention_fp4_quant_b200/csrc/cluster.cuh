@@ -27,6 +27,9 @@ __device__ __forceinline__ void sync() {
 
 // The two halves of sync(): arrive early, wait where the ordering is needed.
 __device__ __forceinline__ void arrive_release() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
+// An arrive that orders nothing: for a CTA whose remaining reads of other CTAs' memory
+// have all returned (their values are used), so its later global stores need not drain first.
+__device__ __forceinline__ void arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory"); }
 __device__ __forceinline__ void wait_acquire() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
 
 // Address of the same shared-memory variable in CTA `r` of the cluster.
