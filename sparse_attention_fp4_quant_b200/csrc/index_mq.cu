@@ -123,14 +123,14 @@ __global__ void __launch_bounds__(kMqThreads, 1) mq_score_kernel(SelectParams p,
             bool stop = false;
             for (int t = 0; t < nstages && !stop; ++t) {
                 const int slot = t % kMqRing;
-                if (!tc::mbar_wait(&s.full[slot], (uint32_t)(t / kMqRing) & 1u)) {
+                if (!tc::mbar_wait_spin(&s.full[slot], (uint32_t)(t / kMqRing) & 1u)) {
                     raise_abort(s, status);
                     break;
                 }
                 const int ntl = min(kTPS, ntiles - t * kTPS);
                 for (int i = 0; i < ntl; ++i, ++u) {
                     const int a = u % kAccT;
-                    if (!tc::mbar_wait(&s.accempty[a], ((uint32_t)(u / kAccT) & 1u) ^ 1u)) {
+                    if (!tc::mbar_wait_spin(&s.accempty[a], ((uint32_t)(u / kAccT) & 1u) ^ 1u)) {
                         raise_abort(s, status);
                         stop = true;
                         break;
@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(kMqThreads, 1) mq_score_kernel(SelectParams p,
             for (int i = 0; i < ntl; ++i, ++u) {
                 const int a = u % kAccT;
                 if (!dead && __any_sync(0xFFFFFFFFu, aborted(s))) dead = true;
-                if (!dead && !__all_sync(0xFFFFFFFFu, tc::mbar_wait(&s.accfull[a], (uint32_t)(u / kAccT) & 1u))) {
+                if (!dead && !__all_sync(0xFFFFFFFFu, tc::mbar_wait_spin(&s.accfull[a], (uint32_t)(u / kAccT) & 1u))) {
                     if (lane == 0) raise_abort(s, status);
                     dead = true;
                 }

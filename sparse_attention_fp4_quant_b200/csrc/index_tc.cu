@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int t = 0; t < nstages && !stop; ++t) {
             const int a = t % kAcc;
             const uint32_t aph = (uint32_t)(t / kAcc) & 1u;
-            const bool ok = __all_sync(0xFFFFFFFFu, tc::mbar_wait(&s.pipe.accfull[a], aph));  // warp-uniform
+            const bool ok = __all_sync(0xFFFFFFFFu, tc::mbar_wait_spin(&s.pipe.accfull[a], aph));  // warp-uniform
             if (!ok && lane == 0) raise_abort(s.pipe, status);
             tc::tc_fence_after();
             uint32_t v[kTPG][16];
