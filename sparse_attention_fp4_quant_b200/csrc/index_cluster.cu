@@ -33,8 +33,10 @@ namespace {
 
 using namespace pipe;
 
-constexpr int kThreads = 320;              // warp 0 copies, warp 1 MMA, warps 2-9 epilogue
+constexpr int kThreads = 512;              // warp 0 copies, warp 1 MMA, warps 2-9 epilogue; all 16 select
 constexpr int kEpiN = 256;
+constexpr int kEpiWarps = kEpiN / 32;
+constexpr int kSwW = kThreads / 32;        // warps that sweep the stored keys: four per TMEM lane quarter
 constexpr int kTPG = kTPS / 2;             // tiles of a stage per epilogue warp group
 constexpr int kRing = 8;                   // shared-memory stages in flight
 constexpr int kMaxTiles = 256;             // 32,768 entries per CTA
@@ -43,8 +45,8 @@ constexpr uint32_t kTmemCols = kPipeCols + kMaxTiles;
 constexpr int kWords = kMaxTiles * kTile / 32;          // bitmap words over the CTA's entries
 constexpr int kNB1 = 2048, kNB2 = 2048, kNB3 = 1024;   // radix digits: bits 31..21, 20..10, 9..0
 constexpr int kSel = 256;                  // threads of the scans (warps 0-7)
-constexpr int kCandPerWarp = 256;          // candidates (keys of the threshold's top bin) a sweeping warp lists
-constexpr int kCandCap = 8 * kCandPerWarp; // and a CTA
+constexpr int kCandPerWarp = 128;          // candidates (keys of the threshold's top bin) a sweeping warp lists
+constexpr int kCandCap = kSwW * kCandPerWarp; // and a CTA
 constexpr int kGatherCap = 8192;           // candidates of a cluster gathered for the local select
 constexpr uint32_t kSlowPath = 0xFFFFFFFFu;
 constexpr int kSelWarps = kSel / 32;
@@ -58,12 +60,12 @@ struct ClSmem {
     alignas(16) uint32_t hist1[kNB1];
     uint32_t wsum[kSelWarps];               // scan: per-warp totals
     uint32_t res[2];                        // find_bin: (bin, keys above the bin)
-    uint32_t wcnt[8][2];                    // per sweeping warp: keys > T, keys == T
+    uint32_t wcnt[kSwW][2];                 // per sweeping warp: keys > T, keys == T
     alignas(8) uint32_t pub[2];             // this CTA's (entries above bin d1, candidates), read by the cluster
     alignas(8) uint32_t pub2[2];            // (> T, == T) counts of the multi-pass path, read by the cluster
     uint32_t cbase[2];                      // this CTA's tie quota and output offset
-    uint32_t wcand[8];                      // candidates each sweeping warp found (may exceed its list)
-    alignas(8) uint32_t coarse[64];         // hist1 in 64 bins of 32
+    uint32_t wcand[kSwW];                   // candidates each sweeping warp found (may exceed its list)
+    alignas(8) uint32_t coarse[16][64];     // every rank's hist1 in 64 bins of 32, pushed by that rank
     uint32_t fast;                          // candidates of the cluster, or kSlowPath
     uint32_t peer[16][2];                   // per CTA: entries above bin d1, candidates of lower ranks
     uint32_t rcnt[16][2];                   // per CTA: candidates above T, equal to T
@@ -132,18 +134,12 @@ __device__ __forceinline__ uint32_t block_scan_excl(ClSmem& s, uint32_t v, int t
 // s.res for the CTA.
 __device__ __forceinline__ void find_top_bin(ClSmem& s, uint32_t C, uint32_t R, int lane) {
     constexpr int RG = 4;   // CTAs whose loads are in flight together
-    // lane l: coarse bins 2l and 2l + 1 (the highest bins on lane 31)
+    // lane l: coarse bins 2l and 2l + 1 (the highest bins on lane 31), every rank's in this CTA
     uint32_t lo = 0, hi = 0;
-    const uint32_t ca = tc::smem_u32(&s.coarse[2 * lane]);
-    for (uint32_t r0 = 0; r0 < C; r0 += RG) {
-        uint2 x[RG];
-#pragma unroll
-        for (int g = 0; g < RG; ++g) x[g] = r0 + g < C ? cl::ld_v2(cl::map_rank(ca, r0 + g)) : make_uint2(0u, 0u);
-#pragma unroll
-        for (int g = 0; g < RG; ++g) {
-            lo += x[g].x;
-            hi += x[g].y;
-        }
+    for (uint32_t r = 0; r < C; ++r) {
+        const uint2 x = *reinterpret_cast<const uint2*>(&s.coarse[r][2 * lane]);
+        lo += x.x;
+        hi += x.y;
     }
     uint32_t suf = lo + hi;   // keys in this lane's coarse bins and every higher lane's
 #pragma unroll
@@ -251,16 +247,16 @@ __device__ __forceinline__ void find_bin(ClSmem& s, const uint32_t* hist, uint32
     __syncthreads();
 }
 
-// Visit every stored key of this CTA, 32 tile columns at a time: warps 2-9,
-// TMEM lane quarter q = warp % 4, columns [128 h, 128 h + 128) with
-// h = (warp - 2) / 4.  f(v, c0, q) gets the keys of columns c0 .. c0 + 31 of
-// this lane; column c of lane l holds CTA-local entry 128 c + 32 q + l.
+// Visit every stored key of this CTA, 32 tile columns at a time: all 16 warps,
+// TMEM lane quarter q = warp % 4, columns [64 h, 64 h + 64) with h = warp / 4.
+// f(v, c0, q) gets the keys of columns c0 .. c0 + 31 of this lane; column c of
+// lane l holds CTA-local entry 128 c + 32 q + l.
 template <class F>
 __device__ __forceinline__ void sweep_cols(uint32_t tbase, int warp, int ntiles, F&& f) {
-    if (warp < 2) return;
-    const int quarter = warp & 3, half = (warp - 2) >> 2;
+    static_assert(kSwW == 16 && kMaxTiles == 4 * 64, "four warps of 64 columns per lane quarter");
+    const int quarter = warp & 3, part = warp >> 2;
     const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
-    for (int c0 = half * 128; c0 < min(ntiles, half * 128 + 128); c0 += 32) {
+    for (int c0 = part * 64; c0 < min(ntiles, part * 64 + 64); c0 += 32) {
         uint32_t v[32];
         tc::tmem_ld_32x32b_x32(tbase + lanes + kColKeys + (uint32_t)c0, v);
         tc::tmem_ld_wait();
@@ -271,6 +267,7 @@ __device__ __forceinline__ void sweep_cols(uint32_t tbase, int warp, int ntiles,
 __global__ void __launch_bounds__(kThreads, 1)
     index_cluster_kernel(SelectParams p) {
     pdl_enter();
+    cl::arrive_relaxed();   // waited on before the first store into another CTA (every CTA has started)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     ClSmem& s = *reinterpret_cast<ClSmem*>(smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -308,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
     } else if (warp == 1) {
         mma_issuer(s.pipe, ntiles, nstages, status, lane);
-    } else {
+    } else if (warp < 2 + kEpiWarps) {
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;             // TMEM lanes this warp may read
         const int group = (warp - 2) >> 2;        // tiles 2*group, 2*group+1 of each stage
@@ -377,6 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc::tc_fence_after();
     tbase = s.pipe.tmem_base;
+    cl::wait_acquire();
 
     // ---------------------------------------------------------------- select
     const uint32_t K1 = (uint32_t)min(k, nvis);
@@ -395,12 +393,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint2* gath = wlist + kCandCap;                            // the cluster's, gathered: (key, entry | rank << 16)
     for (int i = tid; i < kNB2 + kNB3 + 2 * kWords; i += kThreads) hist2[i] = 0;
     if (tid < 32) s.rcnt[tid >> 1][tid & 1] = 0;
-    if (warp >= 2) {   // hist1 in coarse bins of 32, for the cluster's two-level search
+    {   // hist1 in coarse bins of 32, pushed to every rank for the cluster's two-level search
+        static_assert(kSwW * 4 == 64, "four coarse bins per warp");
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int cb = 8 * (warp - 2) + i;
+        for (int i = 0; i < 4; ++i) {
+            const int cb = 4 * warp + i;
             const uint32_t x = __reduce_add_sync(0xFFFFFFFFu, s.hist1[32 * cb + lane]);
-            if (lane == 0) s.coarse[cb] = x;
+            if ((uint32_t)lane < C) cl::st_u32(cl::map_rank(tc::smem_u32(&s.coarse[rank][cb]), (uint32_t)lane), x);
         }
     }
 
@@ -415,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // a bit transpose of the lanes' column masks); an entry of bin d1 is a
     // candidate, appended to this CTA's list.
     uint32_t above = 0, nlist = 0;   // nlist: this warp's candidates (warp-uniform)
-    uint2* mylist = wlist + (warp >= 2 ? warp - 2 : 0) * kCandPerWarp;
+    uint2* mylist = wlist + warp * kCandPerWarp;
     const uint32_t top = ((d1 + 1u) << 21) - 1u;   // keys above bin d1 are > top (none when d1 = 2047)
     const uint32_t bot = d1 << 21;                 // keys of bin d1: key - bot < 2^21
     sweep_cols(tbase, warp, ntiles, [&](const uint32_t(&v)[32], int c0, int q) {
@@ -456,22 +455,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     });
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xFFFFFFFFu, above, o);
-    if (warp >= 2 && lane == 0) {
-        s.wcnt[warp - 2][0] = above;
-        s.wcand[warp - 2] = nlist;
+    if (lane == 0) {
+        s.wcnt[warp][0] = above;
+        s.wcand[warp] = nlist;
     }
     tc::tc_fence_before();
     __syncthreads();
-    if (warp >= 2) {   // compact the warps' lists into this CTA's list, in warp order
+    {   // compact the warps' lists into this CTA's list, in warp order
         uint32_t base = 0;
-        for (int w = 0; w < warp - 2; ++w) base += min(s.wcand[w], (uint32_t)kCandPerWarp);
+        for (int w = 0; w < warp; ++w) base += min(s.wcand[w], (uint32_t)kCandPerWarp);
         const uint32_t n = min(nlist, (uint32_t)kCandPerWarp);
         for (uint32_t i = lane; i < n; i += 32) cand[base + i] = mylist[i];
     }
     if (tid == 0) {
         uint32_t a = 0, n = 0;
         bool over = false;
-        for (int w = 0; w < 8; ++w) {
+        for (int w = 0; w < kSwW; ++w) {
             a += s.wcnt[w][0];
             n += s.wcand[w];
             over = over || s.wcand[w] > (uint32_t)kCandPerWarp;
@@ -628,16 +627,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             gt += __shfl_xor_sync(0xFFFFFFFFu, gt, o);
             eq += __shfl_xor_sync(0xFFFFFFFFu, eq, o);
         }
-        if (warp >= 2 && lane == 0) {
-            s.wcnt[warp - 2][0] = gt;
-            s.wcnt[warp - 2][1] = eq;
+        if (lane == 0) {
+            s.wcnt[warp][0] = gt;
+            s.wcnt[warp][1] = eq;
         }
         tc::tc_fence_before();
         __syncthreads();
         if (warp == 1) tc::tmem_dealloc(tbase, kTmemCols);   // no TMEM reads past this point
         if (tid == 0) {
             uint32_t g = 0, e = 0;
-            for (int w = 0; w < 8; ++w) {
+            for (int w = 0; w < kSwW; ++w) {
                 g += s.wcnt[w][0];
                 e += s.wcnt[w][1];
             }
