@@ -253,6 +253,11 @@ __device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
 
 // The row's four key block scales as (sk_b, sk_b) pairs.
 struct KeyScales {
@@ -273,14 +278,18 @@ __device__ __forceinline__ KeyScales key_scales(uint32_t sk_bytes) {
 //   score = ((w0 r0 + w1 r1) + w2 r2) + w3 r3,
 // every product and sum one fp32 rounding.  Heads (0, 1) and (2, 3) run as
 // packed pairs (lane by lane the same IEEE operations).  w01 = (w0, w1), w23 = (w2, w3).
+// Each block product is exact in fp32 (the accumulator has at most 16
+// significant bits, an E4M3 scale at most 4), so a fused multiply-add of the
+// next block onto the running sum rounds exactly as the separate add of that
+// product does: d_h takes one multiply and three fused multiply-adds.  The head
+// products w_h r_h are not exact and keep their own rounding.
 __device__ __forceinline__ float score_of(const uint32_t (&v)[16], const KeyScales& ks, uint64_t w01, uint64_t w23) {
-    uint64_t d01 = 0, d23 = 0;
+    uint64_t d01 = f2mul(f2pack(__uint_as_float(v[0]), __uint_as_float(v[1])), ks.s2[0]);
+    uint64_t d23 = f2mul(f2pack(__uint_as_float(v[2]), __uint_as_float(v[3])), ks.s2[0]);
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-        const uint64_t t01 = f2mul(f2pack(__uint_as_float(v[4 * b]), __uint_as_float(v[4 * b + 1])), ks.s2[b]);
-        const uint64_t t23 = f2mul(f2pack(__uint_as_float(v[4 * b + 2]), __uint_as_float(v[4 * b + 3])), ks.s2[b]);
-        d01 = b == 0 ? t01 : f2add(d01, t01);
-        d23 = b == 0 ? t23 : f2add(d23, t23);
+    for (int b = 1; b < 4; ++b) {
+        d01 = f2fma(f2pack(__uint_as_float(v[4 * b]), __uint_as_float(v[4 * b + 1])), ks.s2[b], d01);
+        d23 = f2fma(f2pack(__uint_as_float(v[4 * b + 2]), __uint_as_float(v[4 * b + 3])), ks.s2[b], d23);
     }
     float r0, r1, r2, r3;
     f2unpack(d01, r0, r1);
