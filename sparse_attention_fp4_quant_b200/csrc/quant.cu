@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(256) index_k_proj_rows_kernel(const uint16_t* 
 // one NVFP4 block, the CTA quantises its block alone.  The remaining CTAs
 // quantise the latent rows, one thread per 16 channels.
 constexpr int kAppRows = 32;
-constexpr int kAppThreads = kAppRows * 16;
+constexpr int kAppThreads = kAppRows * 4;   // projection: one row x four outputs per thread
 constexpr int kAppXStride = kD + 8;   // bf16 per staged row (16 bytes of padding: no bank conflicts)
 constexpr int kAppSmem = kD * 16 * 4 + kAppRows * kAppXStride * 2 + kAppRows * 16 * 4;
 
@@ -262,12 +262,21 @@ __global__ void __launch_bounds__(kAppThreads) append_kernel(const uint16_t* __r
     }
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
     __syncthreads();
-    const int rr = tid >> 4, o = tid & 15;
+    // four chains per thread (outputs 4 og .. 4 og + 3 of row rr), each in channel order: one
+    // load of x and one 16-byte load of W feed four fused multiply-adds
+    const int rr = tid >> 2, og = tid & 3;
     const uint16_t* xr = xs + rr * kAppXStride;
-    float acc = 0.0f;
-#pragma unroll 16
-    for (int c = 0; c < kD; ++c) acc = __fmaf_rn(__uint_as_float((uint32_t)xr[c] << 16), Wb[c * 16 + o], acc);
-    outs[rr * 16 + o] = acc;
+    float acc0 = 0.0f, acc1 = 0.0f, acc2 = 0.0f, acc3 = 0.0f;
+#pragma unroll 8
+    for (int c = 0; c < kD; ++c) {
+        const float xv = __uint_as_float((uint32_t)xr[c] << 16);
+        const float4 w = *reinterpret_cast<const float4*>(Wb + c * 16 + 4 * og);
+        acc0 = __fmaf_rn(xv, w.x, acc0);
+        acc1 = __fmaf_rn(xv, w.y, acc1);
+        acc2 = __fmaf_rn(xv, w.z, acc2);
+        acc3 = __fmaf_rn(xv, w.w, acc3);
+    }
+    *reinterpret_cast<float4*>(outs + rr * 16 + 4 * og) = make_float4(acc0, acc1, acc2, acc3);
     __syncthreads();
     if (tid < kAppRows && r0 + tid < rows) {
         float v[16];
