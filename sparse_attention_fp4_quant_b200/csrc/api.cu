@@ -184,6 +184,8 @@ csa2_status csa2_pool_build(const float* blockmax, const csa2_kv* kv, const int3
     p.out = pool_out;
     int S = select_splits(CSA2_OP_POOL_BUILD, B, Q, kv->cap, max_blocks, 0);
     select_carve_ws(p, S, ws, B, Q, max_blocks);
+    const int C = pool_build_cluster_size(p);   // decode-sized query counts: the cluster radix select
+    if (C > 0) return cuda_status(launch_pool_build_cluster(p, C, (cudaStream_t)stream));
     return cuda_status(launch_select(CSA2_OP_POOL_BUILD, p, S, (cudaStream_t)stream));
 }
 

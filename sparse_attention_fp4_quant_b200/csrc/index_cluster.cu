@@ -264,6 +264,9 @@ __device__ __forceinline__ void sweep_cols(uint32_t tbase, int warp, int ntiles,
     }
 }
 
+// MODE 0: index + Top-K (keys = the fixed-order scores of the visible entries);
+// MODE 1: pool build (keys = the block maxima of the visible blocks, items = block ids).
+template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     index_cluster_kernel(SelectParams p) {
     pdl_enter();
@@ -277,9 +280,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int k = p.k;
     const int nvis = n_visible(p.q_pos[bq], p.n_entries[b], p.m, p.cap);
     const int64_t row_base = (int64_t)b * p.cap;
-    // this CTA's entries [lo, hi); the host keeps the chunk within kMaxTiles tiles
-    const int chunk = ((nvis + (int)C - 1) / (int)C + kTile - 1) / kTile * kTile;
-    const int lo = min(nvis, (int)rank * chunk), hi = min(nvis, lo + chunk);
+    // the items: visible entries, or visible blocks of 8 entries (at most nb_cap)
+    const int nitems = MODE == 0 ? nvis : (int)min((int64_t)((nvis + kBlk - 1) / kBlk), p.nb_cap);
+    // this CTA's items [lo, hi); the host keeps the chunk within kMaxTiles tiles
+    const int chunk = ((nitems + (int)C - 1) / (int)C + kTile - 1) / kTile * kTile;
+    const int lo = min(nitems, (int)rank * chunk), hi = min(nitems, lo + chunk);
     const int ntiles = (hi - lo + kTile - 1) / kTile;
     const int nstages = (ntiles + kTPS - 1) / kTPS;
     int32_t* status = p.status;
@@ -287,8 +292,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // Warp 0 starts the copies as soon as the barriers exist; the other warps set up
     // the query, TMEM and the histogram meanwhile and meet on named barrier 1 (warp 0
-    // only arrives there).
-    if (warp == 0) {
+    // only arrives there).  The pool build has no pipeline: TMEM and the histogram only.
+    if constexpr (MODE == 1) {
+        if (warp == 1) tc::tmem_alloc(&s.pipe.tmem_base, kTmemCols);
+        for (int i = tid; i < kNB1; i += kThreads) s.hist1[i] = 0;
+        tc::tc_fence_before();
+        __syncthreads();
+        tc::tc_fence_after();
+    } else if (warp == 0) {
         if (lane == 0) init_barriers(s.pipe, kEpiN);
         __syncwarp();
         asm volatile("bar.arrive 1, %0;" ::"n"(kThreads) : "memory");
@@ -300,9 +311,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
         tc::tc_fence_after();
     }
-    uint32_t tbase = warp == 0 ? 0u : s.pipe.tmem_base;   // warp 0 reads it after scoring
+    uint32_t tbase = (MODE == 0 && warp == 0) ? 0u : s.pipe.tmem_base;   // warp 0 reads it after scoring
 
-    if (warp == 0) {
+    if constexpr (MODE == 1) {
+        // ------------------------------------------------------------ block maxima
+        // warps 2-9: lane quarter q, columns [128 h, 128 h + 128) (h = (warp - 2) / 4); the key of
+        // column c, lane l is block lo + 128 c + 32 q + l; eight loads in flight per lane
+        if (warp >= 2 && warp < 2 + kEpiWarps) {
+            const int quarter = warp & 3, half = (warp - 2) >> 2;
+            const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
+            const float* bmr = p.blockmax + (int64_t)bq * p.nb_cap;
+            for (int c0 = half * 128; c0 < min(ntiles, half * 128 + 128); c0 += 8) {
+                float v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int e = lo + 128 * (c0 + j) + 32 * quarter + lane;
+                    v[j] = (c0 + j < ntiles && e < hi) ? __ldg(bmr + e) : 0.0f;
+                }
+#pragma unroll
+                for (int j = 0; j < 8; j += 2) {
+                    uint32_t key[2];
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const int e = lo + 128 * (c0 + j + i) + 32 * quarter + lane;
+                        const bool valid = c0 + j + i < ntiles && e < hi;
+                        key[i] = valid ? score_key(v[j + i]) : 0u;
+                        if (valid) atomicAdd(&s.hist1[key[i] >> 21], 1u);
+                    }
+                    if (c0 + j + 1 < ntiles) tc::tmem_st_32x32b_x2(tbase + lanes + kColKeys + (uint32_t)(c0 + j), key[0], key[1]);
+                    else if (c0 + j < ntiles) tc::tmem_st_32x32b_x1(tbase + lanes + kColKeys + (uint32_t)(c0 + j), key[0]);
+                }
+            }
+            tc::tmem_st_wait();
+        }
+    } else if (warp == 0) {
     } else if (warp == 1) {
         mma_issuer(s.pipe, ntiles, nstages, status, lane);
     } else if (warp < 2 + kEpiWarps) {
@@ -377,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     cl::wait_acquire();
 
     // ---------------------------------------------------------------- select
-    const uint32_t K1 = (uint32_t)min(k, nvis);
+    const uint32_t K1 = (uint32_t)min(k, nitems);
     if (K1 == 0) {   // the same for every CTA of the cluster: nothing visible
         if (rank == 0)
             for (int i = tid; i < k; i += kThreads) out[i] = -1;
@@ -713,18 +755,22 @@ int smem_bytes() { return (int)sizeof(ClSmem) + 1024; }
 DeviceOnce g_attr;
 bool g_nonportable[kMaxDevices];
 
-// Shared-memory size and (where allowed) 16-CTA clusters, once per device.
+// Shared-memory size and (where allowed) 16-CTA clusters of both modes, once per device.
 bool set_attributes() {
     return g_attr.run([] {
         cudaError_t e =
-            cudaFuncSetAttribute(index_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
+            cudaFuncSetAttribute(index_cluster_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(index_cluster_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
         if (e != cudaSuccess) {
             (void)cudaGetLastError();
             return e;
         }
         const int d = current_device();
         g_nonportable[d] =
-            cudaFuncSetAttribute(index_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+            cudaFuncSetAttribute(index_cluster_kernel<0>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                cudaSuccess &&
+            cudaFuncSetAttribute(index_cluster_kernel<1>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
         if (!g_nonportable[d]) (void)cudaGetLastError();
         return cudaSuccess;
     }) == cudaSuccess;
@@ -740,7 +786,8 @@ struct ClusterOcc {
 };
 DeviceValue<ClusterOcc> g_occ;
 
-// Clusters of C CTAs that can be resident at once on the current device (0 if refused).
+// Clusters of C CTAs that can be resident at once on the current device (0 if refused);
+// both modes have the same block and shared-memory size and one CTA per SM.
 int max_active_clusters(int C) {
     const ClusterOcc occ = g_occ.get(
         [] {
@@ -757,7 +804,7 @@ int max_active_clusters(int C) {
                 attr[0].val.clusterDim.z = 1;
                 cfg.attrs = attr;
                 cfg.numAttrs = 1;
-                if (cudaOccupancyMaxActiveClusters(&o.n[c], index_cluster_kernel, &cfg) != cudaSuccess) {
+                if (cudaOccupancyMaxActiveClusters(&o.n[c], index_cluster_kernel<0>, &cfg) != cudaSuccess) {
                     (void)cudaGetLastError();
                     o.n[c] = 0;
                 }
@@ -770,22 +817,34 @@ int max_active_clusters(int C) {
 
 }  // namespace
 
-int index_cluster_size(const SelectParams& p) {
+namespace {
+// Largest cluster whose CTAs each hold at most kMaxTiles tiles of `items` items per query.
+int cluster_size_for(const SelectParams& p, int64_t items) {
     const int bq = p.B * p.Q;
     if (bq <= 0 || !set_attributes()) return 0;
     const int sms = device_sm_count();
     for (int C = nonportable() ? 16 : 8; C >= 1; C >>= 1) {
         if ((int64_t)bq * C > sms) continue;
-        const int64_t chunk = ((p.cap + C - 1) / C + kTile - 1) / kTile * kTile;
+        const int64_t chunk = ((items + C - 1) / C + kTile - 1) / kTile * kTile;
         if (chunk > (int64_t)kMaxTiles * kTile) return 0;   // a smaller cluster only lengthens the chunk
         if (max_active_clusters(C) >= bq) return C;
     }
     return 0;
 }
+}  // namespace
+
+int index_cluster_size(const SelectParams& p) { return cluster_size_for(p, p.cap); }
 
 cudaError_t launch_index_cluster(SelectParams& p, int C, cudaStream_t st) {
     if (!set_attributes()) return cudaErrorInvalidValue;
-    return launch_ex(index_cluster_kernel, dim3(C, p.B * p.Q), dim3(kThreads), smem_bytes(), st, C, p);
+    return launch_ex(index_cluster_kernel<0>, dim3(C, p.B * p.Q), dim3(kThreads), smem_bytes(), st, C, p);
+}
+
+int pool_build_cluster_size(const SelectParams& p) { return cluster_size_for(p, p.nb_cap); }
+
+cudaError_t launch_pool_build_cluster(SelectParams& p, int C, cudaStream_t st) {
+    if (!set_attributes()) return cudaErrorInvalidValue;
+    return launch_ex(index_cluster_kernel<1>, dim3(C, p.B * p.Q), dim3(kThreads), smem_bytes(), st, C, p);
 }
 
 }  // namespace csa2

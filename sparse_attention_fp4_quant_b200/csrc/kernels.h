@@ -82,9 +82,12 @@ cudaError_t launch_index_mq(SelectParams& p, void* mq_ws, cudaStream_t st);
 cudaError_t launch_select(int op, SelectParams& p, int S, cudaStream_t st);
 bool index_tc_supported(const SelectParams& p);
 cudaError_t launch_index_tc(int op, SelectParams& p, int S, cudaStream_t st);
-// One cluster of C CTAs per query (index Top-K only); 0 = the shape does not fit.
+// One cluster of C CTAs per query (index Top-K, and the pool build over the block
+// maxima); 0 = the shape does not fit.
 int index_cluster_size(const SelectParams& p);
 cudaError_t launch_index_cluster(SelectParams& p, int C, cudaStream_t st);
+int pool_build_cluster_size(const SelectParams& p);
+cudaError_t launch_pool_build_cluster(SelectParams& p, int C, cudaStream_t st);
 
 // NVFP4 quantisation and the indexer-K projection.
 cudaError_t launch_quant(const void* x, int64_t rows, int ch, uint8_t* codes, uint8_t* scales,
