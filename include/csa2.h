@@ -325,7 +325,10 @@ CSA2_API csa2_status csa2_device_status(void* ws, int32_t B, int32_t Q, int32_t 
  * entries and a fresh Top-K (and, if pool != NULL, builds the pool from this
  * layer's block maxima); REINDEX re-scores the borrowed KV inside the pool with
  * its own indexer Q; REUSE borrows the indices as well.  Every mode then runs
- * sparse attention with the layer's own Q and SWA KV.
+ * sparse attention with the layer's own Q and SWA KV.  A REINDEX layer's pool
+ * must be one csa2_pool_build wrote (a FULL layer of this call with pool !=
+ * NULL): its valid block ids ascending, which lets the search order and break
+ * ties by pool slot; csa2_pool_topk takes a pool in any order.
  */
 typedef enum { CSA2_MODE_FULL = 0, CSA2_MODE_REINDEX = 1, CSA2_MODE_REUSE = 2 } csa2_mode;
 

@@ -189,9 +189,13 @@ csa2_status csa2_pool_build(const float* blockmax, const csa2_kv* kv, const int3
     return cuda_status(launch_select(CSA2_OP_POOL_BUILD, p, S, (cudaStream_t)stream));
 }
 
-csa2_status csa2_pool_topk(const uint8_t* q, const uint8_t* q_sc, const float* w, const csa2_kv* kv,
-                           const int32_t* pool, int32_t P, const int32_t* q_pos, int32_t B, int32_t Q, int32_t k,
-                           int32_t* idx_out, void* ws, size_t ws_bytes, void* stream) {
+namespace {
+// The pool Top-K; `ascending`: the pool lists its valid blocks in ascending id order (as
+// csa2_pool_build writes it), which the cluster select needs (it orders and breaks ties by
+// pool slot); any other pool takes the per-share select, which sorts by position.
+csa2_status pool_topk(const uint8_t* q, const uint8_t* q_sc, const float* w, const csa2_kv* kv, const int32_t* pool,
+                      int32_t P, const int32_t* q_pos, int32_t B, int32_t Q, int32_t k, int32_t* idx_out, void* ws,
+                      size_t ws_bytes, void* stream, bool ascending) {
     if (B < 1 || Q < 1 || (int64_t)B * Q > 65535 || k < 1 || k > CSA2_MAX_K || P < 1 || P > 65536) return CSA2_ERR_INVALID_ARG;
     if (!q || !q_sc || !w || !pool || !q_pos || !idx_out || !kv_index_ok(kv) || !aligned16(q))
         return CSA2_ERR_INVALID_ARG;
@@ -206,7 +210,16 @@ csa2_status csa2_pool_topk(const uint8_t* q, const uint8_t* q_sc, const float* w
     p.out = idx_out;
     int S = select_splits(CSA2_OP_POOL_TOPK, B, Q, kv->cap, k, P);
     select_carve_ws(p, S, ws, B, Q, k);
+    const int C = ascending ? pool_topk_cluster_size(p) : 0;   // decode-sized query counts: the cluster select
+    if (C > 0) return cuda_status(launch_pool_topk_cluster(p, C, (cudaStream_t)stream));
     return cuda_status(launch_select(CSA2_OP_POOL_TOPK, p, S, (cudaStream_t)stream));
+}
+}  // namespace
+
+csa2_status csa2_pool_topk(const uint8_t* q, const uint8_t* q_sc, const float* w, const csa2_kv* kv,
+                           const int32_t* pool, int32_t P, const int32_t* q_pos, int32_t B, int32_t Q, int32_t k,
+                           int32_t* idx_out, void* ws, size_t ws_bytes, void* stream) {
+    return pool_topk(q, q_sc, w, kv, pool, P, q_pos, B, Q, k, idx_out, ws, ws_bytes, stream, false);
 }
 
 csa2_status csa2_sparse_attn(const void* q, const csa2_kv* kv, const int32_t* idx, int32_t k, const uint8_t* swa,
@@ -273,8 +286,8 @@ csa2_status csa2_layer_step(const csa2_layer_args* a, void* stream) {
             if (st != CSA2_OK) return st;
         }
     } else if (a->mode == CSA2_MODE_REINDEX) {
-        st = csa2_pool_topk(a->iq, a->iq_sc, a->w, kv, a->pool, a->pool_blocks, a->q_pos, a->B, a->Q, a->k, a->idx,
-                            a->ws, a->ws_bytes, stream);
+        st = pool_topk(a->iq, a->iq_sc, a->w, kv, a->pool, a->pool_blocks, a->q_pos, a->B, a->Q, a->k, a->idx,
+                       a->ws, a->ws_bytes, stream, true);
         if (st != CSA2_OK) return st;
     }
     return csa2_sparse_attn(a->q, kv, a->idx, a->k, a->swa, a->swa_sc, a->swa_pos0, a->T, a->window,

@@ -265,7 +265,9 @@ __device__ __forceinline__ void sweep_cols(uint32_t tbase, int warp, int ntiles,
 }
 
 // MODE 0: index + Top-K (keys = the fixed-order scores of the visible entries);
-// MODE 1: pool build (keys = the block maxima of the visible blocks, items = block ids).
+// MODE 1: pool build (keys = the block maxima of the visible blocks, items = block ids);
+// MODE 2: pool Top-K (items = the pool's slots x 8 positions, in ascending position order
+//         since the pool lists its blocks ascending; keys = the scores of the visible ones).
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     index_cluster_kernel(SelectParams p) {
@@ -281,7 +283,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nvis = n_visible(p.q_pos[bq], p.n_entries[b], p.m, p.cap);
     const int64_t row_base = (int64_t)b * p.cap;
     // the items: visible entries, or visible blocks of 8 entries (at most nb_cap)
-    const int nitems = MODE == 0 ? nvis : (int)min((int64_t)((nvis + kBlk - 1) / kBlk), p.nb_cap);
+    const int nitems = MODE == 0 ? nvis
+                       : MODE == 1 ? (int)min((int64_t)((nvis + kBlk - 1) / kBlk), p.nb_cap)
+                                   : p.P * kBlk;
+    const int32_t* pool = MODE == 2 ? p.pool + (int64_t)bq * p.P : nullptr;
     // this CTA's items [lo, hi); the host keeps the chunk within kMaxTiles tiles
     const int chunk = ((nitems + (int)C - 1) / (int)C + kTile - 1) / kTile * kTile;
     const int lo = min(nitems, (int)rank * chunk), hi = min(nitems, lo + chunk);
@@ -303,7 +308,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) init_barriers(s.pipe, kEpiN);
         __syncwarp();
         asm volatile("bar.arrive 1, %0;" ::"n"(kThreads) : "memory");
-        producer_dense(s.pipe, p.ik, p.ik_sc, row_base, lo, ntiles, nstages, status, lane);
+        if constexpr (MODE == 2)
+            producer_pool(s.pipe, p.ik, p.ik_sc, row_base, lo / kBlk, hi / kBlk, ntiles, nstages, pool, nvis, status, lane);
+        else
+            producer_dense(s.pipe, p.ik, p.ik_sc, row_base, lo, ntiles, nstages, status, lane);
     } else {
         if (warp == 1) setup_query(s.pipe, p.q + (int64_t)bq * 128, p.q_sc + (int64_t)bq * 16, lane, kTmemCols);
         for (int i = tid - 32; i < kNB1; i += kThreads - 32) s.hist1[i] = 0;
@@ -355,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
         const uint64_t w01 = f2pack(__ldg(p.w + (int64_t)bq * 4 + 0), __ldg(p.w + (int64_t)bq * 4 + 1));
         const uint64_t w23 = f2pack(__ldg(p.w + (int64_t)bq * 4 + 2), __ldg(p.w + (int64_t)bq * 4 + 3));
-        float* bm = p.blockmax ? p.blockmax + (int64_t)bq * p.nb_cap : nullptr;
+        float* bm = (MODE == 0 && p.blockmax) ? p.blockmax + (int64_t)bq * p.nb_cap : nullptr;
         bool dead = false;   // this warp stopped after a failed wait (or another role's)
         for (int t = 0; t < nstages; ++t) {
             const int a = t % kAcc;
@@ -388,7 +396,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < kTPG; ++j) {
                     const int g = g0 + j;
-                    const bool valid = g < ntiles && lo + g * kTile + eo < hi;
+                    bool valid = g < ntiles && lo + g * kTile + eo < hi;
+                    if (MODE == 2 && valid) {   // slot (item / 8) of the pool, position blk 8 + item % 8
+                        const int item = lo + g * kTile + eo;
+                        const int blk = __ldg(pool + item / kBlk);
+                        valid = blk >= 0 && (int64_t)blk * kBlk + (item % kBlk) < nvis;
+                    }
                     const float score = valid ? score_of(v[j], key_scales(skw[j]), w01, w23) : -INFINITY;
                     key[j] = valid ? score_key(score) : 0u;
                     if (valid) atomicAdd(&s.hist1[key[j] >> 21], 1u);
@@ -419,8 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     cl::wait_acquire();
 
     // ---------------------------------------------------------------- select
-    const uint32_t K1 = (uint32_t)min(k, nitems);
-    if (K1 == 0) {   // the same for every CTA of the cluster: nothing visible
+    uint32_t K1 = (uint32_t)min(k, nitems);   // the pool mode takes its count of valid items below
+    if (MODE != 2 && K1 == 0) {   // the same for every CTA of the cluster: nothing visible
         if (rank == 0)
             for (int i = tid; i < k; i += kThreads) out[i] = -1;
         if (warp == 1) tc::tmem_dealloc(tbase, kTmemCols);
@@ -446,6 +459,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     cl::sync();                                   // every CTA's hist1 is complete
+    if constexpr (MODE == 2) {   // the cluster's valid items: the sum of every rank's coarse bins
+        if (warp == 0) {
+            uint32_t t = 0;
+            for (uint32_t r = 0; r < C; ++r) t += s.coarse[r][2 * lane] + s.coarse[r][2 * lane + 1];
+            t = __reduce_add_sync(0xFFFFFFFFu, t);
+            if (lane == 0) s.res[0] = t;
+        }
+        __syncthreads();
+        K1 = min((uint32_t)k, s.res[0]);
+        __syncthreads();
+        if (K1 == 0) {   // the same for every CTA of the cluster (the same totals)
+            if (rank == 0)
+                for (int i = tid; i < k; i += kThreads) out[i] = -1;
+            if (warp == 1) tc::tmem_dealloc(tbase, kTmemCols);
+            return;
+        }
+    }
     if (warp == 0) find_top_bin(s, C, K1, lane);
     __syncthreads();
     const uint32_t d1 = s.res[0];
@@ -740,7 +770,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             while (m != 0u) {
                 const int bit = __ffs(m) - 1;
                 m &= m - 1u;
-                if (o < (uint32_t)k) out[o] = lo + 32 * (4 * tid + j) + bit;
+                if (o < (uint32_t)k) {
+                    const int item = lo + 32 * (4 * tid + j) + bit;
+                    out[o] = MODE == 2 ? __ldg(pool + item / kBlk) * kBlk + item % kBlk : item;
+                }
                 ++o;
             }
         }
@@ -762,6 +795,8 @@ bool set_attributes() {
             cudaFuncSetAttribute(index_cluster_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(index_cluster_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(index_cluster_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
         if (e != cudaSuccess) {
             (void)cudaGetLastError();
             return e;
@@ -770,7 +805,9 @@ bool set_attributes() {
         g_nonportable[d] =
             cudaFuncSetAttribute(index_cluster_kernel<0>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
                 cudaSuccess &&
-            cudaFuncSetAttribute(index_cluster_kernel<1>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+            cudaFuncSetAttribute(index_cluster_kernel<1>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                cudaSuccess &&
+            cudaFuncSetAttribute(index_cluster_kernel<2>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
         if (!g_nonportable[d]) (void)cudaGetLastError();
         return cudaSuccess;
     }) == cudaSuccess;
@@ -841,6 +878,13 @@ cudaError_t launch_index_cluster(SelectParams& p, int C, cudaStream_t st) {
 }
 
 int pool_build_cluster_size(const SelectParams& p) { return cluster_size_for(p, p.nb_cap); }
+
+int pool_topk_cluster_size(const SelectParams& p) { return cluster_size_for(p, (int64_t)p.P * kBlk); }
+
+cudaError_t launch_pool_topk_cluster(SelectParams& p, int C, cudaStream_t st) {
+    if (!set_attributes()) return cudaErrorInvalidValue;
+    return launch_ex(index_cluster_kernel<2>, dim3(C, p.B * p.Q), dim3(kThreads), smem_bytes(), st, C, p);
+}
 
 cudaError_t launch_pool_build_cluster(SelectParams& p, int C, cudaStream_t st) {
     if (!set_attributes()) return cudaErrorInvalidValue;

@@ -88,6 +88,8 @@ int index_cluster_size(const SelectParams& p);
 cudaError_t launch_index_cluster(SelectParams& p, int C, cudaStream_t st);
 int pool_build_cluster_size(const SelectParams& p);
 cudaError_t launch_pool_build_cluster(SelectParams& p, int C, cudaStream_t st);
+int pool_topk_cluster_size(const SelectParams& p);
+cudaError_t launch_pool_topk_cluster(SelectParams& p, int C, cudaStream_t st);
 
 // NVFP4 quantisation and the indexer-K projection.
 cudaError_t launch_quant(const void* x, int64_t rows, int ch, uint8_t* codes, uint8_t* scales,

@@ -345,6 +345,37 @@ def test_pool_build_and_pool_topk(csa):
             assert np.array_equal(np_(got), ref)
 
 
+def test_pool_topk_through_layer_step(csa):
+    """The Reindex layer of csa2_layer_step searches a pool csa2_pool_build wrote (block ids
+    ascending) with the cluster select: indices equal the oracle's, also for a query whose
+    weights are all zero (every score +0, so the lowest positions win every tie)."""
+    B, Q, cap, T = 4, 1, 30080, 128
+    n_entries = [30000, 17001, 29000, 25000]
+    q_pos = [[29999], [17000], [28999], [24000]]
+    grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(33, B, Q, cap, n_entries, 1, q_pos, 512)
+    _, bm = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, 512, blockmax=True)
+    _, rbm = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, 1, np.array(q_pos, np.int32), 512,
+                               blockmax=True)
+    pos0 = [n - T for n in n_entries]
+    swa, swa_sc = swa_for(34, B, T, pos0)
+    p0 = torch.tensor(pos0, dtype=torch.int32, device="cuda")
+    q = synth.attn_q(35, B, Q, "cuda")
+    for P in (2048, 300):
+        pool = csa.csa2_pool_build(bm, grp.kv, qp, P)
+        rpool = oracle.pool_build(rbm, grp.n_entries, 1, np.array(q_pos, np.int32), P)
+        assert np.array_equal(np_(pool), rpool)
+        for zero_w in (False, True):
+            riq, riqs, rw, roiq, roiqs, row_ = index_query(36 + P, B, Q)
+            if zero_w:
+                rw.zero_()
+                row_ = np.zeros_like(row_)
+            idx = torch.full((B, Q, 512), -7, dtype=torch.int32, device="cuda")
+            csa.csa2_layer_step("reindex", grp.kv, qp, q, swa, swa_sc, p0, idx, 512, riq, riqs, rw, pool=pool)
+            ref = oracle.pool_topk(roiq, roiqs, row_, o["ik"], o["iks"], grp.n_entries, 1, rpool,
+                                   np.array(q_pos, np.int32), 512)
+            assert np.array_equal(np_(idx), ref), (P, zero_w)
+
+
 # ---------------------------------------------------------------- attention
 def _attn_case(csa, seed, B, Q, cap, n_entries, k, T, window, q_pos, pos0, replay, idx_np):
     grp = Group(seed, B, cap, n_entries)
