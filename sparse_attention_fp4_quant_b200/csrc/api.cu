@@ -121,11 +121,13 @@ size_t csa2_workspace_bytes(csa2_op op, int32_t B, int32_t Q, int64_t cap, int32
     if (B < 1 || Q < 1) return 0;
     switch (op) {
         case CSA2_OP_INDEX_TOPK:
+            return ((select_ws_bytes((int)op, B, Q, cap, k, P) + 255) & ~(size_t)255) + cluster_keys_bytes(B, Q, cap);
         case CSA2_OP_POOL_BUILD:
         case CSA2_OP_POOL_TOPK: return select_ws_bytes((int)op, B, Q, cap, k, P);
         case CSA2_OP_SPARSE_ATTN: return attn_ws_bytes(B, Q, k, CSA2_MAX_WINDOW);
         case CSA2_OP_LAYER: {
-            size_t a = select_ws_bytes(CSA2_OP_INDEX_TOPK, B, Q, cap, k, P);
+            size_t a = ((select_ws_bytes(CSA2_OP_INDEX_TOPK, B, Q, cap, k, P) + 255) & ~(size_t)255) +
+                       cluster_keys_bytes(B, Q, cap);
             size_t b = select_ws_bytes(CSA2_OP_POOL_BUILD, B, Q, cap, P > 0 ? P : 1, P);
             size_t c = select_ws_bytes(CSA2_OP_POOL_TOPK, B, Q, cap, k, P);
             size_t d = attn_ws_bytes(B, Q, k, CSA2_MAX_WINDOW);
@@ -171,6 +173,12 @@ csa2_status csa2_index_topk(const uint8_t* q, const uint8_t* q_sc, const float* 
     p.test_starve = test_starve_copies();
     int S = select_splits(CSA2_OP_INDEX_TOPK, B, Q, kv->cap, k, 0);
     select_carve_ws(p, S, ws, B, Q, k);
+    // the cluster index keeps its keys in the workspace when they outgrow TMEM and the
+    // workspace has room for them (csa2_workspace_bytes counts it; the minimum does not)
+    const size_t need = select_ws_bytes(CSA2_OP_INDEX_TOPK, B, Q, kv->cap, k, 0);
+    const size_t kb = cluster_keys_bytes(B, Q, kv->cap);
+    const size_t off = (need + 255) & ~(size_t)255;
+    if (kb > 0 && ws_bytes >= off + kb) p.keys = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + off);
     return cuda_status(launch_select(CSA2_OP_INDEX_TOPK, p, S, (cudaStream_t)stream));
 }
 

@@ -196,8 +196,9 @@ cudaError_t launch_select(int op, SelectParams& p, int S, cudaStream_t st) {
     if ((op == CSA2_OP_INDEX_TOPK || op == CSA2_OP_POOL_TOPK) && index_tc_supported(p)) {
         if (op == CSA2_OP_INDEX_TOPK && p.mq_ws) return launch_index_mq(p, p.mq_ws, st);
         if (op == CSA2_OP_INDEX_TOPK) {
-            const int C = index_cluster_size(p);
-            if (C > 0) return launch_index_cluster(p, C, st);
+            bool keys_in_ws = false;
+            const int C = index_cluster_size(p, &keys_in_ws);
+            if (C > 0) return launch_index_cluster(p, C, keys_in_ws, st);
         }
         return launch_index_tc(op, p, S, st);
     }

@@ -39,10 +39,12 @@ constexpr int kEpiWarps = kEpiN / 32;
 constexpr int kSwW = kThreads / 32;        // warps that sweep the stored keys: four per TMEM lane quarter
 constexpr int kTPG = kTPS / 2;             // tiles of a stage per epilogue warp group
 constexpr int kRing = 8;                   // shared-memory stages in flight
-constexpr int kMaxTiles = 256;             // 32,768 entries per CTA
+constexpr int kMaxTiles = 256;             // 32,768 entries per CTA with the keys in TMEM
+constexpr int kMaxTilesG = 512;            // 65,536 entries per CTA with the keys in the workspace
 constexpr uint32_t kColKeys = kPipeCols;   // key of tile g, row m: TMEM lane m, column kColKeys + g
 constexpr uint32_t kTmemCols = kPipeCols + kMaxTiles;
-constexpr int kWords = kMaxTiles * kTile / 32;          // bitmap words over the CTA's entries
+constexpr int kWords = kMaxTilesG * kTile / 32;         // bitmap words over the CTA's entries
+constexpr int kWPT = kWords / 256;                      // bitmap words per scanning thread
 constexpr int kNB1 = 2048, kNB2 = 2048, kNB3 = 1024;   // radix digits: bits 31..21, 20..10, 9..0
 constexpr int kSel = 256;                  // threads of the scans (warps 0-7)
 constexpr int kCandPerWarp = 128;          // candidates (keys of the threshold's top bin) a sweeping warp lists
@@ -54,6 +56,7 @@ using ClPipe = Pipe<kRing>;
 static_assert((kNB2 + kNB3 + 2 * kWords) * 4 + (2 * kCandCap + kGatherCap) * 8 <= (int)sizeof(ClPipe::A),
               "select scratch fits the ring");
 static_assert(kTmemCols == 512, "TMEM");
+static_assert(kWPT * 256 == kWords && kSel == 256, "bitmap words per scanning thread");
 
 struct ClSmem {
     ClPipe pipe;                            // its A ring holds hist2, hist3 and two bitmaps after scoring
@@ -264,11 +267,29 @@ __device__ __forceinline__ void sweep_cols(uint32_t tbase, int warp, int ntiles,
     }
 }
 
+// The same visit when the keys sit in the workspace (key of CTA-local entry l at keys[l]):
+// columns [128 h, 128 h + 128) for h = warp / 4, each lane's 32 keys of a chunk by 32
+// coalesced loads (the keys were written moments before and are in L2).
+template <class F>
+__device__ __forceinline__ void sweep_cols_g(const uint32_t* keys, int warp, int ntiles, F&& f) {
+    static_assert(kSwW == 16 && kMaxTilesG == 4 * 128, "four warps of 128 columns per lane quarter");
+    const int quarter = warp & 3, part = warp >> 2, lane = threadIdx.x & 31;
+    for (int c0 = part * 128; c0 < min(ntiles, part * 128 + 128); c0 += 32) {
+        uint32_t v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            v[j] = c0 + j < ntiles ? __ldcg(keys + 128 * (c0 + j) + 32 * quarter + lane) : 0u;
+        f(v, c0, quarter);
+    }
+}
+
 // MODE 0: index + Top-K (keys = the fixed-order scores of the visible entries);
 // MODE 1: pool build (keys = the block maxima of the visible blocks, items = block ids);
 // MODE 2: pool Top-K (items = the pool's slots x 8 positions, in ascending position order
 //         since the pool lists its blocks ascending; keys = the scores of the visible ones).
-template <int MODE>
+// KG: the keys go to the workspace (p.keys, [B Q][cap]) instead of TMEM, for up to
+// kMaxTilesG tiles per CTA (the index of a query with more entries than 16 CTAs hold in TMEM).
+template <int MODE, bool KG = false>
 __global__ void __launch_bounds__(kThreads, 1)
     index_cluster_kernel(SelectParams p) {
     pdl_enter();
@@ -294,6 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nstages = (ntiles + kTPS - 1) / kTPS;
     int32_t* status = p.status;
     int32_t* out = p.out + (int64_t)bq * k;
+    static_assert(!KG || MODE == 0, "workspace keys: the index only");
+    uint32_t* const keys = KG ? p.keys + (int64_t)bq * p.cap + lo : nullptr;   // key of CTA-local entry l at keys[l]
 
     // Warp 0 starts the copies as soon as the barriers exist; the other warps set up
     // the query, TMEM and the histogram meanwhile and meet on named barrier 1 (warp 0
@@ -410,8 +433,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if ((lane & (kBlk - 1)) == 0 && valid) bm[(lo + g * kTile + eo) >> 3] = mx;
                     }
                 }
-                if (g0 + 1 < ntiles) tc::tmem_st_32x32b_x2(tbase + lanes + kColKeys + (uint32_t)g0, key[0], key[1]);
-                else if (g0 < ntiles) tc::tmem_st_32x32b_x1(tbase + lanes + kColKeys + (uint32_t)g0, key[0]);
+                if constexpr (KG) {   // every row of a live column, 128 bytes per warp
+#pragma unroll
+                    for (int j = 0; j < kTPG; ++j)
+                        if (g0 + j < ntiles) __stcg(keys + (g0 + j) * kTile + eo, key[j]);
+                } else if (g0 + 1 < ntiles) {
+                    tc::tmem_st_32x32b_x2(tbase + lanes + kColKeys + (uint32_t)g0, key[0], key[1]);
+                } else if (g0 < ntiles) {
+                    tc::tmem_st_32x32b_x1(tbase + lanes + kColKeys + (uint32_t)g0, key[0]);
+                }
             }
         }
         tc::tmem_st_wait();
@@ -430,6 +460,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tc_fence_after();
     tbase = s.pipe.tmem_base;
     cl::wait_acquire();
+    // a visit of every stored key, from TMEM or (KG) from the workspace
+    auto sweep = [&](auto&& f) {
+        if constexpr (KG) sweep_cols_g(keys, warp, ntiles, f);
+        else sweep_cols(tbase, warp, ntiles, f);
+    };
 
     // ---------------------------------------------------------------- select
     uint32_t K1 = (uint32_t)min(k, nitems);   // the pool mode takes its count of valid items below
@@ -489,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint2* mylist = wlist + warp * kCandPerWarp;
     const uint32_t top = ((d1 + 1u) << 21) - 1u;   // keys above bin d1 are > top (none when d1 = 2047)
     const uint32_t bot = d1 << 21;                 // keys of bin d1: key - bot < 2^21
-    sweep_cols(tbase, warp, ntiles, [&](const uint32_t(&v)[32], int c0, int q) {
+    sweep([&](const uint32_t(&v)[32], int c0, int q) {
         uint32_t ma4[4] = {0u, 0u, 0u, 0u}, mc4[4] = {0u, 0u, 0u, 0u};   // four short chains
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
@@ -640,7 +675,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- a threshold bin too large to gather (many equal or close keys):
         // two more radix passes over the keys in TMEM, each with a cluster-wide find
         uint32_t Rs = R;
-        sweep_cols(tbase, warp, ntiles, [&](const uint32_t(&v)[32], int c0, int) {
+        sweep([&](const uint32_t(&v)[32], int c0, int) {
             uint32_t m = 0;   // bit j: column c0 + j matches (independent compares, then a short loop)
 #pragma unroll
             for (int j = 0; j < 32; ++j) m |= (uint32_t)(c0 + j < ntiles && (v[j] >> 21) == d1) << j;
@@ -654,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         find_bin<kNB2>(s, hist2, 0, C, Rs, tid);
         const uint32_t p2 = (d1 << 11) | s.res[0];
         Rs -= s.res[1];
-        sweep_cols(tbase, warp, ntiles, [&](const uint32_t(&v)[32], int c0, int) {
+        sweep([&](const uint32_t(&v)[32], int c0, int) {
             uint32_t m = 0;
 #pragma unroll
             for (int j = 0; j < 32; ++j) m |= (uint32_t)(c0 + j < ntiles && (v[j] >> 10) == p2) << j;
@@ -671,7 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // keys > T and == T: counted, and marked in position bitmaps (column c of lane l
         // is entry 128 c + 32 q + l: bitmap word 4 c + q, bit l)
         uint32_t gt = 0, eq = 0;
-        sweep_cols(tbase, warp, ntiles, [&](const uint32_t(&v)[32], int c0, int q) {
+        sweep([&](const uint32_t(&v)[32], int c0, int q) {
             uint32_t mg = 0, me = 0;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
@@ -735,22 +770,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     __syncthreads();
-    // take the lowest-positioned `quota` ties: thread t owns bitmap words 4t .. 4t + 3
+    // take the lowest-positioned `quota` ties: thread t owns bitmap words kWPT t .. kWPT t + kWPT - 1
     const uint32_t quota = s.cbase[0];
-    uint32_t tw[4] = {0u, 0u, 0u, 0u}, nt = 0;
+    uint32_t tw[kWPT] = {}, nt = 0;
     if (tid < kSel) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            tw[j] = tiebm[4 * tid + j];
+        for (int j = 0; j < kWPT; ++j) {
+            tw[j] = tiebm[kWPT * tid + j];
             nt += __popc(tw[j]);
         }
     }
     uint32_t total;
     uint32_t tpre = block_scan_excl(s, nt, tid, &total);
-    uint32_t sw[4] = {0u, 0u, 0u, 0u}, ns = 0;
+    uint32_t sw[kWPT] = {}, ns = 0;
     if (tid < kSel) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < kWPT; ++j) {
             uint32_t m = tw[j], keep = 0;
             while (m != 0u && tpre < quota) {
                 const uint32_t low = m & (0u - m);
@@ -758,20 +793,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m ^= low;
                 ++tpre;
             }
-            sw[j] = selbm[4 * tid + j] | keep;
+            sw[j] = selbm[kWPT * tid + j] | keep;
             ns += __popc(sw[j]);
         }
     }
     uint32_t o = s.cbase[1] + block_scan_excl(s, ns, tid, &total);
     if (tid < kSel) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < kWPT; ++j) {
             uint32_t m = sw[j];
             while (m != 0u) {
                 const int bit = __ffs(m) - 1;
                 m &= m - 1u;
                 if (o < (uint32_t)k) {
-                    const int item = lo + 32 * (4 * tid + j) + bit;
+                    const int item = lo + 32 * (kWPT * tid + j) + bit;
                     out[o] = MODE == 2 ? __ldg(pool + item / kBlk) * kBlk + item % kBlk : item;
                 }
                 ++o;
@@ -797,6 +832,9 @@ bool set_attributes() {
             e = cudaFuncSetAttribute(index_cluster_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(index_cluster_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(index_cluster_kernel<0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     smem_bytes());
         if (e != cudaSuccess) {
             (void)cudaGetLastError();
             return e;
@@ -807,7 +845,10 @@ bool set_attributes() {
                 cudaSuccess &&
             cudaFuncSetAttribute(index_cluster_kernel<1>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
                 cudaSuccess &&
-            cudaFuncSetAttribute(index_cluster_kernel<2>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+            cudaFuncSetAttribute(index_cluster_kernel<2>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                cudaSuccess &&
+            cudaFuncSetAttribute(index_cluster_kernel<0, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                cudaSuccess;
         if (!g_nonportable[d]) (void)cudaGetLastError();
         return cudaSuccess;
     }) == cudaSuccess;
@@ -855,26 +896,42 @@ int max_active_clusters(int C) {
 }  // namespace
 
 namespace {
-// Largest cluster whose CTAs each hold at most kMaxTiles tiles of `items` items per query.
-int cluster_size_for(const SelectParams& p, int64_t items) {
+// Largest cluster whose CTAs each hold at most `tiles` tiles of `items` items per query.
+int cluster_size_for(const SelectParams& p, int64_t items, int tiles = kMaxTiles) {
     const int bq = p.B * p.Q;
     if (bq <= 0 || !set_attributes()) return 0;
     const int sms = device_sm_count();
     for (int C = nonportable() ? 16 : 8; C >= 1; C >>= 1) {
         if ((int64_t)bq * C > sms) continue;
         const int64_t chunk = ((items + C - 1) / C + kTile - 1) / kTile * kTile;
-        if (chunk > (int64_t)kMaxTiles * kTile) return 0;   // a smaller cluster only lengthens the chunk
+        if (chunk > (int64_t)tiles * kTile) return 0;   // a smaller cluster only lengthens the chunk
         if (max_active_clusters(C) >= bq) return C;
     }
     return 0;
 }
 }  // namespace
 
-int index_cluster_size(const SelectParams& p) { return cluster_size_for(p, p.cap); }
+int index_cluster_size(const SelectParams& p, bool* keys_in_ws) {
+    if (keys_in_ws) *keys_in_ws = false;
+    const int C = cluster_size_for(p, p.cap);
+    if (C > 0 || !p.keys || !keys_in_ws) return C;
+    const int Cg = cluster_size_for(p, p.cap, kMaxTilesG);   // the keys in the workspace
+    *keys_in_ws = Cg > 0;
+    return Cg;
+}
 
-cudaError_t launch_index_cluster(SelectParams& p, int C, cudaStream_t st) {
+cudaError_t launch_index_cluster(SelectParams& p, int C, bool keys_in_ws, cudaStream_t st) {
     if (!set_attributes()) return cudaErrorInvalidValue;
+    if (keys_in_ws)
+        return launch_ex(index_cluster_kernel<0, true>, dim3(C, p.B * p.Q), dim3(kThreads), smem_bytes(), st, C, p);
     return launch_ex(index_cluster_kernel<0>, dim3(C, p.B * p.Q), dim3(kThreads), smem_bytes(), st, C, p);
+}
+
+size_t cluster_keys_bytes(int B, int Q, int64_t cap) {
+    const int64_t bq = (int64_t)B * Q;
+    if (bq < 1 || bq * 16 > kSplitSMs) return 0;                       // one 16-CTA cluster per query
+    if (cap <= 16ll * kMaxTiles * kTile || cap > 16ll * kMaxTilesG * kTile) return 0;
+    return ((size_t)(bq * cap * 4) + 255) & ~(size_t)255;
 }
 
 int pool_build_cluster_size(const SelectParams& p) { return cluster_size_for(p, p.nb_cap); }

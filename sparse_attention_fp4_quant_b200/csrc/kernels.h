@@ -66,6 +66,7 @@ struct SelectParams {
     int32_t* cand_pos;     // [B*Q][S][k]
     void* mq_ws;           // index Top-K for many queries: key prefixes and histograms (else null)
     int test_starve;       // test hook (csa2_test_starve_copies): the per-share producer issues no copies
+    uint32_t* keys;        // [B Q][cap] order keys of the cluster index when they outgrow TMEM, or null
 };
 
 // The test hook's current setting (read by the index entry points).
@@ -84,8 +85,11 @@ bool index_tc_supported(const SelectParams& p);
 cudaError_t launch_index_tc(int op, SelectParams& p, int S, cudaStream_t st);
 // One cluster of C CTAs per query (index Top-K, and the pool build over the block
 // maxima); 0 = the shape does not fit.
-int index_cluster_size(const SelectParams& p);
-cudaError_t launch_index_cluster(SelectParams& p, int C, cudaStream_t st);
+int index_cluster_size(const SelectParams& p, bool* keys_in_ws = nullptr);
+cudaError_t launch_index_cluster(SelectParams& p, int C, bool keys_in_ws, cudaStream_t st);
+// Workspace bytes for the cluster index's keys (0 when its keys fit TMEM or the shape
+// takes another kernel): B Q cap x 4 for decode-sized query counts above 16 x 32,768 entries.
+size_t cluster_keys_bytes(int B, int Q, int64_t cap);
 int pool_build_cluster_size(const SelectParams& p);
 cudaError_t launch_pool_build_cluster(SelectParams& p, int C, cudaStream_t st);
 int pool_topk_cluster_size(const SelectParams& p);

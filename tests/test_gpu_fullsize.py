@@ -151,6 +151,29 @@ def test_c1_decode_group_b32_131k(csa):
             assert ok, (layer, b, st)
 
 
+def test_index_keys_in_workspace_b2_640k(csa):
+    """B=2 at 655,360 entries: more than 16 CTAs hold in TMEM, so the cluster index keeps its
+    keys in the workspace (csa2_workspace_bytes counts them); both rows equal the oracle's
+    Top-512, and the same call with only the minimum workspace (the per-share select) agrees."""
+    B, n = 2, 655360
+    nv = [n, n - 4321]
+    grp = BigGroup(csa, 125, B, n, nv, keep=(0, 1))
+    iq, iqs, w, oiq, oiqs, ow = index_query(126, B, 1)
+    qp_np = np.array([[nv[0] - 1], [nv[1] - 1]], np.int32)
+    qp = torch.from_numpy(qp_np).cuda()
+    full = csa.csa2_workspace_bytes(csa.OP_INDEX_TOPK, B, 1, n, 512)
+    assert full >= B * n * 4   # the keys' room
+    idx = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, 512,
+                              ws=torch.zeros(full, dtype=torch.uint8, device="cuda"))
+    for b in range(B):
+        ridx = _index_ref(grp, b, oiq, oiqs, ow, qp_np[b], 512)
+        assert np.array_equal(np_(idx)[b], ridx[0]), b
+    small = full - B * n * 4   # the minimum the call accepts
+    idx2 = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, 512,
+                               ws=torch.zeros(max(small, 1), dtype=torch.uint8, device="cuda"))
+    assert np.array_equal(np_(idx2), np_(idx))
+
+
 def test_c2_hierarchical_b8_1m(csa):
     """B=8, 1,048,576 entries: Full (Top-512 + block maxima) -> pool of 2,048 blocks -> Reindex Top-512."""
     B, n = 8, 1 << 20
