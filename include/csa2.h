@@ -297,7 +297,11 @@ CSA2_API csa2_status csa2_sparse_attn(const void* q, const csa2_kv* kv, const in
                              float sm_scale, void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /* Workspace sizes.  `op` selects the call; the other arguments are those of the
- * call (k = Top-K or max_blocks; P = pool size for CSA2_OP_POOL_TOPK, else 0). */
+ * call (k = Top-K or max_blocks; P = pool size for CSA2_OP_POOL_TOPK, else 0).
+ * The sizes returned can exceed the minimum a call accepts: the largest decode
+ * contexts (the index's order keys) and the Reindex layer of csa2_layer_step at
+ * one CTA per query (its pool search's order keys, 4 bytes per pool entry) use
+ * the extra space for a faster kernel, and take a slower one without it. */
 typedef enum {
     CSA2_OP_INDEX_TOPK = 0,
     CSA2_OP_POOL_BUILD = 1,

@@ -130,6 +130,8 @@ size_t csa2_workspace_bytes(csa2_op op, int32_t B, int32_t Q, int64_t cap, int32
                        cluster_keys_bytes(B, Q, cap);
             size_t b = select_ws_bytes(CSA2_OP_POOL_BUILD, B, Q, cap, P > 0 ? P : 1, P);
             size_t c = select_ws_bytes(CSA2_OP_POOL_TOPK, B, Q, cap, k, P);
+            if (P > 0 && select_splits(CSA2_OP_POOL_TOPK, B, Q, cap, k, P) == 1)   // Reindex keeps its keys
+                c = ((c + 255) & ~(size_t)255) + pool_keys_bytes(B, Q, P);
             size_t d = attn_ws_bytes(B, Q, k, CSA2_MAX_WINDOW);
             size_t m = a;
             if (b > m) m = b;
@@ -220,6 +222,10 @@ csa2_status pool_topk(const uint8_t* q, const uint8_t* q_sc, const float* w, con
     select_carve_ws(p, S, ws, B, Q, k);
     const int C = ascending ? pool_topk_cluster_size(p) : 0;   // decode-sized query counts: the cluster select
     if (C > 0) return cuda_status(launch_pool_topk_cluster(p, C, (cudaStream_t)stream));
+    if (ascending && S == 1) {   // one CTA per query: keep the keys when the workspace has room for them
+        const size_t off = (select_ws_bytes(CSA2_OP_POOL_TOPK, B, Q, kv->cap, k, P) + 255) & ~(size_t)255;
+        if (ws_bytes >= off + pool_keys_bytes(B, Q, P)) p.keys = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + off);
+    }
     return cuda_status(launch_select(CSA2_OP_POOL_TOPK, p, S, (cudaStream_t)stream));
 }
 }  // namespace

@@ -68,12 +68,12 @@ template <class P>
 __device__ __forceinline__ bool aborted(const P& s) { return *reinterpret_cast<const volatile int*>(&s.abort_flag) != 0; }
 
 // One thread: barrier init.  `full_arrivals` = arrivals that fill a stage (the
-// expect_tx arrive, plus 32 cp.async arrivals when the scales come by cp.async);
+// producer's expect_tx arrive, or one per lane of producer_pool_async);
 // `epi_arrivals` = arrivals that free an accumulator stage.
 template <class P>
-__device__ __forceinline__ void init_barriers(P& s, uint32_t epi_arrivals) {
+__device__ __forceinline__ void init_barriers(P& s, uint32_t epi_arrivals, uint32_t full_arrivals = 1) {
     for (int i = 0; i < P::kStages; ++i) {
-        tc::mbar_init(&s.full[i], 1);                 // the producer's expect_tx
+        tc::mbar_init(&s.full[i], full_arrivals);
         tc::mbar_init(&s.empty[i], 1 + kEpiWarps);    // MMA commit + each epilogue warp
     }
     for (int i = 0; i < kAcc; ++i) {
@@ -195,6 +195,87 @@ __device__ __forceinline__ void producer_pool(P& s, const uint8_t* ik, const uin
         for (int t = max(0, issued - kStages); t < issued; ++t)
             if (!tc::mbar_wait(&s.full[t % kStages], (uint32_t)(t / kStages) & 1u)) raise_abort(s, status);
     }
+    __syncwarp();
+}
+
+// Warp 0, the same pool slots as producer_pool, copied by the 32 lanes with 16-byte
+// cp.async instead of two bulk copies per block.  Each bulk copy is one request to the
+// copy engine, and at 8 blocks a share of 2,048 slots issue thousands of them; here lane l
+// copies half (l % 2) of the codes of block l / 2 of each tile (8 chunks) and one of the
+// block's two scale chunks.  The copies write through the generic proxy, so a lane waits
+// for its own copies of a stage, fences them to the async proxy (the MMA reads the codes
+// there) and then arrives on the stage's barrier, which expects kPoolLanes arrivals.  The
+// wait trails the issue by kLag stages so that copies of several stages are in flight.
+// The pool slots are read kAhead stages before their copies are issued (a dependent
+// global load per stage would otherwise sit in front of every issue), and each stage's
+// block ids (-1 = no block) go to `stage_blk` ([kStages][kTPS][kPoolPerTile] in shared
+// memory) before the stage's arrivals, for the epilogue to read after its wait.
+constexpr uint32_t kPoolLanes = 32;
+template <class P>
+__device__ __forceinline__ void producer_pool_async(P& s, const uint8_t* ik, const uint8_t* iks, int64_t row_base,
+                                                    int lo, int hi, int ntiles, int nstages, const int32_t* pool,
+                                                    int nvis, int32_t* stage_blk, int32_t* status, int lane) {
+    constexpr int kStages = P::kStages;
+    constexpr int kLag = kStages > 2 ? 2 : 1;   // < kStages: stage t - kStages has arrived before t waits
+    constexpr int kAhead = 2;
+    const int j = lane >> 1, half = lane & 1;
+    int nxt[kAhead + 1][kTPS];
+    auto read_slots = [&](int t, int (&b)[kTPS]) {
+#pragma unroll
+        for (int i = 0; i < kTPS; ++i) {
+            const int g = t * kTPS + i;
+            const int sl = lo + g * kPoolPerTile + j;
+            b[i] = (t < nstages && g < ntiles && sl < hi) ? __ldg(pool + sl) : -1;
+        }
+    };
+#pragma unroll
+    for (int a = 0; a < kAhead; ++a) read_slots(a, nxt[a]);
+    int issued = 0, arrived = 0;
+    for (int t = 0; t < nstages; ++t) {
+        const int slot = t % kStages;
+        const uint32_t ph = (uint32_t)(t / kStages) & 1u;
+        read_slots(t + kAhead, nxt[kAhead]);
+        int cur[kTPS];
+#pragma unroll
+        for (int i = 0; i < kTPS; ++i) {
+            cur[i] = nxt[0][i];
+#pragma unroll
+            for (int a = 0; a < kAhead; ++a) nxt[a][i] = nxt[a + 1][i];
+        }
+        int ok = 1;
+        if (lane == 0) ok = tc::mbar_wait_spin(&s.empty[slot], ph ^ 1u);
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (lane == 0 && !ok) raise_abort(s, status);
+        if (__any_sync(0xFFFFFFFFu, !ok || aborted(s))) break;   // warp-uniform
+#pragma unroll
+        for (int i = 0; i < kTPS; ++i) {
+            int blk = cur[i];
+            if (blk >= 0 && (int64_t)blk * kBlk >= nvis) blk = -1;
+            if (half == 0) stage_blk[(slot * kTPS + i) * kPoolPerTile + j] = blk;
+            if (blk < 0) continue;
+            const int64_t e = row_base + (int64_t)blk * kBlk;
+            const uint32_t dA = tc::smem_u32(s.A[slot][i] + 256 * j + 128 * half);
+            const uint8_t* sA = ik + ik_code_off(e, 0) + 128 * half;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dA + 16u * c), "l"(sA + 16 * c) : "memory");
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(s.SF[slot][i] + 32 * j + 16 * half)),
+                         "l"(iks + ik_scale_off(e) + 16 * half)
+                         : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        ++issued;
+        if (issued - arrived > kLag) {
+            asm volatile("cp.async.wait_group %0;" ::"n"(kLag) : "memory");
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(&s.full[arrived % kStages]);
+            ++arrived;
+        }
+    }
+    // never leave copies in flight, and complete every stage that was issued
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    tc::fence_proxy_async_smem();
+    for (; arrived < issued; ++arrived) tc::mbar_arrive(&s.full[arrived % kStages]);
     __syncwarp();
 }
 

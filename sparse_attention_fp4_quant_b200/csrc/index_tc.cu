@@ -1,11 +1,16 @@
 // index_tc.cu -- FP4 index scoring on the tcgen05 tensor cores (index_pipe.cuh),
-// fused with a streaming exact Top-K (Full layers: csa2_index_topk when the
-// query count is too large for one cluster per query; Reindex layers:
-// csa2_pool_topk).
+// fused with an exact Top-K (Full layers: csa2_index_topk when the query count
+// is too large for one cluster per query; Reindex layers: csa2_pool_topk, and
+// csa2_layer_step's Reindex for many queries).
 //
 // One CTA = one share of one query's candidates.  Warps 0 and 1 run the
-// scoring pipeline; warps 2-9 finish the scores and run the Top-K filter
-// (named barrier 1).  The last CTA of a query merges the shares.
+// scoring pipeline; warps 2-9 finish the scores and select (named barrier 1).
+// Modes 0 and 1 stream the scores through a threshold filter into a buffer
+// that an exact radix select compacts; the last CTA of a query merges the
+// shares.  Mode 2 (an ascending pool, one CTA per query) keeps every order key
+// in the workspace and counts its top 11 bits while scoring, then offers only
+// the entries at or above the bin that holds the k-th key to the exact Top-K:
+// no per-stage barrier, and typically no compaction before the last.
 #include "index_pipe.cuh"
 #include "topk.cuh"
 
@@ -19,13 +24,28 @@ constexpr int kThreads = kEpiT0 + kEpiN;
 constexpr int kTPG = kTPS / 2;   // tiles of a stage per epilogue warp group
 
 constexpr int kRing = 4;   // shared-memory stages in flight
+constexpr int kHistBits = 11, kHistBins = 1 << kHistBits;   // mode 2: bins of the keys' top bits
 
 template <int CAP>
 struct TcSmem {
     Pipe<kRing> pipe;
+    int32_t stage_blk[kRing][kTPS][kPoolPerTile];   // pool modes: each stage's block ids (-1 = none)
     int last;
-    typename TopK<kEpiN, CAP, 1, kEpiT0>::Smem topk;
+    uint32_t sel_bin, sel_count;    // mode 2: the bin of the k-th key, entries in it or above
+    uint32_t warp_sum[kEpiN / 32];  // mode 2: per-warp histogram sums
+    union {
+        typename TopK<kEpiN, CAP, 1, kEpiT0>::Smem topk;
+        uint32_t hist[kHistBins];   // mode 2, while scoring (the Top-K takes the space afterwards)
+    };
 };
+static_assert(sizeof(uint32_t) * kHistBins <= sizeof(typename TopK<kEpiN, 2048, 1, kEpiT0>::Smem), "histogram fits");
+
+// One shared-memory add per entry (bin < 0: none).  Lanes that hit the same bin are
+// serialised by the hardware; grouping them first (match.any) cost more than it saved
+// on pool scores.
+__device__ __forceinline__ void hist_add(uint32_t hist_base, int bin) {
+    if (bin >= 0) shm::red_add(hist_base + 4u * (uint32_t)bin, 1u);
+}
 
 // OR of `v` over the epilogue warps, through named barrier 1 (every epilogue
 // thread gets the same answer, so they all leave or all stay).
@@ -39,7 +59,87 @@ __device__ __forceinline__ bool epilogue_any(bool v) {
     return r != 0;
 }
 
-template <int MODE, int CAP>  // MODE 0 = dense range (index Top-K), 1 = pool blocks (pool Top-K)
+// Epilogue warps, mode 2, after scoring: the bin d that holds the k-th largest key (bins
+// scanned from the top; every key when there are at most k), then one read of the keys
+// offers each entry in bin d or above to the exact Top-K, the entry index standing for the
+// position (the pool is ascending, so the two orders agree).  When those entries fit the
+// buffer nothing is compacted before the final select; otherwise the buffer makes room as
+// it fills, which is exact too, only slower.
+template <int CAP>
+__device__ __forceinline__ void pool_select(TcSmem<CAP>& s, TopK<kEpiN, CAP, 1, kEpiT0>& tk, const uint32_t* qkeys,
+                                            int n_items, int k, int lane, int warp) {
+    using TKE = TopK<kEpiN, CAP, 1, kEpiT0>;
+    const int et = (int)threadIdx.x - kEpiT0, ew = warp - kEpiT0 / 32;
+    constexpr int kPer = kHistBins / kEpiN;   // bins per thread, highest first
+    uint32_t c[kPer], tot = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        c[j] = s.hist[kHistBins - 1 - (kPer * et + j)];
+        tot += c[j];
+    }
+    uint32_t incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) s.warp_sum[ew] = incl;
+    TKE::sync();
+    uint32_t before = incl - tot, total = 0;
+#pragma unroll
+    for (int w = 0; w < kEpiN / 32; ++w) {
+        const uint32_t v = s.warp_sum[w];
+        if (w < ew) before += v;
+        total += v;
+    }
+    const uint32_t kk = (uint32_t)k;
+    if (total <= kk) {
+        if (et == 0) {
+            s.sel_bin = 0;
+            s.sel_count = total;
+        }
+    } else if (before < kk && kk <= before + tot) {
+        uint32_t run = before;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            if (run + c[j] >= kk) {
+                s.sel_bin = (uint32_t)(kHistBins - 1 - (kPer * et + j));
+                s.sel_count = run + c[j];
+                break;
+            }
+            run += c[j];
+        }
+    }
+    TKE::sync();   // after it no thread reads the histogram, whose space the Top-K now takes
+    const uint32_t d = s.sel_bin;
+    const bool fast = s.sel_count <= (uint32_t)CAP;
+    tk.init();
+    constexpr int kBatch = 4;   // rounds of 4 keys a thread whose loads are in flight together
+    for (int base = 0; base < n_items; base += kBatch * 4 * kEpiN) {   // uniform trip count
+        uint4 kv[kBatch];
+#pragma unroll
+        for (int r = 0; r < kBatch; ++r) {
+            const int i0 = base + r * 4 * kEpiN + 4 * et;   // n_items is a multiple of 4
+            kv[r] = i0 < n_items ? __ldcg(reinterpret_cast<const uint4*>(qkeys + i0)) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int r = 0; r < kBatch; ++r) {
+            const int i0 = base + r * 4 * kEpiN + 4 * et;
+            const uint32_t key4[4] = {kv[r].x, kv[r].y, kv[r].z, kv[r].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (!fast) tk.make_room(k, kEpiN);
+                const bool take = key4[q] != 0u && (key4[q] >> (32 - kHistBits)) >= d;
+                tk.offer(take, key4[q], i0 + q);
+            }
+        }
+    }
+    tk.finish(k);
+}
+
+// MODE 0 = dense range (index Top-K), 1 = pool blocks (pool Top-K), 2 = pool blocks of an
+// ascending pool with the keys kept in the workspace (one share per query)
+template <int MODE, int CAP>
 __global__ void __launch_bounds__(kThreads, 2)
     index_tc_kernel(SelectParams p) {
     pdl_enter();
@@ -70,24 +170,34 @@ __global__ void __launch_bounds__(kThreads, 2)
         ntiles = (hi - lo + kPoolPerTile - 1) / kPoolPerTile;
     }
     const int nstages = (ntiles + kTPS - 1) / kTPS;
-    const int32_t* pool = (MODE == 1) ? p.pool + (int64_t)bq * p.P : nullptr;
+    const int32_t* pool = (MODE != 0) ? p.pool + (int64_t)bq * p.P : nullptr;
+    // mode 2: this query's order keys, one per (tile, row): entry index i = slot * 8 + row
+    uint32_t* qkeys = (MODE == 2) ? p.keys + (int64_t)bq * ntiles * kTile : nullptr;
 
-    if (tid == 0) init_barriers(s.pipe, kEpiN);
+    if (tid == 0) init_barriers(s.pipe, kEpiN, MODE == 0 ? 1u : kPoolLanes);
     if (warp == 1) setup_query(s.pipe, p.q + (int64_t)bq * 128, p.q_sc + (int64_t)bq * 16, lane, kPipeCols);
     __syncthreads();
     const uint32_t tbase = s.pipe.tmem_base;
     int32_t* status = p.status;
 
     if (warp == 0) {
-        if (MODE == 0)
+        if constexpr (MODE == 0)
             producer_dense(s.pipe, p.ik, p.ik_sc, row_base, lo, ntiles, nstages, status, lane, p.test_starve != 0);
-        else producer_pool(s.pipe, p.ik, p.ik_sc, row_base, lo, hi, ntiles, nstages, pool, nvis, status, lane);
+        else
+            producer_pool_async(s.pipe, p.ik, p.ik_sc, row_base, lo, hi, ntiles, nstages, pool, nvis, &s.stage_blk[0][0][0],
+                                status, lane);
     } else if (warp == 1) {
         mma_issuer(s.pipe, ntiles, nstages, status, lane);
     } else {
         // ------------------------------------------------------------ epilogue
         TKE tk(s.topk);
-        tk.init();
+        const uint32_t hist_base = tc::smem_u32(&s.hist[0]);
+        if constexpr (MODE == 2) {
+            for (int i = tid - kEpiT0; i < kHistBins; i += kEpiN) shm::st(hist_base + 4u * (uint32_t)i, 0u);
+            TKE::sync();
+        } else {
+            tk.init();
+        }
         const int quarter = warp & 3;             // TMEM lanes this warp may read
         const int group = (warp - 2) >> 2;        // tiles 2*group, 2*group+1 of each stage
         const int row = quarter * 32 + lane;
@@ -116,9 +226,35 @@ __global__ void __launch_bounds__(kThreads, 2)
             const bool landed = ok && __all_sync(0xFFFFFFFFu, stage_landed(s.pipe, t));   // warp-uniform
             if (ok && !landed && lane == 0) raise_abort(s.pipe, status);
             uint32_t skw[kTPG];
+            int sblk[kTPG];   // pool mode: the row's block id (read before the stage is released)
 #pragma unroll
-            for (int j = 0; j < kTPG; ++j) skw[j] = landed ? stage_scales(s.pipe, t % kRing, kTPG * group + j, row) : 0u;
+            for (int j = 0; j < kTPG; ++j) {
+                skw[j] = landed ? stage_scales(s.pipe, t % kRing, kTPG * group + j, row) : 0u;
+                sblk[j] = (MODE != 0 && landed) ? s.stage_blk[t % kRing][kTPG * group + j][row >> 3] : -1;
+            }
             if (landed) release_stage(s.pipe, t, lane);
+            if constexpr (MODE == 2) {
+                if (!landed) {   // warp-uniform; the warps meet again after the loop
+                    stop = true;
+                    break;
+                }
+#pragma unroll
+                for (int j = 0; j < kTPG; ++j) {
+                    const int g = t * kTPS + kTPG * group + j;
+                    if (g >= ntiles) break;   // warp-uniform
+                    int64_t e = -1;
+                    if (sblk[j] >= 0) {
+                        const int64_t ee = (int64_t)sblk[j] * kBlk + (row & 7);
+                        if (ee < nvis) e = ee;
+                    }
+                    const bool valid = e >= 0;
+                    // key 0 marks "no entry": a finite score's key is never 0
+                    const uint32_t key = valid ? score_key(score_of(v[j], key_scales(skw[j]), w01, w23)) : 0u;
+                    __stcg(qkeys + g * kTile + row, key);
+                    hist_add(hist_base, valid ? (int)(key >> (32 - kHistBits)) : -1);
+                }
+                continue;
+            }
             if (epilogue_any(aborted(s.pipe))) {   // also the barrier that orders the previous offers
                 stop = true;
                 break;
@@ -133,13 +269,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                     if (MODE == 0) {
                         const int ee = lo + g * kTile + row;
                         if (ee < hi) e = ee;
-                    } else {
-                        const int sl = lo + g * kPoolPerTile + (row >> 3);
-                        if (sl < hi) {
-                            const int blk = __ldg(pool + sl);
-                            const int64_t ee = (int64_t)blk * kBlk + (row & 7);
-                            if (blk >= 0 && ee < nvis) e = ee;
-                        }
+                    } else if (sblk[j] >= 0) {   // the producer wrote -1 past the share and for unseen blocks
+                        const int64_t ee = (int64_t)sblk[j] * kBlk + (row & 7);
+                        if (ee < nvis) e = ee;
                     }
                 }
                 const bool valid = e >= 0;
@@ -160,7 +292,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int64_t j = j0 + (tid - kEpiT0); j < j1; j += kEpiN) bm[j] = -INFINITY;
             }
         }
-        if (!stop) tk.finish(k);
+        if constexpr (MODE == 2) {
+            stop = epilogue_any(stop || aborted(s.pipe));
+            if (!stop) pool_select<CAP>(s, tk, qkeys, ntiles * kTile, k, lane, warp);
+        } else {
+            if (!stop) tk.finish(k);
+        }
     }
     __syncthreads();
     if (warp == 1) tc::tmem_dealloc(tbase, kPipeCols);
@@ -201,7 +338,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     const int cnt = tk.count();
     tk.sort_positions(cnt);
-    for (int i = et; i < k; i += kEpiN) p.out[(int64_t)bq * k + i] = i < cnt ? tk.pos_at(i) : -1;
+    if constexpr (MODE == 2) {   // entry index -> position (ascending pool: the same order)
+        for (int i = et; i < k; i += kEpiN) {
+            int32_t r = -1;
+            if (i < cnt) {
+                const int32_t it = tk.pos_at(i);
+                r = __ldg(pool + (it >> 3)) * kBlk + (it & 7);
+            }
+            p.out[(int64_t)bq * k + i] = r;
+        }
+    } else {
+        for (int i = et; i < k; i += kEpiN) p.out[(int64_t)bq * k + i] = i < cnt ? tk.pos_at(i) : -1;
+    }
 }
 
 // two CTAs per SM for the usual k (the k > 1536 variant runs one)
@@ -213,6 +361,8 @@ bool index_tc_supported(const SelectParams& p) {
     return (((uintptr_t)p.ik) & 15u) == 0 && (((uintptr_t)p.ik_sc) & 15u) == 0 && p.cap % kTile == 0 &&
            (int64_t)p.B * p.cap < (int64_t(1) << 31);
 }
+
+size_t pool_keys_bytes(int B, int Q, int P) { return (size_t)B * Q * (size_t)((P + kPoolPerTile - 1) / kPoolPerTile) * kTile * 4; }
 
 template <int MODE, int CAP>
 cudaError_t launch_tc(SelectParams& p, int S, cudaStream_t st) {
@@ -226,10 +376,12 @@ cudaError_t launch_tc(SelectParams& p, int S, cudaStream_t st) {
 }
 
 cudaError_t launch_index_tc(int op, SelectParams& p, int S, cudaStream_t st) {
-    const int mode = (op == CSA2_OP_POOL_TOPK) ? 1 : 0;
+    // a pool search with its keys in the workspace (the caller vouches for an ascending pool)
+    const int mode = (op == CSA2_OP_POOL_TOPK) ? ((p.keys && S == 1) ? 2 : 1) : 0;
     // the buffer must hold k survivors plus one stage of offers
-    if (p.k <= 2048 - kTPS * kTile) return mode == 0 ? launch_tc<0, 2048>(p, S, st) : launch_tc<1, 2048>(p, S, st);
-    return mode == 0 ? launch_tc<0, 4096>(p, S, st) : launch_tc<1, 4096>(p, S, st);
+    if (p.k <= 2048 - kTPS * kTile)
+        return mode == 0 ? launch_tc<0, 2048>(p, S, st) : mode == 1 ? launch_tc<1, 2048>(p, S, st) : launch_tc<2, 2048>(p, S, st);
+    return mode == 0 ? launch_tc<0, 4096>(p, S, st) : mode == 1 ? launch_tc<1, 4096>(p, S, st) : launch_tc<2, 4096>(p, S, st);
 }
 
 }  // namespace csa2

@@ -66,7 +66,8 @@ struct SelectParams {
     int32_t* cand_pos;     // [B*Q][S][k]
     void* mq_ws;           // index Top-K for many queries: key prefixes and histograms (else null)
     int test_starve;       // test hook (csa2_test_starve_copies): the per-share producer issues no copies
-    uint32_t* keys;        // [B Q][cap] order keys of the cluster index when they outgrow TMEM, or null
+    uint32_t* keys;        // order keys in the workspace, or null: [B Q][cap] for the cluster index when they
+                           // outgrow TMEM, [B Q][ceil(P / 16) 128] for the search of an ascending pool
 };
 
 // The test hook's current setting (read by the index entry points).
@@ -83,6 +84,9 @@ cudaError_t launch_index_mq(SelectParams& p, void* mq_ws, cudaStream_t st);
 cudaError_t launch_select(int op, SelectParams& p, int S, cudaStream_t st);
 bool index_tc_supported(const SelectParams& p);
 cudaError_t launch_index_tc(int op, SelectParams& p, int S, cudaStream_t st);
+// Workspace bytes for the order keys of a one-share-per-query search of an ascending pool
+// (index_tc mode 2): 4 bytes per slot row, the slots rounded up to whole 128-row tiles.
+size_t pool_keys_bytes(int B, int Q, int P);
 // One cluster of C CTAs per query (index Top-K, and the pool build over the block
 // maxima); 0 = the shape does not fit.
 int index_cluster_size(const SelectParams& p, bool* keys_in_ws = nullptr);

@@ -376,6 +376,40 @@ def test_pool_topk_through_layer_step(csa):
             assert np.array_equal(np_(idx), ref), (P, zero_w)
 
 
+def test_pool_topk_many_queries_layer_step(csa):
+    """Reindex for many queries (one CTA per query, order keys kept in the workspace and a
+    histogram pre-selection): indices equal the oracle's for pools of 2,048 and 300 blocks,
+    queries that see a few blocks only, and all-zero weights (every score +0: one histogram
+    bin holds every entry, so the exact Top-K has to make room as it fills)."""
+    B, Q, cap, T = 2, 80, 30080, 128
+    n_entries = [30000, 22001]
+    q_pos = [[n_entries[b] - 1 - 97 * j for j in range(Q)] for b in range(B)]
+    q_pos[1][-3:] = [5, 700, 4100]
+    grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(41, B, Q, cap, n_entries, 1, q_pos, 512)
+    _, bm = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, 512, blockmax=True)
+    _, rbm = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, 1, np.array(q_pos, np.int32), 512,
+                               blockmax=True)
+    assert np.array_equal(np_(bm), rbm)
+    pos0 = [n - T for n in n_entries]
+    swa, swa_sc = swa_for(42, B, T, pos0)
+    p0 = torch.tensor(pos0, dtype=torch.int32, device="cuda")
+    q = synth.attn_q(43, B, Q, "cuda")
+    for P in (2048, 300):
+        pool = csa.csa2_pool_build(bm, grp.kv, qp, P)
+        rpool = oracle.pool_build(rbm, grp.n_entries, 1, np.array(q_pos, np.int32), P)
+        assert np.array_equal(np_(pool), rpool)
+        for zero_w in (False, True):
+            riq, riqs, rw, roiq, roiqs, row_ = index_query(44 + P, B, Q)
+            if zero_w:
+                rw.zero_()
+                row_ = np.zeros_like(row_)
+            idx = torch.full((B, Q, 512), -7, dtype=torch.int32, device="cuda")
+            csa.csa2_layer_step("reindex", grp.kv, qp, q, swa, swa_sc, p0, idx, 512, riq, riqs, rw, pool=pool)
+            ref = oracle.pool_topk(roiq, roiqs, row_, o["ik"], o["iks"], grp.n_entries, 1, rpool,
+                                   np.array(q_pos, np.int32), 512)
+            assert np.array_equal(np_(idx), ref), (P, zero_w)
+
+
 # ---------------------------------------------------------------- attention
 def _attn_case(csa, seed, B, Q, cap, n_entries, k, T, window, q_pos, pos0, replay, idx_np):
     grp = Group(seed, B, cap, n_entries)
