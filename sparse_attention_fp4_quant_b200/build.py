@@ -7,7 +7,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libcsa2.so")
-SOURCES = ["api.cu", "quant.cu", "index.cu", "index_tc.cu", "index_cluster.cu", "index_mq.cu", "attn.cu", "attn_cluster.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "quant.cu", "index.cu", "index_tc.cu", "index_cluster.cu", "index_mq.cu", "attn.cu", "attn_cluster.cu", "noalloc.cu", "pool_build.cu"]
 HEADERS = ["common.cuh", "topk.cuh", "tc.cuh", "index_pipe.cuh", "cluster.cuh", "attn_common.cuh", "score_cc.cuh", "kernels.h", "host_util.h"]
 
 NVCC_FLAGS = [

@@ -196,6 +196,8 @@ csa2_status csa2_pool_build(const float* blockmax, const csa2_kv* kv, const int3
     select_carve_ws(p, S, ws, B, Q, max_blocks);
     const int C = pool_build_cluster_size(p);   // decode-sized query counts: the cluster radix select
     if (C > 0) return cuda_status(launch_pool_build_cluster(p, C, (cudaStream_t)stream));
+    // one CTA per query fills the GPU: the per-query radix select
+    if (S == 1 && pool_build_radix_ok(p)) return cuda_status(launch_pool_build_radix(p, (cudaStream_t)stream));
     return cuda_status(launch_select(CSA2_OP_POOL_BUILD, p, S, (cudaStream_t)stream));
 }
 

@@ -95,6 +95,10 @@ cudaError_t launch_index_cluster(SelectParams& p, int C, bool keys_in_ws, cudaSt
 // takes another kernel): B Q cap x 4 for decode-sized query counts above 16 x 32,768 entries.
 size_t cluster_keys_bytes(int B, int Q, int64_t cap);
 int pool_build_cluster_size(const SelectParams& p);
+// Pool build for many queries (pool_build.cu): one CTA per query, radix select over
+// its block maxima; ok = the shape fits (at most 131,072 blocks, aligned maxima).
+bool pool_build_radix_ok(const SelectParams& p);
+cudaError_t launch_pool_build_radix(SelectParams& p, cudaStream_t st);
 cudaError_t launch_pool_build_cluster(SelectParams& p, int C, cudaStream_t st);
 int pool_topk_cluster_size(const SelectParams& p);
 cudaError_t launch_pool_topk_cluster(SelectParams& p, int C, cudaStream_t st);

@@ -377,10 +377,12 @@ def test_pool_topk_through_layer_step(csa):
 
 
 def test_pool_topk_many_queries_layer_step(csa):
-    """Reindex for many queries (one CTA per query, order keys kept in the workspace and a
-    histogram pre-selection): indices equal the oracle's for pools of 2,048 and 300 blocks,
+    """Pool build and Reindex for many queries (one CTA per query: the radix select over the
+    block maxima; the pool search with its order keys in the workspace and a histogram
+    pre-selection): pools and indices equal the oracle's for pools of 2,048 and 300 blocks,
     queries that see a few blocks only, and all-zero weights (every score +0: one histogram
-    bin holds every entry, so the exact Top-K has to make room as it fills)."""
+    bin holds every entry, so the exact Top-K has to make room as it fills; for the build,
+    every block maximum ties and the lowest blocks win)."""
     B, Q, cap, T = 2, 80, 30080, 128
     n_entries = [30000, 22001]
     q_pos = [[n_entries[b] - 1 - 97 * j for j in range(Q)] for b in range(B)]
@@ -390,6 +392,14 @@ def test_pool_topk_many_queries_layer_step(csa):
     _, rbm = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, 1, np.array(q_pos, np.int32), 512,
                                blockmax=True)
     assert np.array_equal(np_(bm), rbm)
+    w0 = torch.zeros_like(w)
+    _, bm0 = csa.csa2_index_topk(iq, iqs, w0, grp.kv, qp, 512, blockmax=True)
+    _, rbm0 = oracle.index_topk(oiq, oiqs, np.zeros_like(ow), o["ik"], o["iks"], grp.n_entries, 1,
+                                np.array(q_pos, np.int32), 512, blockmax=True)
+    assert np.array_equal(np_(bm0), rbm0)
+    for P in (2048, 300):
+        pool0 = csa.csa2_pool_build(bm0, grp.kv, qp, P)
+        assert np.array_equal(np_(pool0), oracle.pool_build(rbm0, grp.n_entries, 1, np.array(q_pos, np.int32), P)), P
     pos0 = [n - T for n in n_entries]
     swa, swa_sc = swa_for(42, B, T, pos0)
     p0 = torch.tensor(pos0, dtype=torch.int32, device="cuda")
