@@ -225,9 +225,9 @@ CSA2_API csa2_status csa2_front_end(const void* x, int64_t rows, const float* ro
  *                 blocks with no visible position ([Blog] Fig. 5)
  *   ws, ws_bytes  device workspace of at least csa2_workspace_bytes(CSA2_OP_INDEX_TOPK, ...);
  *                 for more than 148 queries with at least 8 per batch row and
- *                 cap <= 65,536 (a prefill chunk) it also holds every query's
- *                 16-bit key prefixes and 2,048-bin histogram (2 B per query
- *                 and entry + 8 KB per query)
+ *                 cap <= 262,144 (a prefill chunk, a replay) it also holds every
+ *                 query's 16-bit key prefixes and 2,048-bin histogram (2 B per
+ *                 query and entry + 8 KB per query)
  *                 bytes, zero-filled before its first use; every call leaves its
  *                 counters at zero again.  Calls that share a workspace must not
  *                 overlap on the GPU.  The int32 at byte offset

@@ -2,8 +2,9 @@
 // chunks): the indexer keys are scored once for 8 queries at a time, then one
 // CTA per query selects its Top-K.
 //
-// Scoring (mq_score_kernel, one CTA per 8 consecutive queries of a batch
-// row; 16 epilogue warps, two queries each, so that four warps share each SM
+// Scoring (mq_score_kernel, one CTA per 8 consecutive queries of a batch row
+// and share of its entry range (shares when the groups alone leave SMs idle,
+// their histograms added in the workspace); 16 epilogue warps, two queries each, so that four warps share each SM
 // sub-partition and hide each other's latency).  The block-scaled FP4 MMA of index_pipe.cuh with B = 8 block-diagonal
 // query operands side by side (N = 128: column 16 g + 4 h + b holds query g's
 // head h codes of block b only), so every key tile crosses shared memory once
@@ -19,8 +20,10 @@
 // exact keys are recomputed on CUDA cores (score_cc.cuh: the same defined
 // score) and two radix passes over them give the threshold T.  The selection
 // is every key above T plus the lowest-positioned keys equal to T, written in
-// ascending position order.  A threshold bin larger than the list (many equal
-// or close keys) is resolved by passes that re-score the bin's entries.
+// ascending position order.  A threshold bin larger than the list is narrowed by
+// a second read to the sub-bin of the prefix's next 5 bits (counted in the first
+// read) that holds the K-th key; one still too large (many equal or close keys)
+// is resolved by passes that re-score its entries.
 #include "index_pipe.cuh"
 #include "score_cc.cuh"
 
@@ -65,13 +68,19 @@ __global__ void __launch_bounds__(kMqThreads, 1) mq_score_kernel(SelectParams p,
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = blockIdx.y;
     const int q0 = blockIdx.x * kG;
+    const int share = blockIdx.z, S = gridDim.z;
     const int ng = min(kG, p.Q - q0);          // queries of this CTA (the rest of B is zero)
     const int64_t bq0 = (int64_t)b * p.Q + q0;
     const int64_t row_base = (int64_t)b * p.cap;
     int nmax = 0;
     for (int g = 0; g < ng; ++g) nmax = max(nmax, n_visible(p.q_pos[bq0 + g], p.n_entries[b], p.m, p.cap));
-    const int ntiles = (nmax + kTile - 1) / kTile;
+    // this share's tiles [t_lo, t_lo + ntiles) of the group's range, whole stages
+    const int ntiles_all = (nmax + kTile - 1) / kTile;
+    const int chunk = ((ntiles_all + S - 1) / S + kTPS - 1) / kTPS * kTPS;
+    const int t_lo = min(ntiles_all, share * chunk);
+    const int ntiles = min(ntiles_all, t_lo + chunk) - t_lo;
     const int nstages = (ntiles + kTPS - 1) / kTPS;
+    const int lo = t_lo * kTile;               // first entry of the share
     int32_t* status = p.status;
 
     if (tid == 0) {
@@ -112,7 +121,7 @@ __global__ void __launch_bounds__(kMqThreads, 1) mq_score_kernel(SelectParams p,
     const uint32_t tbase = s.tmem_base;
 
     if (warp == 0) {
-        producer_dense(s, p.ik, p.ik_sc, row_base, 0, ntiles, nstages, status, lane);
+        producer_dense(s, p.ik, p.ik_sc, row_base, lo, ntiles, nstages, status, lane);
     } else if (warp == 1) {
         if (lane == 0) {
             tc::tc_fence_after();
@@ -196,7 +205,7 @@ __global__ void __launch_bounds__(kMqThreads, 1) mq_score_kernel(SelectParams p,
                 }
                 const KeyScales ks = key_scales(stage_scales(s, t % kMqRing, i, row));   // shared by the queries
                 if (i == ntl - 1) release_stage(s, t, lane);
-                const int e = u * kTile + row;
+                const int e = lo + u * kTile + row;
 #pragma unroll
                 for (int j = 0; j < kQPW; ++j) {
                     const int g = gb + j;
@@ -220,8 +229,15 @@ __global__ void __launch_bounds__(kMqThreads, 1) mq_score_kernel(SelectParams p,
     __syncthreads();
     if (warp == 1) tc::tmem_dealloc(tbase, kMqCols);
     if (aborted(s)) return;
-    for (int i = tid; i < ng * kNB1; i += kMqThreads) hist_out[bq0 * kNB1 + i] = (&s.hist[0][0])[i];
-    if (p.blockmax) {   // blocks with no visible position
+    if (S == 1) {
+        for (int i = tid; i < ng * kNB1; i += kMqThreads) hist_out[bq0 * kNB1 + i] = (&s.hist[0][0])[i];
+    } else {   // the shares add into the zeroed workspace histograms
+        for (int i = tid; i < ng * kNB1; i += kMqThreads) {
+            const uint32_t c = (&s.hist[0][0])[i];
+            if (c) atomicAdd(&hist_out[bq0 * kNB1 + i], c);
+        }
+    }
+    if (p.blockmax && share == 0) {   // blocks with no visible position
         for (int g = 0; g < ng; ++g) {
             const int nvg = n_visible(p.q_pos[bq0 + g], p.n_entries[b], p.m, p.cap);
             for (int64_t j = (nvg + kBlk - 1) / kBlk + tid; j < p.nb_cap; j += kMqThreads)
@@ -231,19 +247,25 @@ __global__ void __launch_bounds__(kMqThreads, 1) mq_score_kernel(SelectParams p,
 }
 
 // ---------------------------------------------------------------------------- selection
-constexpr int kST = 256;                      // threads of a selecting CTA
-constexpr int kMaxVis = 65536;                // entries a query may see on this path
-constexpr int kSW = kMaxVis / 32;             // bitmap words
-constexpr int kWPT = kSW / kST;               // bitmap words per thread (8)
+constexpr int kMaxVis = 262144;               // entries a query may see on this path
+constexpr int kSmallVis = 65536;              // the smaller selector (two CTAs per SM)
 constexpr int kCandMax = 4096;                // threshold-bin entries listed
 constexpr int kNB2 = 2048, kNB3 = 1024;
+constexpr int kPB = 8;                        // prefix loads of a thread in flight together
 
+template <int MAXVIS>
 struct SelSmem {
+    // threads of a selecting CTA: the large selector runs alone on its SM (its bitmaps),
+    // with twice the threads to keep as many prefix loads in flight
+    static constexpr int kST = MAXVIS > kSmallVis ? 512 : 256;
+    static constexpr int kSW = MAXVIS / 32;   // bitmap words
+    static constexpr int kWPT = kSW / kST;    // bitmap words per thread
     uint32_t hist[kNB1];
     uint32_t hist2[kNB2];
     uint32_t hist3[kNB3];
     uint32_t selbm[kSW];                      // entries above T (and the ties taken)
     uint32_t tiebm[kSW];                      // entries equal to T
+    uint32_t h16[kST / 32][32];               // bin d1's entries by the prefix's low 5 bits, per warp
     int32_t cpos[kCandMax];                   // the threshold bin's entries
     uint32_t ckey[kCandMax];                  // and their exact keys
     uint32_t wsum[kST / 32];
@@ -261,7 +283,9 @@ __device__ __forceinline__ uint32_t warp_incl_scan_u(uint32_t v, int lane) {
 }
 
 // Exclusive prefix of v over the CTA's threads in order; *total = the sum.
+template <class SelSmem>
 __device__ __forceinline__ uint32_t scan_excl(SelSmem& s, uint32_t v, int tid, uint32_t* total) {
+    constexpr int kST = SelSmem::kST;
     const int warp = tid >> 5, lane = tid & 31;
     const uint32_t inc = warp_incl_scan_u(v, lane);
     if (lane == 31) s.wsum[warp] = inc;
@@ -280,8 +304,9 @@ __device__ __forceinline__ uint32_t scan_excl(SelSmem& s, uint32_t v, int tid, u
 // The bin b of the NB-bin histogram holding the R-th largest key (R >= 1):
 // keys above b < R <= keys above b + count of b.  Leaves (b, keys above b) in
 // s.res.  All threads call it.
-template <int NB>
+template <int NB, class SelSmem>
 __device__ __forceinline__ void find_bin_local(SelSmem& s, const uint32_t* hist, uint32_t R, int tid) {
+    constexpr int kST = SelSmem::kST;
     constexpr int PER = NB / kST;             // bins per thread, the highest on thread 0
     const int b0 = NB - PER * (tid + 1);
     uint32_t h[PER], sum = 0;
@@ -306,9 +331,13 @@ __device__ __forceinline__ void find_bin_local(SelSmem& s, const uint32_t* hist,
     __syncthreads();
 }
 
-__global__ void __launch_bounds__(kST) mq_select_kernel(SelectParams p, const uint16_t* prefix, const uint32_t* hist_in) {
+template <int MAXVIS>
+__global__ void __launch_bounds__(SelSmem<MAXVIS>::kST, MAXVIS > kSmallVis ? 1 : 2)
+    mq_select_kernel(SelectParams p, const uint16_t* prefix, const uint32_t* hist_in) {
     pdl_enter();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
+    using SelSmem = csa2::SelSmem<MAXVIS>;
+    constexpr int kSW = SelSmem::kSW, kWPT = SelSmem::kWPT, kST = SelSmem::kST;
     SelSmem& s = *reinterpret_cast<SelSmem*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31;
     const int64_t bq = blockIdx.x;
@@ -322,41 +351,94 @@ __global__ void __launch_bounds__(kST) mq_select_kernel(SelectParams p, const ui
         return;
     }
     for (int i = tid; i < kNB1; i += kST) s.hist[i] = hist_in[bq * kNB1 + i];
-    for (int i = tid; i < kNB2 + kNB3 + 2 * kSW; i += kST) s.hist2[i] = 0u;   // hist2, hist3, both bitmaps
+    for (int i = tid; i < kNB2 + kNB3 + 2 * kSW + kST; i += kST) s.hist2[i] = 0u;   // hist2, hist3, both bitmaps, h16
     if (tid == 0) s.ncand = 0;
     __syncthreads();
     find_bin_local<kNB1>(s, s.hist, K1, tid);
     const uint32_t d1 = s.res[0];
-    const uint32_t R = K1 - s.res[1];   // keys to take from bin d1 (1 <= R)
+    uint32_t R = K1 - s.res[1];   // keys to take from bin d1 (1 <= R)
 
-    // one read of the prefixes: bins above d1 into the bitmap, bin d1 listed
+    // reads of the prefixes, kPB loads of a thread in flight together (a uniform trip count,
+    // for the warp scans): classify(prefix) = 1 puts the entry into the bitmap (above the
+    // threshold bin), 2 lists it (in the bin), 0 neither
     const uint16_t* pre = prefix + bq * p.cap;
-    for (int c = tid; 8 * (c - lane) < nvis; c += kST) {   // warp-uniform trip count
-        const int e0 = 8 * c;
-        const uint4 x = e0 < nvis ? *reinterpret_cast<const uint4*>(pre + e0) : make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-        uint32_t ma = 0, mc = 0;
+    const int n8 = (nvis + 7) >> 3;
+    auto sweep = [&](auto classify) {
+        for (int base = 0; base < n8; base += kPB * kST) {
+            uint4 xs[kPB];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint32_t bin = ((w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu) >> 5;
-            const bool in = e0 + j < nvis;
-            ma |= (uint32_t)(in && bin > d1) << j;
-            mc |= (uint32_t)(in && bin == d1) << j;
-        }
-        if (ma) atomicOr(&s.selbm[e0 >> 5], ma << (e0 & 31));
-        const uint32_t n = __popc(mc);
-        const uint32_t incl = warp_incl_scan_u(n, lane);
-        uint32_t base = 0;
-        if (lane == 31 && incl) base = atomicAdd(&s.ncand, incl);
-        base = __shfl_sync(0xFFFFFFFFu, base, 31) + incl - n;
+            for (int r = 0; r < kPB; ++r) {
+                const int c = base + r * kST + tid;
+                xs[r] = c < n8 ? __ldcg(reinterpret_cast<const uint4*>(pre) + c) : make_uint4(0u, 0u, 0u, 0u);
+            }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint32_t slot = base + (uint32_t)__popc(mc & ((1u << j) - 1u));
-            if (((mc >> j) & 1u) && slot < (uint32_t)kCandMax) s.cpos[slot] = e0 + j;
+            for (int r = 0; r < kPB; ++r) {
+                const int e0 = 8 * (base + r * kST + tid);
+                const uint32_t w[4] = {xs[r].x, xs[r].y, xs[r].z, xs[r].w};
+                uint32_t ma = 0, mc = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t p16 = (w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+                    const int c = e0 + j < nvis ? classify(p16) : 0;
+                    ma |= (uint32_t)(c == 1) << j;
+                    mc |= (uint32_t)(c == 2) << j;
+                }
+                if (ma) atomicOr(&s.selbm[e0 >> 5], ma << (e0 & 31));
+                const uint32_t n = __popc(mc);
+                const uint32_t incl = warp_incl_scan_u(n, lane);
+                uint32_t cbase = 0;
+                if (lane == 31 && incl) cbase = atomicAdd(&s.ncand, incl);
+                cbase = __shfl_sync(0xFFFFFFFFu, cbase, 31) + incl - n;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t slot = cbase + (uint32_t)__popc(mc & ((1u << j) - 1u));
+                    if (((mc >> j) & 1u) && slot < (uint32_t)kCandMax) s.cpos[slot] = e0 + j;
+                }
+            }
         }
-    }
+    };
+    // first read: bins above d1 into the bitmap, bin d1 listed and counted by the prefix's
+    // low 5 bits
+    sweep([&](uint32_t p16) -> int {
+        const uint32_t bin = p16 >> 5;
+        if (bin == d1) {
+            atomicAdd(&s.h16[tid >> 5][p16 & 31u], 1u);
+            return 2;
+        }
+        return bin > d1 ? 1 : 0;
+    });
     __syncthreads();
-    const uint32_t nc = s.ncand;
+    uint32_t nc = s.ncand;
+    uint32_t pmask = 0xFFE0u, pval = d1 << 5;   // the prefixes of the threshold bin
+    if (nc > (uint32_t)kCandMax) {
+        // too many to list (a far tail of close keys): a second read keeps the sub-bin of the
+        // prefix's low 5 bits that holds the R-th key, marks the sub-bins above it
+        if (tid == 0) {
+            uint32_t above = 0;
+            int bb = 31;
+            for (; bb > 0; --bb) {
+                uint32_t c = 0;
+                for (int w = 0; w < kST / 32; ++w) c += s.h16[w][bb];
+                if (above + c >= R) break;
+                above += c;
+            }
+            s.res[0] = (uint32_t)bb;
+            s.res[1] = above;
+            s.ncand = 0;
+        }
+        __syncthreads();
+        const uint32_t d1b = s.res[0];
+        R -= s.res[1];
+        pmask = 0xFFFFu;
+        pval = (d1 << 5) | d1b;
+        sweep([&](uint32_t p16) -> int {
+            if ((p16 >> 5) != d1) return 0;
+            const uint32_t lo5 = p16 & 31u;
+            return lo5 > d1b ? 1 : (lo5 == d1b ? 2 : 0);
+        });
+        __syncthreads();
+        nc = s.ncand;
+    }
     QReg Rq;
     load_query(Rq, p.q + bq * 128, p.q_sc + bq * 16, p.w + bq * 4);
     const uint8_t* ik = p.ik + (int64_t)b * p.cap * 32;
@@ -388,9 +470,9 @@ __global__ void __launch_bounds__(kST) mq_select_kernel(SelectParams p, const ui
             else if (key == T) atomicOr(&s.tiebm[e >> 5], 1u << (e & 31));
         }
     } else {
-        // too many to list: passes over bin d1 that re-score its entries
+        // still too many (many equal or close keys): passes that re-score the bin's entries
         for (int e = tid; e < nvis; e += kST) {
-            if ((uint32_t)(pre[e] >> 5) != d1) continue;
+            if (((uint32_t)pre[e] & pmask) != pval) continue;
             const uint32_t key = score_key(entry_score_at(Rq, ik, iks, e));
             atomicAdd(&s.hist2[(key >> 10) & (kNB2 - 1)], 1u);
         }
@@ -399,7 +481,7 @@ __global__ void __launch_bounds__(kST) mq_select_kernel(SelectParams p, const ui
         const uint32_t p2 = (d1 << 11) | s.res[0];
         const uint32_t R3 = R - s.res[1];
         for (int e = tid; e < nvis; e += kST) {
-            if ((uint32_t)(pre[e] >> 5) != d1) continue;
+            if (((uint32_t)pre[e] & pmask) != pval) continue;
             const uint32_t key = score_key(entry_score_at(Rq, ik, iks, e));
             if ((key >> 10) == p2) atomicAdd(&s.hist3[key & (kNB3 - 1)], 1u);
         }
@@ -408,7 +490,7 @@ __global__ void __launch_bounds__(kST) mq_select_kernel(SelectParams p, const ui
         T = (p2 << 10) | s.res[0];
         Rt = R3 - s.res[1];
         for (int e = tid; e < nvis; e += kST) {
-            if ((uint32_t)(pre[e] >> 5) != d1) continue;
+            if (((uint32_t)pre[e] & pmask) != pval) continue;
             const uint32_t key = score_key(entry_score_at(Rq, ik, iks, e));
             if (key > T) atomicOr(&s.selbm[e >> 5], 1u << (e & 31));
             else if (key == T) atomicOr(&s.tiebm[e >> 5], 1u << (e & 31));
@@ -461,6 +543,14 @@ bool index_mq_eligible(int B, int Q, int64_t cap) {
     return (int64_t)B * Q > kSplitSMs && Q >= kG && cap <= kMaxVis;
 }
 
+// Entry-range shares of the scoring: enough CTAs for the SMs when the groups of 8
+// queries alone are fewer (one CTA per SM).
+static int mq_shares(int B, int Q) {
+    const int groups = ((Q + kG - 1) / kG) * B;
+    int S = kSplitSMs / groups;
+    return S < 1 ? 1 : (S > 16 ? 16 : S);
+}
+
 size_t index_mq_ws_bytes(int B, int Q, int64_t cap) {
     const size_t bq = (size_t)B * Q;
     return align256(bq * (size_t)cap * 2) + align256(bq * kNB1 * 4);
@@ -471,18 +561,28 @@ cudaError_t launch_index_mq(SelectParams& p, void* mq_ws, cudaStream_t st) {
     uint16_t* prefix = (uint16_t*)mq_ws;
     uint32_t* hist = (uint32_t*)((char*)mq_ws + align256(bq * (size_t)p.cap * 2));
     const int smem1 = (int)sizeof(MqSmem) + 1024;
-    const int smem2 = (int)sizeof(SelSmem);
+    const int smem_small = (int)sizeof(SelSmem<kSmallVis>), smem_large = (int)sizeof(SelSmem<kMaxVis>);
     cudaError_t e = g_mq_attr.run([&] {
         cudaError_t r = cudaFuncSetAttribute(mq_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
-        if (r == cudaSuccess) r = cudaFuncSetAttribute(mq_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2);
+        if (r == cudaSuccess)
+            r = cudaFuncSetAttribute(mq_select_kernel<kSmallVis>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_small);
+        if (r == cudaSuccess)
+            r = cudaFuncSetAttribute(mq_select_kernel<kMaxVis>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_large);
         return r;
     });
     if (e != cudaSuccess) return e;
-    e = launch_ex(mq_score_kernel, dim3((p.Q + kG - 1) / kG, p.B), dim3(kMqThreads), smem1, st, 0, p,
-                              prefix, hist);
+    const int S = mq_shares(p.B, p.Q);
+    if (S > 1) {   // the shares add their histograms
+        e = cudaMemsetAsync(hist, 0, bq * kNB1 * sizeof(uint32_t), st);
+        if (e != cudaSuccess) return e;
+    }
+    e = launch_ex(mq_score_kernel, dim3((p.Q + kG - 1) / kG, p.B, S), dim3(kMqThreads), smem1, st, 0, p, prefix, hist);
     if (e != cudaSuccess) return e;
-    return launch_ex(mq_select_kernel, dim3((unsigned)bq), dim3(kST), smem2, st, 0, p, (const uint16_t*)prefix,
-                     (const uint32_t*)hist);
+    if (p.cap <= kSmallVis)
+        return launch_ex(mq_select_kernel<kSmallVis>, dim3((unsigned)bq), dim3(SelSmem<kSmallVis>::kST), smem_small, st, 0, p,
+                         (const uint16_t*)prefix, (const uint32_t*)hist);
+    return launch_ex(mq_select_kernel<kMaxVis>, dim3((unsigned)bq), dim3(SelSmem<kMaxVis>::kST), smem_large, st, 0, p,
+                     (const uint16_t*)prefix, (const uint32_t*)hist);
 }
 
 }  // namespace csa2

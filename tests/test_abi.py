@@ -49,8 +49,10 @@ def test_workspace_sizes_are_host_only(L):
     # 16-bit key prefixes and its 2,048-bin histogram for the many-query path
     many = L.csa2_workspace_bytes(csa.OP_INDEX_TOPK, 1, 4096, 32768, 512, 0)
     assert many >= 4096 * 32768 * 2 + 4096 * 2048 * 4
-    # beyond 65,536 entries that path is not taken, and nothing is reserved for it
-    assert L.csa2_workspace_bytes(csa.OP_INDEX_TOPK, 1, 4096, 131072, 512, 0) < 4096 * 131072 * 2
+    # up to 262,144 entries (a replay through a long decoder context) too
+    assert L.csa2_workspace_bytes(csa.OP_INDEX_TOPK, 4, 128, 262144, 512, 0) >= 512 * 262144 * 2 + 512 * 2048 * 4
+    # beyond that the path is not taken, and nothing is reserved for it
+    assert L.csa2_workspace_bytes(csa.OP_INDEX_TOPK, 1, 4096, 524288, 512, 0) < 4096 * 524288 * 2
 
 
 def test_invalid_arguments_rejected_before_launch(L):

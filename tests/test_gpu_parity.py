@@ -157,6 +157,22 @@ def test_index_topk_many_queries(csa, B, Q):
     assert np.array_equal(np_(bm), rbm)
 
 
+def test_index_topk_many_queries_large_cache(csa):
+    # the many-query path above 65,536 entries: 152 queries = 19 groups of 8, so the
+    # scoring splits each group's entry range into 7 shares whose histograms add up,
+    # and the selector keeps 131,072-entry position bitmaps
+    B, Q, cap, m, k = 1, 152, 131072, 1, 512
+    rng = np.random.default_rng(57)
+    q_pos = np.sort(rng.integers(0, 130000, size=(B, Q))).astype(np.int32)
+    q_pos[0, :5] = [0, 7, 127, 65535, 65536]
+    q_pos[0, -3:] = [129998, 129999, 129999]
+    grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(151, B, Q, cap, [130000], m, q_pos.tolist(), k)
+    idx, bm = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, k, blockmax=True)
+    ridx, rbm = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, m, q_pos, k, blockmax=True)
+    assert np.array_equal(np_(idx), ridx)
+    assert np.array_equal(np_(bm).view(np.uint32), rbm.view(np.uint32))
+
+
 def test_index_topk_many_queries_threshold_bin_overflow(csa):
     # all-tie queries on the many-query path: with zero query codes or zero head
     # weights every visible score is +0, so the threshold bin holds every visible
