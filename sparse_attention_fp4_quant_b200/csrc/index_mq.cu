@@ -332,7 +332,7 @@ __device__ __forceinline__ void find_bin_local(SelSmem& s, const uint32_t* hist,
 }
 
 template <int MAXVIS>
-__global__ void __launch_bounds__(SelSmem<MAXVIS>::kST, MAXVIS > kSmallVis ? 1 : 2)
+__global__ void __launch_bounds__(SelSmem<MAXVIS>::kST, MAXVIS > kSmallVis ? 1 : 3)
     mq_select_kernel(SelectParams p, const uint16_t* prefix, const uint32_t* hist_in) {
     pdl_enter();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -543,12 +543,25 @@ bool index_mq_eligible(int B, int Q, int64_t cap) {
     return (int64_t)B * Q > kSplitSMs && Q >= kG && cap <= kMaxVis;
 }
 
-// Entry-range shares of the scoring: enough CTAs for the SMs when the groups of 8
-// queries alone are fewer (one CTA per SM).
-static int mq_shares(int B, int Q) {
-    const int groups = ((Q + kG - 1) / kG) * B;
-    int S = kSplitSMs / groups;
-    return S < 1 ? 1 : (S > 16 ? 16 : S);
+// Entry-range shares of the scoring (one CTA per SM): the count that minimises waves x
+// tiles per CTA, each CTA also paying its set-up (TMEM, the query operands, the histogram
+// flush: about kSetupTiles tiles' time).  A last wave that leaves most SMs idle costs
+// as much as a full one.
+static int mq_shares(int B, int Q, int64_t cap) {
+    constexpr int64_t kSetupTiles = 8;
+    const int64_t groups = (int64_t)((Q + kG - 1) / kG) * B;
+    const int64_t tiles = (cap + kTile - 1) / kTile;
+    int best = 1;
+    int64_t best_cost = -1;
+    for (int S = 1; S <= 16; ++S) {
+        const int64_t waves = (groups * S + kSplitSMs - 1) / kSplitSMs;
+        const int64_t cost = waves * ((tiles + S - 1) / S + kSetupTiles);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = S;
+        }
+    }
+    return best;
 }
 
 size_t index_mq_ws_bytes(int B, int Q, int64_t cap) {
@@ -571,7 +584,7 @@ cudaError_t launch_index_mq(SelectParams& p, void* mq_ws, cudaStream_t st) {
         return r;
     });
     if (e != cudaSuccess) return e;
-    const int S = mq_shares(p.B, p.Q);
+    const int S = mq_shares(p.B, p.Q, p.cap);
     if (S > 1) {   // the shares add their histograms
         e = cudaMemsetAsync(hist, 0, bq * kNB1 * sizeof(uint32_t), st);
         if (e != cudaSuccess) return e;
