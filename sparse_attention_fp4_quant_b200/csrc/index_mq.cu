@@ -549,12 +549,14 @@ bool index_mq_eligible(int B, int Q, int64_t cap) {
 // as much as a full one.
 static int mq_shares(int B, int Q, int64_t cap) {
     constexpr int64_t kSetupTiles = 8;
+    const int dev_sms = device_sm_count();   // a grid choice only: the workspace does not depend on it
+    const int64_t sms = dev_sms > 0 ? dev_sms : kSplitSMs;
     const int64_t groups = (int64_t)((Q + kG - 1) / kG) * B;
     const int64_t tiles = (cap + kTile - 1) / kTile;
     int best = 1;
     int64_t best_cost = -1;
     for (int S = 1; S <= 16; ++S) {
-        const int64_t waves = (groups * S + kSplitSMs - 1) / kSplitSMs;
+        const int64_t waves = (groups * S + sms - 1) / sms;
         const int64_t cost = waves * ((tiles + S - 1) / S + kSetupTiles);
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;

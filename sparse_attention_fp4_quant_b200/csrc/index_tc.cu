@@ -59,15 +59,12 @@ __device__ __forceinline__ bool epilogue_any(bool v) {
     return r != 0;
 }
 
-// Epilogue warps, mode 2, after scoring: the bin d that holds the k-th largest key (bins
-// scanned from the top; every key when there are at most k), then one read of the keys
-// offers each entry in bin d or above to the exact Top-K, the entry index standing for the
-// position (the pool is ascending, so the two orders agree).  When those entries fit the
-// buffer nothing is compacted before the final select; otherwise the buffer makes room as
-// it fills, which is exact too, only slower.
+// Epilogue warps: from the histogram of the keys' top bits in s.hist, the bin that holds
+// the k-th largest key (bins scanned from the top; bin 0 when there are at most k keys)
+// into s.sel_bin, and the number of keys in it or above into s.sel_count.  After it no
+// thread reads the histogram, whose space the Top-K may take.
 template <int CAP>
-__device__ __forceinline__ void pool_select(TcSmem<CAP>& s, TopK<kEpiN, CAP, 1, kEpiT0>& tk, const uint32_t* qkeys,
-                                            int n_items, int k, int lane, int warp) {
+__device__ __forceinline__ void threshold_bin(TcSmem<CAP>& s, int k, int lane, int warp) {
     using TKE = TopK<kEpiN, CAP, 1, kEpiT0>;
     const int et = (int)threadIdx.x - kEpiT0, ew = warp - kEpiT0 / 32;
     constexpr int kPer = kHistBins / kEpiN;   // bins per thread, highest first
@@ -110,7 +107,19 @@ __device__ __forceinline__ void pool_select(TcSmem<CAP>& s, TopK<kEpiN, CAP, 1, 
             run += c[j];
         }
     }
-    TKE::sync();   // after it no thread reads the histogram, whose space the Top-K now takes
+    TKE::sync();
+}
+
+// Epilogue warps, mode 2, after scoring: the bin d that holds the k-th largest key, then
+// one read of the keys offers each entry in bin d or above to the exact Top-K, the entry
+// index standing for the position (the pool is ascending, so the two orders agree).  When
+// those entries fit the buffer nothing is compacted before the final select; otherwise
+// the buffer makes room as it fills, which is exact too, only slower.
+template <int CAP>
+__device__ __forceinline__ void pool_select(TcSmem<CAP>& s, TopK<kEpiN, CAP, 1, kEpiT0>& tk, const uint32_t* qkeys,
+                                            int n_items, int k, int lane, int warp) {
+    const int et = (int)threadIdx.x - kEpiT0;
+    threshold_bin<CAP>(s, k, lane, warp);
     const uint32_t d = s.sel_bin;
     const bool fast = s.sel_count <= (uint32_t)CAP;
     tk.init();
@@ -132,6 +141,60 @@ __device__ __forceinline__ void pool_select(TcSmem<CAP>& s, TopK<kEpiN, CAP, 1, 
                 const bool take = key4[q] != 0u && (key4[q] >> (32 - kHistBits)) >= d;
                 tk.offer(take, key4[q], i0 + q);
             }
+        }
+    }
+    tk.finish(k);
+}
+
+// The last CTA of a query, once every share has written its best k (padded to k with key
+// 0, which no finite score maps to): the histogram of all S k keys' top 11 bits gives the
+// bin of the k-th best, and only the keys in it or above are offered to the exact Top-K.
+// Offering all of them compacted the buffer every few hundred offers.  Every batch of
+// loads is in flight together.
+template <int CAP>
+__device__ __forceinline__ void merge_shares(TcSmem<CAP>& s, TopK<kEpiN, CAP, 1, kEpiT0>& tk, const uint32_t* keys,
+                                             const int32_t* poss, int total, int k, int lane, int warp) {
+    using TKE = TopK<kEpiN, CAP, 1, kEpiT0>;
+    constexpr int kB = 8;
+    const int et = (int)threadIdx.x - kEpiT0;
+    const uint32_t hist_base = tc::smem_u32(&s.hist[0]);
+    for (int i = et; i < kHistBins; i += kEpiN) shm::st(hist_base + 4u * (uint32_t)i, 0u);
+    TKE::sync();
+    for (int base = 0; base < total; base += kB * kEpiN) {
+        uint32_t kv[kB];
+#pragma unroll
+        for (int r = 0; r < kB; ++r) {
+            const int g = base + r * kEpiN + et;
+            kv[r] = g < total ? __ldcg(keys + g) : 0u;
+        }
+#pragma unroll
+        for (int r = 0; r < kB; ++r)
+            if (kv[r] != 0u) shm::red_add(hist_base + 4u * (kv[r] >> (32 - kHistBits)), 1u);
+    }
+    TKE::sync();
+    threshold_bin<CAP>(s, k, lane, warp);
+    const uint32_t d = s.sel_bin;
+    const bool fast = s.sel_count <= (uint32_t)CAP;
+    tk.init();
+    for (int base = 0; base < total; base += kB * kEpiN) {   // uniform trip count
+        uint32_t kv[kB];
+        int32_t pv[kB];
+#pragma unroll
+        for (int r = 0; r < kB; ++r) {
+            const int g = base + r * kEpiN + et;
+            kv[r] = g < total ? __ldcg(keys + g) : 0u;
+        }
+#pragma unroll
+        for (int r = 0; r < kB; ++r) {
+            const int g = base + r * kEpiN + et;
+            const bool take = kv[r] != 0u && (kv[r] >> (32 - kHistBits)) >= d;
+            pv[r] = take ? __ldcg(poss + g) : 0;
+            if (!take) kv[r] = 0u;
+        }
+#pragma unroll
+        for (int r = 0; r < kB; ++r) {
+            if (!fast) tk.make_room(k, kEpiN);
+            tk.offer(kv[r] != 0u, kv[r], pv[r]);
         }
     }
     tk.finish(k);
@@ -309,9 +372,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (S > 1) {
         const int cnt = tk.count();
         const int64_t off = ((int64_t)bq * S + share) * k;
-        for (int i = et; i < cnt; i += kEpiN) {
-            p.cand_key[off + i] = tk.key_at(i);
-            p.cand_pos[off + i] = tk.pos_at(i);
+        for (int i = et; i < k; i += kEpiN) {   // padded to k with key 0 (no entry)
+            p.cand_key[off + i] = i < cnt ? tk.key_at(i) : 0u;
+            if (i < cnt) p.cand_pos[off + i] = tk.pos_at(i);
         }
         if (et == 0) p.cand_cnt[(int64_t)bq * S + share] = cnt;
         __threadfence();
@@ -320,20 +383,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         TKE::sync();
         if (!s.last) return;
         __threadfence();
-        tk.init();
-        for (int c = 0; c < S; ++c) {
-            const int n = __ldcg(&p.cand_cnt[(int64_t)bq * S + c]);
-            const int64_t coff = ((int64_t)bq * S + c) * k;
-            for (int base = 0; base < n; base += kEpiN) {
-                tk.make_room(k, kEpiN);
-                const int i = base + et;
-                const bool valid = i < n;
-                const uint32_t key = valid ? __ldcg(&p.cand_key[coff + i]) : 0u;
-                const int32_t pos = valid ? __ldcg(&p.cand_pos[coff + i]) : 0;
-                tk.offer(valid, key, pos);
-            }
-        }
-        tk.finish(k);
+        merge_shares<CAP>(s, tk, p.cand_key + (int64_t)bq * S * k, p.cand_pos + (int64_t)bq * S * k, S * k, k, lane, warp);
         if (et == 0) p.counters[bq] = 0;
     }
     const int cnt = tk.count();
