@@ -110,14 +110,15 @@ __device__ __forceinline__ void threshold_bin(TcSmem<CAP>& s, int k, int lane, i
     TKE::sync();
 }
 
-// Epilogue warps, mode 2, after scoring: the bin d that holds the k-th largest key, then
-// one read of the keys offers each entry in bin d or above to the exact Top-K, the entry
-// index standing for the position (the pool is ascending, so the two orders agree).  When
-// those entries fit the buffer nothing is compacted before the final select; otherwise
-// the buffer makes room as it fills, which is exact too, only slower.
+// Epilogue warps, modes 2 and 3, after scoring: the bin d that holds the k-th largest
+// key, then one read of the keys offers each item i in bin d or above to the exact Top-K
+// as position pos0 + i (mode 3: the share's entries from pos0; mode 2: the entry index of
+// an ascending pool, which orders like the position).  When those items fit the buffer
+// nothing is compacted before the final select; otherwise the buffer makes room as it
+// fills, which is exact too, only slower.
 template <int CAP>
-__device__ __forceinline__ void pool_select(TcSmem<CAP>& s, TopK<kEpiN, CAP, 1, kEpiT0>& tk, const uint32_t* qkeys,
-                                            int n_items, int k, int lane, int warp) {
+__device__ __forceinline__ void keys_select(TcSmem<CAP>& s, TopK<kEpiN, CAP, 1, kEpiT0>& tk, const uint32_t* qkeys,
+                                            int n_items, int pos0, int k, int lane, int warp) {
     const int et = (int)threadIdx.x - kEpiT0;
     threshold_bin<CAP>(s, k, lane, warp);
     const uint32_t d = s.sel_bin;
@@ -139,7 +140,7 @@ __device__ __forceinline__ void pool_select(TcSmem<CAP>& s, TopK<kEpiN, CAP, 1, 
             for (int q = 0; q < 4; ++q) {
                 if (!fast) tk.make_room(k, kEpiN);
                 const bool take = key4[q] != 0u && (key4[q] >> (32 - kHistBits)) >= d;
-                tk.offer(take, key4[q], i0 + q);
+                tk.offer(take, key4[q], pos0 + i0 + q);
             }
         }
     }
@@ -201,7 +202,8 @@ __device__ __forceinline__ void merge_shares(TcSmem<CAP>& s, TopK<kEpiN, CAP, 1,
 }
 
 // MODE 0 = dense range (index Top-K), 1 = pool blocks (pool Top-K), 2 = pool blocks of an
-// ascending pool with the keys kept in the workspace (one share per query)
+// ascending pool with the keys kept in the workspace (one share per query), 3 = dense range
+// with the keys kept in the workspace ([B Q][cap])
 template <int MODE, int CAP>
 __global__ void __launch_bounds__(kThreads, 2)
     index_tc_kernel(SelectParams p) {
@@ -219,9 +221,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int nvis = n_visible(p.q_pos[bq], p.n_entries[b], p.m, p.cap);
     const int64_t row_base = (int64_t)b * p.cap;
 
+    constexpr bool kDense = MODE == 0 || MODE == 3, kKeys = MODE >= 2;
     // this share's candidates: dense = entries [lo, hi); pool = pool slots [lo, hi)
     int lo, hi, ntiles;
-    if (MODE == 0) {
+    if (kDense) {
         int chunk = (((nvis + S - 1) / S) + (kTPS * kTile - 1)) / (kTPS * kTile) * (kTPS * kTile);
         lo = min(nvis, share * chunk);
         hi = min(nvis, lo + chunk);
@@ -233,18 +236,20 @@ __global__ void __launch_bounds__(kThreads, 2)
         ntiles = (hi - lo + kPoolPerTile - 1) / kPoolPerTile;
     }
     const int nstages = (ntiles + kTPS - 1) / kTPS;
-    const int32_t* pool = (MODE != 0) ? p.pool + (int64_t)bq * p.P : nullptr;
-    // mode 2: this query's order keys, one per (tile, row): entry index i = slot * 8 + row
-    uint32_t* qkeys = (MODE == 2) ? p.keys + (int64_t)bq * ntiles * kTile : nullptr;
+    const int32_t* pool = kDense ? nullptr : p.pool + (int64_t)bq * p.P;
+    // this share's order keys, one per (tile, row): mode 2 item i = slot * 8 + row of the
+    // query's pool; mode 3 item i = entry lo + i of the query's [cap] row
+    uint32_t* qkeys = MODE == 2 ? p.keys + (int64_t)bq * ntiles * kTile
+                                : (MODE == 3 ? p.keys + (int64_t)bq * p.cap + lo : nullptr);
 
-    if (tid == 0) init_barriers(s.pipe, kEpiN, MODE == 0 ? 1u : kPoolLanes);
+    if (tid == 0) init_barriers(s.pipe, kEpiN, kDense ? 1u : kPoolLanes);
     if (warp == 1) setup_query(s.pipe, p.q + (int64_t)bq * 128, p.q_sc + (int64_t)bq * 16, lane, kPipeCols);
     __syncthreads();
     const uint32_t tbase = s.pipe.tmem_base;
     int32_t* status = p.status;
 
     if (warp == 0) {
-        if constexpr (MODE == 0)
+        if constexpr (kDense)
             producer_dense(s.pipe, p.ik, p.ik_sc, row_base, lo, ntiles, nstages, status, lane, p.test_starve != 0);
         else
             producer_pool_async(s.pipe, p.ik, p.ik_sc, row_base, lo, hi, ntiles, nstages, pool, nvis, &s.stage_blk[0][0][0],
@@ -255,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         // ------------------------------------------------------------ epilogue
         TKE tk(s.topk);
         const uint32_t hist_base = tc::smem_u32(&s.hist[0]);
-        if constexpr (MODE == 2) {
+        if constexpr (kKeys) {
             for (int i = tid - kEpiT0; i < kHistBins; i += kEpiN) shm::st(hist_base + 4u * (uint32_t)i, 0u);
             TKE::sync();
         } else {
@@ -266,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int row = quarter * 32 + lane;
         const uint64_t w01 = f2pack(__ldg(p.w + (int64_t)bq * 4 + 0), __ldg(p.w + (int64_t)bq * 4 + 1));
         const uint64_t w23 = f2pack(__ldg(p.w + (int64_t)bq * 4 + 2), __ldg(p.w + (int64_t)bq * 4 + 3));
-        float* bm = (MODE == 0 && p.blockmax) ? p.blockmax + (int64_t)bq * p.nb_cap : nullptr;
+        float* bm = (kDense && p.blockmax) ? p.blockmax + (int64_t)bq * p.nb_cap : nullptr;
         bool stop = false;
         for (int t = 0; t < nstages && !stop; ++t) {
             const int a = t % kAcc;
@@ -293,10 +298,10 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
             for (int j = 0; j < kTPG; ++j) {
                 skw[j] = landed ? stage_scales(s.pipe, t % kRing, kTPG * group + j, row) : 0u;
-                sblk[j] = (MODE != 0 && landed) ? s.stage_blk[t % kRing][kTPG * group + j][row >> 3] : -1;
+                sblk[j] = (!kDense && landed) ? s.stage_blk[t % kRing][kTPG * group + j][row >> 3] : -1;
             }
             if (landed) release_stage(s.pipe, t, lane);
-            if constexpr (MODE == 2) {
+            if constexpr (kKeys) {
                 if (!landed) {   // warp-uniform; the warps meet again after the loop
                     stop = true;
                     break;
@@ -306,13 +311,21 @@ __global__ void __launch_bounds__(kThreads, 2)
                     const int g = t * kTPS + kTPG * group + j;
                     if (g >= ntiles) break;   // warp-uniform
                     int64_t e = -1;
-                    if (sblk[j] >= 0) {
+                    if (MODE == 3) {
+                        const int ee = lo + g * kTile + row;
+                        if (ee < hi) e = ee;
+                    } else if (sblk[j] >= 0) {
                         const int64_t ee = (int64_t)sblk[j] * kBlk + (row & 7);
                         if (ee < nvis) e = ee;
                     }
                     const bool valid = e >= 0;
+                    const float score = valid ? score_of(v[j], key_scales(skw[j]), w01, w23) : -INFINITY;
+                    if (MODE == 3 && bm) {
+                        const float m8 = block_max8(score, lane);
+                        if ((lane & 7) == 0 && valid) bm[e >> 3] = m8;
+                    }
                     // key 0 marks "no entry": a finite score's key is never 0
-                    const uint32_t key = valid ? score_key(score_of(v[j], key_scales(skw[j]), w01, w23)) : 0u;
+                    const uint32_t key = valid ? score_key(score) : 0u;
                     __stcg(qkeys + g * kTile + row, key);
                     hist_add(hist_base, valid ? (int)(key >> (32 - kHistBits)) : -1);
                 }
@@ -346,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 tk.offer(th, valid, score_key(valid ? score : 0.0f), (int32_t)(valid ? e : 0));
             }
         }
-        if (!stop && MODE == 0 && bm) {  // blocks with no visible position
+        if (!stop && kDense && bm) {  // blocks with no visible position
             const int64_t jb = (nvis + kBlk - 1) / kBlk;
             const int64_t rest = p.nb_cap - jb;
             if (rest > 0) {
@@ -355,9 +368,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int64_t j = j0 + (tid - kEpiT0); j < j1; j += kEpiN) bm[j] = -INFINITY;
             }
         }
-        if constexpr (MODE == 2) {
+        if constexpr (kKeys) {
             stop = epilogue_any(stop || aborted(s.pipe));
-            if (!stop) pool_select<CAP>(s, tk, qkeys, ntiles * kTile, k, lane, warp);
+            if (!stop) keys_select<CAP>(s, tk, qkeys, ntiles * kTile, MODE == 3 ? lo : 0, k, lane, warp);
         } else {
             if (!stop) tk.finish(k);
         }
@@ -426,12 +439,24 @@ cudaError_t launch_tc(SelectParams& p, int S, cudaStream_t st) {
 }
 
 cudaError_t launch_index_tc(int op, SelectParams& p, int S, cudaStream_t st) {
-    // a pool search with its keys in the workspace (the caller vouches for an ascending pool)
-    const int mode = (op == CSA2_OP_POOL_TOPK) ? ((p.keys && S == 1) ? 2 : 1) : 0;
+    // with the keys in the workspace: a pool search (the caller vouches for an ascending
+    // pool, one share per query) or a dense index
+    const int mode = (op == CSA2_OP_POOL_TOPK) ? ((p.keys && S == 1) ? 2 : 1) : (p.keys ? 3 : 0);
     // the buffer must hold k survivors plus one stage of offers
-    if (p.k <= 2048 - kTPS * kTile)
-        return mode == 0 ? launch_tc<0, 2048>(p, S, st) : mode == 1 ? launch_tc<1, 2048>(p, S, st) : launch_tc<2, 2048>(p, S, st);
-    return mode == 0 ? launch_tc<0, 4096>(p, S, st) : mode == 1 ? launch_tc<1, 4096>(p, S, st) : launch_tc<2, 4096>(p, S, st);
+    if (p.k <= 2048 - kTPS * kTile) {
+        switch (mode) {
+            case 0: return launch_tc<0, 2048>(p, S, st);
+            case 1: return launch_tc<1, 2048>(p, S, st);
+            case 2: return launch_tc<2, 2048>(p, S, st);
+            default: return launch_tc<3, 2048>(p, S, st);
+        }
+    }
+    switch (mode) {
+        case 0: return launch_tc<0, 4096>(p, S, st);
+        case 1: return launch_tc<1, 4096>(p, S, st);
+        case 2: return launch_tc<2, 4096>(p, S, st);
+        default: return launch_tc<3, 4096>(p, S, st);
+    }
 }
 
 }  // namespace csa2

@@ -65,19 +65,29 @@ class Group:
     """A CSA2 layer group: bf16 latent rows (generator), the oracle's quantised
     cache (numpy) and the CUDA path's own quantised cache (device)."""
 
-    def __init__(self, seed, B, cap, n_entries, m=1, device="cuda", latent_device=None):
+    def __init__(self, seed, B, cap, n_entries, m=1, device="cuda", latent_device=None, rows=None):
+        """rows (a multiple of 128, at least every n_entries): only the first rows entries of
+        each batch row hold data, the rest of the capacity stays zero on both sides."""
         import sparse_attention_fp4_quant_b200 as csa
         self.B, self.cap, self.m = B, cap, m
+        self.rows = cap if rows is None else rows
+        assert self.rows % 128 == 0 and self.rows <= cap and max(n_entries) <= self.rows
         latent_device = latent_device or device
-        self.latent = torch.stack([synth.latent(synth.seed_of("grp", seed, b), cap, 0, latent_device)
-                                   for b in range(B)])  # [B, cap, 512] bf16
+        self.latent = torch.stack([synth.latent(synth.seed_of("grp", seed, b), self.rows, 0, latent_device)
+                                   for b in range(B)])  # [B, rows, 512] bf16
         self.W = synth.proj_w(seed).to(device)
         self.n_entries = np.array(n_entries, np.int32)
         # CUDA path: its own quantiser and projection write the cache
         self.kv = csa.KV(B, cap, m, device)
-        lat_dev = self.latent.to(device).reshape(-1, 512)
-        csa.csa2_quant_nvfp4(lat_dev, self.kv.lat.view(-1, 256), self.kv.lat_sc.view(-1, 32))
-        csa.csa2_index_k_proj(lat_dev, self.W, self.kv.ik.view(-1, 32), self.kv.ik_sc.view(-1, 4))
+        if self.rows == cap:
+            lat_dev = self.latent.to(device).reshape(-1, 512)
+            csa.csa2_quant_nvfp4(lat_dev, self.kv.lat.view(-1, 256), self.kv.lat_sc.view(-1, 32))
+            csa.csa2_index_k_proj(lat_dev, self.W, self.kv.ik.view(-1, 32), self.kv.ik_sc.view(-1, 4))
+        else:   # per batch row: the first rows entries (whole 128-entry tiles of the indexer-K image)
+            for b in range(B):
+                lat_b = self.latent[b].to(device)
+                csa.csa2_quant_nvfp4(lat_b, self.kv.lat[b, :self.rows], self.kv.lat_sc[b, :self.rows])
+                csa.csa2_index_k_proj(lat_b, self.W, self.kv.ik[b, :self.rows], self.kv.ik_sc[b, :self.rows])
         self.kv.n_entries.copy_(torch.from_numpy(self.n_entries))
         self._oracle = None
 
@@ -86,9 +96,13 @@ class Group:
             lb = bits(self.latent.reshape(-1, 512))
             lat, lat_sc = oracle.quant_nvfp4(lb)
             ik, iks = oracle.index_k_proj(lb, np_(self.W))
-            B, cap = self.B, self.cap
-            self._oracle = dict(lat=lat.reshape(B, cap, 256), lat_sc=lat_sc.reshape(B, cap, 32),
-                                ik=ik.reshape(B, cap, 32), iks=iks.reshape(B, cap, 4))
+            B, cap, rows = self.B, self.cap, self.rows
+
+            def full(a, width):   # [B, rows, width] -> [B, cap, width], zero beyond rows
+                out = np.zeros((B, cap, width), a.dtype)
+                out[:, :rows] = a.reshape(B, rows, width)
+                return out
+            self._oracle = dict(lat=full(lat, 256), lat_sc=full(lat_sc, 32), ik=full(ik, 32), iks=full(iks, 4))
         return self._oracle
 
 

@@ -116,8 +116,8 @@ def test_append_tokens_bit_exact(csa, rows):
 
 
 # ---------------------------------------------------------------- index / Top-K
-def _index_case(seed, B, Q, cap, n_entries, m, q_pos, k):
-    grp = Group(seed, B, cap, n_entries, m)
+def _index_case(seed, B, Q, cap, n_entries, m, q_pos, k, rows=None):
+    grp = Group(seed, B, cap, n_entries, m, rows=rows)
     o = grp.oracle_cache()
     gik, giks = kv_ik_rows(grp.kv)
     assert np.array_equal(gik, o["ik"]) and np.array_equal(giks, o["iks"])
@@ -171,6 +171,28 @@ def test_index_topk_many_queries_large_cache(csa):
     ridx, rbm = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, m, q_pos, k, blockmax=True)
     assert np.array_equal(np_(idx), ridx)
     assert np.array_equal(np_(bm).view(np.uint32), rbm.view(np.uint32))
+
+
+def test_index_topk_shares_with_keys_in_workspace(csa):
+    # 8 decode queries over a cache sized above 16 x 32,768 entries: the workspace holds
+    # every order key, eight 16-CTA clusters do not fit at once, so the per-share kernel
+    # keeps its keys there and selects through a histogram (short ragged caches: shares
+    # with no entries, ragged tails; one query with zero weights ties every score)
+    B, Q, m = 8, 1, 1
+    cap = 524288 + 128
+    n_entries = [30000, 1, 129, 5000, 45000, 20000, 7, 44000]
+    q_pos = [[n - 1] for n in n_entries]
+    q_pos[4] = [40000]
+    grp, o, iq, iqs, w, oiq, oiqs, ow, qp = _index_case(171, B, Q, cap, n_entries, m, q_pos, 512, rows=45056)
+    w[5] = 0.0
+    ow = np_(w)
+    assert csa.csa2_workspace_bytes(csa.OP_INDEX_TOPK, B, Q, cap, 512, 0) >= B * cap * 4   # the keys' space
+    for k in (512, 2048):
+        idx, bm = csa.csa2_index_topk(iq, iqs, w, grp.kv, qp, k, blockmax=True)
+        ridx, rbm = oracle.index_topk(oiq, oiqs, ow, o["ik"], o["iks"], grp.n_entries, m, np.array(q_pos, np.int32),
+                                      k, blockmax=True)
+        assert np.array_equal(np_(idx), ridx), k
+        assert np.array_equal(np_(bm).view(np.uint32), rbm.view(np.uint32)), k
 
 
 def test_index_topk_many_queries_threshold_bin_overflow(csa):
