@@ -88,8 +88,10 @@ def job_value(world, ms_max):
 
 
 def _kernel_hash():
+    """The index kernel's translation unit: index_cluster.cu and every header it includes."""
     h = hashlib.sha256()
-    for f in ("index_cluster.cu", "index_pipe.cuh", "index_tc.cu", "tc.cuh", "common.cuh", "cluster.cuh", "kernels.h"):
+    for f in ("index_cluster.cu", "cluster.cuh", "index_pipe.cuh", "common.cuh", "kernels.h", "host_util.h", "tc.cuh",
+              os.path.join("..", "..", "include", "csa2.h")):
         with open(os.path.join(ROOT, "sparse_attention_fp4_quant_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
