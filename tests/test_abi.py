@@ -53,6 +53,14 @@ def test_workspace_sizes_are_host_only(L):
     assert L.csa2_workspace_bytes(csa.OP_INDEX_TOPK, 4, 128, 262144, 512, 0) >= 512 * 262144 * 2 + 512 * 2048 * 4
     # beyond that the path is not taken, and nothing is reserved for it
     assert L.csa2_workspace_bytes(csa.OP_INDEX_TOPK, 1, 4096, 524288, 512, 0) < 4096 * 524288 * 2
+    # a layer whose Reindex runs one CTA per query also keeps the pool search's order keys:
+    # 4 B per pool entry, the pool's slots rounded up to whole 128-entry tiles
+    for P in (2048, 300):
+        layer = L.csa2_workspace_bytes(csa.OP_LAYER, 2, 80, 30080, 512, P)
+        pool = L.csa2_workspace_bytes(csa.OP_POOL_TOPK, 2, 80, 30080, 512, P)
+        assert layer >= pool + 160 * ((P + 15) // 16) * 128 * 4
+    # a decode group above 16 x 32,768 entries keeps the index's order keys (4 B per entry)
+    assert L.csa2_workspace_bytes(csa.OP_INDEX_TOPK, 8, 1, 1048576, 512, 0) >= 8 * 1048576 * 4
 
 
 def test_invalid_arguments_rejected_before_launch(L):
