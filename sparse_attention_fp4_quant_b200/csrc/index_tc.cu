@@ -124,7 +124,7 @@ __device__ __forceinline__ void keys_select(TcSmem<CAP>& s, TopK<kEpiN, CAP, 1, 
     const uint32_t d = s.sel_bin;
     const bool fast = s.sel_count <= (uint32_t)CAP;
     tk.init();
-    constexpr int kBatch = 4;   // rounds of 4 keys a thread whose loads are in flight together
+    constexpr int kBatch = 8;   // rounds of 4 keys a thread whose loads are in flight together
     for (int base = 0; base < n_items; base += kBatch * 4 * kEpiN) {   // uniform trip count
         uint4 kv[kBatch];
 #pragma unroll
@@ -156,7 +156,7 @@ template <int CAP>
 __device__ __forceinline__ void merge_shares(TcSmem<CAP>& s, TopK<kEpiN, CAP, 1, kEpiT0>& tk, const uint32_t* keys,
                                              const int32_t* poss, int total, int k, int lane, int warp) {
     using TKE = TopK<kEpiN, CAP, 1, kEpiT0>;
-    constexpr int kB = 8;
+    constexpr int kB = 16;
     const int et = (int)threadIdx.x - kEpiT0;
     const uint32_t hist_base = tc::smem_u32(&s.hist[0]);
     for (int i = et; i < kHistBins; i += kEpiN) shm::st(hist_base + 4u * (uint32_t)i, 0u);
