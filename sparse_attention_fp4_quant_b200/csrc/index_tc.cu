@@ -1,16 +1,18 @@
 // index_tc.cu -- FP4 index scoring on the tcgen05 tensor cores (index_pipe.cuh),
-// fused with an exact Top-K (Full layers: csa2_index_topk when the query count
-// is too large for one cluster per query; Reindex layers: csa2_pool_topk, and
+// fused with an exact Top-K (Full layers: csa2_index_topk for shapes the cluster
+// and many-query kernels do not take; Reindex layers: csa2_pool_topk, and
 // csa2_layer_step's Reindex for many queries).
 //
 // One CTA = one share of one query's candidates.  Warps 0 and 1 run the
 // scoring pipeline; warps 2-9 finish the scores and select (named barrier 1).
-// Modes 0 and 1 stream the scores through a threshold filter into a buffer
-// that an exact radix select compacts; the last CTA of a query merges the
-// shares.  Mode 2 (an ascending pool, one CTA per query) keeps every order key
-// in the workspace and counts its top 11 bits while scoring, then offers only
-// the entries at or above the bin that holds the k-th key to the exact Top-K:
-// no per-stage barrier, and typically no compaction before the last.
+// Modes 0 and 1 (dense range, pool) stream the scores through a threshold
+// filter into a buffer that an exact radix select compacts.  Modes 2 (an
+// ascending pool, one CTA per query) and 3 (dense range) keep every order key
+// in the workspace and count its top 11 bits while scoring, then offer only the
+// items at or above the bin that holds the k-th key to the exact Top-K: no
+// per-stage barrier, and typically no compaction before the last.  With several
+// shares the last CTA of a query merges their best k through a histogram of all
+// their keys.
 #include "index_pipe.cuh"
 #include "topk.cuh"
 
