@@ -578,9 +578,12 @@ class LayerStack:
                                  blockmax=self.bm if self.bm is not None else False, ws=self.ws)
 
     def launches(self):
+        # the many-query index (more than 148 queries, at least 8 per batch row, at most 262,144
+        # entries) is two kernels, scoring then selection; the other index paths are one
+        mq = self.B * self.Q > 148 and self.Q >= 8 and self.cap <= 262144
         n = 1 if self.append else 0
         for mode in self.pattern:
-            n += {"full": 3 + (1 if self.pool is not None else 0), "reindex": 3, "reuse": 1}[mode]
+            n += {"full": (4 if mq else 3) + (1 if self.pool is not None else 0), "reindex": 3, "reuse": 1}[mode]
         return n
 
 
